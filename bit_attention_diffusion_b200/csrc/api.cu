@@ -1,0 +1,450 @@
+// api.cu - the C ABI of libvcattn (declared in include/vc_attn.h): argument
+// validation, workspace layout, TMA tensor maps and kernel launches.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "attn_bf16.cuh"
+#include "attn_fp8.cuh"
+#include "common.cuh"
+#include "prologue.cuh"
+
+namespace vc {
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+Shape make_shape(int B, int H, int N, const vc_params &p, int R) {
+  Shape s{};
+  s.B = B;
+  s.H = H;
+  s.N = N;
+  s.BH = B * H;
+  s.Nb = (N + TILE - 1) / TILE;
+  s.Npad = s.Nb * TILE;
+  s.k = p.k;
+  s.iters = p.iters;
+  s.R = R;
+  s.Rpad = R > 0 ? ((R + 127) / 128) * 128 : 0;
+  s.nch32 = (s.Nb + CHUNK32 - 1) / CHUNK32;
+  const int target = std::max(1, (4 * 148 + s.BH - 1) / s.BH);  // k-means blocks per (b,h)
+  s.km_cpb = std::max(1, (s.Nb + target - 1) / target);
+  s.km_nblk = (s.Nb + s.km_cpb - 1) / s.km_cpb;
+  s.kb_nchunk = std::max(1, std::min(s.Nb, (2 * 148 + s.BH - 1) / s.BH));
+  s.flags = p.flags;
+  return s;
+}
+
+WsLayout make_layout(const Shape &s) {
+  WsLayout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + std::max<size_t>(bytes, 1));
+    return at;
+  };
+  const size_t BH = static_cast<size_t>(s.BH), N = static_cast<size_t>(s.N), Nb = static_cast<size_t>(s.Nb),
+               Npad = static_cast<size_t>(s.Npad), k = static_cast<size_t>(s.k);
+  L.status = take(256);
+  L.km_counter = take(BH * 4);
+  L.vq_counter = take(BH * 4);
+  L.perm = take(BH * N * 4);
+  L.labels = take(BH * N * 4);
+  L.cent = take(BH * k * D * 4);
+  L.km_psum = take(BH * s.km_nblk * k * D * 8);
+  L.km_pcnt = take(BH * s.km_nblk * k * 4);
+  L.kbar_part = take(BH * s.kb_nchunk * D * 8);
+  L.kbar = take(BH * D * 4);
+  L.q8 = take(BH * Npad * D);
+  L.sq = take(BH * Nb * 4);
+  L.k8 = take(BH * Npad * D);
+  L.sk = take(BH * Nb * 4);
+  L.v8t = take(BH * D * Npad);
+  L.vscale = take(BH * D * 4);
+  L.vexpo = take(BH * D * 4);
+  L.vmean = take(BH * Nb * D * 2);
+  L.amax_part = take(BH * Nb * D * 4);
+  L.mut2 = take(BH * s.nch32 * D * 64 * 2);
+  L.err = take(BH * N * 4);
+  L.rep_idx = take(BH * std::max(s.R, 1) * 4);
+  L.rep_delta = take(BH * std::max(s.R, 1) * D * 2);
+  L.deltat = take(BH * D * std::max(s.Rpad, 1) * 2);
+  L.total = o;
+  return L;
+}
+
+}  // namespace vc
+
+using namespace vc;
+
+// ====================================================================== helpers
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major [outer][inner] array, 128-byte swizzle.
+bool map2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, uint64_t inner, uint64_t outer,
+           uint32_t box_in, uint32_t box_out) {
+  EncodeTiledFn f = encoder();
+  if (!f) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * static_cast<uint64_t>(esize)};
+  cuuint32_t box[2] = {box_in, box_out};
+  cuuint32_t es[2] = {1, 1};
+  return f(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// 3-D map over bf16 [BH][N][128] with boxes of 64 channels x 128 rows x 1 head
+// (rows past N read as zero).
+bool map3d_bf16(CUtensorMap *m, const void *base, int N, int BH) {
+  EncodeTiledFn f = encoder();
+  if (!f) return false;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(N) * 256};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+vc_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VC_ERR_CUDA;
+  static int ok_cache[64];  // 0 unknown, 1 ok, 2 unsupported
+  if (dev < 0 || dev >= 64) return VC_ERR_UNSUPPORTED;
+  if (ok_cache[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return VC_ERR_CUDA;
+    ok_cache[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    if (ok_cache[dev] == 1) {
+      if (cudaFuncSetAttribute(k_vc_attn_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(attn_fp8_smem_bytes())) != cudaSuccess ||
+          cudaFuncSetAttribute(k_attn_ref_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(attn_bf16_smem_bytes())) != cudaSuccess ||
+          cudaFuncSetAttribute(k_kmeans_pass, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               KMEANS_SMEM_FIXED + 64 * D * 12) != cudaSuccess ||
+          cudaFuncSetAttribute(k_quantv_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, QUANTV2_SMEM) !=
+              cudaSuccess) {
+        ok_cache[dev] = 0;
+        return VC_ERR_CUDA;
+      }
+    }
+  }
+  return ok_cache[dev] == 1 ? VC_OK : VC_ERR_UNSUPPORTED;
+}
+
+vc_status check_params(const vc_params *p) {
+  if (!p) return VC_ERR_INVALID_ARG;
+  if (p->k < 1 || p->k > 64 || p->iters < 0 || p->iters > 64) return VC_ERR_INVALID_ARG;
+  if (!(p->rho >= 0.0f && p->rho < 1.0f)) return VC_ERR_INVALID_ARG;
+  if (!(p->softmax_scale >= 0.0f) || !std::isfinite(p->softmax_scale)) return VC_ERR_INVALID_ARG;
+  if (p->expcast_bias < 8 || p->expcast_bias > 126) return VC_ERR_INVALID_ARG;
+  if (p->flags & ~(VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH)) return VC_ERR_INVALID_ARG;
+  return VC_OK;
+}
+
+vc_status check_shape(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1) return VC_ERR_INVALID_ARG;
+  if (d != 128) return VC_ERR_UNSUPPORTED;
+  const long long Npad = ((static_cast<long long>(N) + 127) / 128) * 128;
+  const long long elems = static_cast<long long>(B) * H * Npad * d;
+  if (elems >= (1ll << 31)) return VC_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 65535) return VC_ERR_INVALID_ARG;  // grid.y
+  return VC_OK;
+}
+
+struct Ws {
+  uint8_t *base;
+  WsLayout L;
+  template <class T>
+  T *at(size_t off) const { return reinterpret_cast<T *>(base + off); }
+};
+
+vc_status prep(int B, int H, int N, int d, const vc_params *p, void *ws, size_t ws_bytes, Shape *sh, Ws *w) {
+  vc_status st = check_shape(B, H, N, d);
+  if (st != VC_OK) return st;
+  if ((st = check_params(p)) != VC_OK) return st;
+  if (!ws || !aligned(ws, 256)) return VC_ERR_INVALID_ARG;
+  *sh = make_shape(B, H, N, *p, vc_attn_repair_count(N, p));
+  w->base = static_cast<uint8_t *>(ws);
+  w->L = make_layout(*sh);
+  if (ws_bytes < w->L.total) return VC_ERR_WORKSPACE;
+  return VC_OK;
+}
+
+vc_status last_error() { return cudaGetLastError() == cudaSuccess ? VC_OK : VC_ERR_CUDA; }
+
+// Clear the completion counters and the status word at the start of a call.
+vc_status clear_small(const Ws &w, cudaStream_t s) {
+  // status, km_counter and vq_counter are the first three regions of the layout
+  if (cudaMemsetAsync(w.base, 0, w.L.perm, s) != cudaSuccess) return VC_ERR_CUDA;
+  return VC_OK;
+}
+
+void launch_cluster(const Shape &sh, const Ws &w, const uint16_t *V, int32_t *perm, float *cent, cudaStream_t s) {
+  int32_t *labels = w.at<int32_t>(w.L.labels);
+  k_kmeans_init<<<sh.BH, 128, 0, s>>>(V, sh.N, sh.k, cent);
+  count_launch();
+  const size_t smem = KMEANS_SMEM_FIXED + static_cast<size_t>(sh.k) * D * 12;
+  const dim3 grid(sh.km_nblk, sh.BH);
+  for (int it = 0; it <= sh.iters; ++it) {
+    k_kmeans_pass<<<grid, 128, smem, s>>>(V, sh.N, sh.k, sh.km_cpb, sh.km_nblk, cent, labels,
+                                          w.at<double>(w.L.km_psum), w.at<int>(w.L.km_pcnt),
+                                          w.at<unsigned>(w.L.km_counter), it < sh.iters ? 1 : 0);
+    count_launch();
+  }
+  k_perm_sort<<<sh.BH, 1024, 0, s>>>(labels, sh.N, sh.k, perm);
+  count_launch();
+}
+
+void launch_quant_qk(const Shape &sh, const Ws &w, const uint16_t *Q, const uint16_t *K, const int32_t *perm,
+                     uint8_t *q8, float *sq, uint8_t *k8, float *sk, cudaStream_t s) {
+  const int ks = (sh.flags & VC_KSMOOTH) ? 1 : 0;
+  double *part = w.at<double>(w.L.kbar_part);
+  float *kbar = w.at<float>(w.L.kbar);
+  if (ks) {
+    k_kbar_partial<<<dim3(sh.kb_nchunk, sh.BH), 128, 0, s>>>(K, sh.N, sh.kb_nchunk, part);
+    count_launch();
+  }
+  k_kbar_final<<<sh.BH, 128, 0, s>>>(part, sh.N, ks ? sh.kb_nchunk : 0, ks, kbar);
+  count_launch();
+  k_qk_quant<<<dim3(sh.Nb, sh.BH, 2), 256, 0, s>>>(Q, K, perm, kbar, sh.N, sh.Npad, q8, sq, k8, sk);
+  count_launch();
+}
+
+void launch_quant_v(const Shape &sh, const Ws &w, const uint16_t *V, const int32_t *perm, uint8_t *v8t,
+                    float *vscale, uint16_t *vmean, int32_t *rep_idx, uint16_t *rep_delta, cudaStream_t s) {
+  const int demean = (sh.flags & VC_VSMOOTH) ? 1 : 0;
+  int *vexpo = w.at<int>(w.L.vexpo);
+  k_quantv_pass1<<<dim3(sh.Nb, sh.BH), 128, 0, s>>>(V, perm, sh.N, sh.Nb, demean, vmean,
+                                                     w.at<float>(w.L.amax_part), vscale, vexpo,
+                                                     w.at<unsigned>(w.L.vq_counter));
+  count_launch();
+  k_quantv_pass2<<<dim3(sh.Nb, sh.BH), 128, QUANTV2_SMEM, s>>>(V, perm, sh.N, sh.Nb, sh.Npad, sh.nch32, vmean, vscale, vexpo,
+                                                     v8t, w.at<float>(w.L.err), w.at<uint16_t>(w.L.mut2));
+  count_launch();
+  if (sh.R > 0) {
+    k_repair_select<<<sh.BH, 1024, 0, s>>>(w.at<float>(w.L.err), sh.N, sh.R, rep_idx);
+    count_launch();
+    k_repair_delta<<<dim3((sh.Rpad + 7) / 8, sh.BH), 256, 0, s>>>(V, perm, sh.N, sh.Nb, sh.R, sh.Rpad, rep_idx,
+                                                                  vmean, vscale, vexpo, rep_delta,
+                                                                  w.at<uint16_t>(w.L.deltat));
+    count_launch();
+  }
+}
+
+float kappa_of(float softmax_scale) {
+  return static_cast<float>(8.0 * 1.4426950408889634074 * static_cast<double>(softmax_scale));
+}
+float scale_or_default(float s) { return s > 0.0f ? s : static_cast<float>(1.0 / std::sqrt(128.0)); }
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+void vc_params_default(vc_params *p) {
+  if (!p) return;
+  p->k = 8;
+  p->iters = 3;
+  p->rho = 0.005f;
+  p->softmax_scale = 0.0f;
+  p->expcast_bias = 120;
+  p->flags = VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH;
+}
+
+const char *vc_status_str(vc_status s) {
+  switch (s) {
+    case VC_OK: return "ok";
+    case VC_ERR_INVALID_ARG: return "invalid argument";
+    case VC_ERR_UNSUPPORTED: return "unsupported (d must be 128; device must be compute capability 10.0)";
+    case VC_ERR_WORKSPACE: return "workspace too small";
+    case VC_ERR_CUDA: return "CUDA runtime error";
+    case VC_ERR_TIMEOUT: return "a bounded device wait ran out";
+  }
+  return "unknown status";
+}
+
+int vc_attn_repair_count(int N, const vc_params *p) {
+  if (!p || !(p->flags & VC_REPAIR) || N < 1) return 0;
+  double r = std::ceil(static_cast<double>(p->rho) * static_cast<double>(N));
+  if (r < 0) r = 0;
+  if (r > N) r = N;
+  return static_cast<int>(r);
+}
+
+size_t vc_attn_workspace_bytes(int B, int H, int N, int d, const vc_params *p) {
+  if (check_shape(B, H, N, d) != VC_OK || check_params(p) != VC_OK) return 0;
+  return make_layout(make_shape(B, H, N, *p, vc_attn_repair_count(N, p))).total;
+}
+
+vc_status vc_attn_cluster(const void *V, int B, int H, int N, int d, const vc_params *p, int32_t *perm,
+                          float *centroids, void *ws, size_t ws_bytes, void *stream) {
+  Shape sh;
+  Ws w;
+  vc_status st = prep(B, H, N, d, p, ws, ws_bytes, &sh, &w);
+  if (st != VC_OK) return st;
+  if (!V || !perm || !aligned(V, 16) || !aligned(perm, 16) || (centroids && !aligned(centroids, 16)))
+    return VC_ERR_INVALID_ARG;
+  if ((st = check_device()) != VC_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = clear_small(w, s)) != VC_OK) return st;
+  launch_cluster(sh, w, static_cast<const uint16_t *>(V), perm, centroids ? centroids : w.at<float>(w.L.cent), s);
+  return last_error();
+}
+
+vc_status vc_attn_quant_qk(const void *Q, const void *K, const int32_t *perm, int B, int H, int N, int d,
+                           const vc_params *p, uint8_t *q8, float *sq, uint8_t *k8, float *sk, void *ws,
+                           size_t ws_bytes, void *stream) {
+  Shape sh;
+  Ws w;
+  vc_status st = prep(B, H, N, d, p, ws, ws_bytes, &sh, &w);
+  if (st != VC_OK) return st;
+  if (!Q || !K || !q8 || !sq || !k8 || !sk || !aligned(Q, 16) || !aligned(K, 16) || !aligned(q8, 16) ||
+      !aligned(k8, 16) || !aligned(sq, 4) || !aligned(sk, 4) || (perm && !aligned(perm, 4)))
+    return VC_ERR_INVALID_ARG;
+  if ((st = check_device()) != VC_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = clear_small(w, s)) != VC_OK) return st;
+  launch_quant_qk(sh, w, static_cast<const uint16_t *>(Q), static_cast<const uint16_t *>(K), perm, q8, sq, k8, sk, s);
+  return last_error();
+}
+
+vc_status vc_attn_quant_v(const void *V, const int32_t *perm, int B, int H, int N, int d, const vc_params *p,
+                          uint8_t *v8, float *v_scale, void *v_mean, int32_t *rep_idx, void *rep_delta, void *ws,
+                          size_t ws_bytes, void *stream) {
+  Shape sh;
+  Ws w;
+  vc_status st = prep(B, H, N, d, p, ws, ws_bytes, &sh, &w);
+  if (st != VC_OK) return st;
+  if (!V || !v8 || !v_scale || !v_mean || !aligned(V, 16) || !aligned(v8, 16) || !aligned(v_scale, 4) ||
+      !aligned(v_mean, 4) || (perm && !aligned(perm, 4)))
+    return VC_ERR_INVALID_ARG;
+  if (sh.R > 0 && (!rep_idx || !rep_delta || !aligned(rep_idx, 4) || !aligned(rep_delta, 8)))
+    return VC_ERR_INVALID_ARG;
+  if ((st = check_device()) != VC_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = clear_small(w, s)) != VC_OK) return st;
+  launch_quant_v(sh, w, static_cast<const uint16_t *>(V), perm, v8, v_scale, static_cast<uint16_t *>(v_mean),
+                 rep_idx, static_cast<uint16_t *>(rep_delta), s);
+  return last_error();
+}
+
+vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H, int N, int d, const int32_t *perm,
+                      const vc_params *p, void *O, void *ws, size_t ws_bytes, void *stream) {
+  Shape sh;
+  Ws w;
+  vc_status st = prep(B, H, N, d, p, ws, ws_bytes, &sh, &w);
+  if (st != VC_OK) return st;
+  if (!Q || !K || !V || !O || !aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) ||
+      (perm && !aligned(perm, 4)))
+    return VC_ERR_INVALID_ARG;
+  if ((st = check_device()) != VC_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint16_t *Qh = static_cast<const uint16_t *>(Q), *Kh = static_cast<const uint16_t *>(K),
+                 *Vh = static_cast<const uint16_t *>(V);
+  if ((st = clear_small(w, s)) != VC_OK) return st;
+  const int32_t *pm = perm;
+  if (!pm && (sh.flags & VC_VSMOOTH)) {
+    launch_cluster(sh, w, Vh, w.at<int32_t>(w.L.perm), w.at<float>(w.L.cent), s);
+    pm = w.at<int32_t>(w.L.perm);
+  }
+  uint8_t *q8 = w.at<uint8_t>(w.L.q8), *k8 = w.at<uint8_t>(w.L.k8), *v8t = w.at<uint8_t>(w.L.v8t);
+  float *sq = w.at<float>(w.L.sq), *sk = w.at<float>(w.L.sk), *vscale = w.at<float>(w.L.vscale);
+  int32_t *rep_idx = w.at<int32_t>(w.L.rep_idx);
+  launch_quant_qk(sh, w, Qh, Kh, pm, q8, sq, k8, sk, s);
+  launch_quant_v(sh, w, Vh, pm, v8t, vscale, w.at<uint16_t>(w.L.vmean), rep_idx, w.at<uint16_t>(w.L.rep_delta), s);
+
+  CUtensorMap tq, tk, tv, tmu, tdt;
+  const uint64_t rows = static_cast<uint64_t>(sh.BH) * sh.Npad;
+  bool ok = map2d(&tq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, rows, 128, 128) &&
+            map2d(&tk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, rows, 128, 128) &&
+            map2d(&tv, v8t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, sh.Npad, static_cast<uint64_t>(sh.BH) * 128, 128, 128) &&
+            map2d(&tmu, w.at<uint16_t>(w.L.mut2), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64,
+                  static_cast<uint64_t>(sh.BH) * sh.nch32 * 128, 64, 128);
+  if (ok) {
+    if (sh.R > 0)
+      ok = map2d(&tdt, w.at<uint16_t>(w.L.deltat), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sh.Rpad,
+                 static_cast<uint64_t>(sh.BH) * 128, 64, 128);
+    else
+      tdt = tmu;  // unused when R == 0
+  }
+  if (!ok) return VC_ERR_CUDA;
+  AttnFp8Params ap{};
+  ap.N = sh.N;
+  ap.Nb = sh.Nb;
+  ap.Npad = sh.Npad;
+  ap.nch32 = sh.nch32;
+  ap.R = sh.R;
+  ap.Rpad = sh.Rpad;
+  ap.C = p->expcast_bias;
+  ap.kappa = kappa_of(scale_or_default(p->softmax_scale));
+  ap.sq = sq;
+  ap.sk = sk;
+  ap.vscale = vscale;
+  ap.rep_idx = rep_idx;
+  ap.k8 = k8;
+  ap.O = static_cast<uint16_t *>(O);
+  ap.status = w.at<uint32_t>(w.L.status);
+  k_vc_attn_fwd<<<dim3(sh.Nb, sh.BH), 192, attn_fp8_smem_bytes(), s>>>(tq, tk, tv, tmu, tdt, ap);
+  count_launch();
+  return last_error();
+}
+
+vc_status vc_attn_fwd_ref_bf16(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
+                               float softmax_scale, void *O, void *stream) {
+  vc_status st = check_shape(B, H, N, d);
+  if (st != VC_OK) return st;
+  if (!(softmax_scale >= 0.0f) || !std::isfinite(softmax_scale)) return VC_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !O || !aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16))
+    return VC_ERR_INVALID_ARG;
+  if ((st = check_device()) != VC_OK) return st;
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv;
+  if (!map3d_bf16(&tq, Q, N, BH) || !map3d_bf16(&tk, K, N, BH) || !map3d_bf16(&tv, V, N, BH)) return VC_ERR_CUDA;
+  AttnBf16Params ap{};
+  ap.N = N;
+  ap.Nb = (N + 127) / 128;
+  ap.scale_log2 = static_cast<float>(static_cast<double>(scale_or_default(softmax_scale)) * 1.4426950408889634074);
+  ap.O = static_cast<uint16_t *>(O);
+  ap.status = nullptr;  // no workspace here: a timeout shows as a wrong result only
+  k_attn_ref_bf16<<<dim3(ap.Nb, BH), 192, attn_bf16_smem_bytes(), static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, ap);
+  count_launch();
+  return last_error();
+}
+
+vc_status vc_attn_device_status(void *ws, void *stream) {
+  if (!ws || !aligned(ws, 256)) return VC_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return VC_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return VC_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return VC_ERR_CUDA;
+  return (v & ST_TIMEOUT) ? VC_ERR_TIMEOUT : VC_OK;
+}
+
+unsigned long long vc_attn_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,496 @@
+// attn_fp8.cu - the fused VC-Attention FP8 forward kernel for sm_100a.
+//
+// Page "VC-Attention acelera atenção em modelos de vídeo de IA em até 3,58× sem
+// retreinamento": low-bit tensor cores for both products QK^T and PV ("Por que
+// a atenção é o gargalo"); the value block mean is restored through the row sum
+// the online softmax keeps ("V-Smooth: corrigindo outliers de valor", item
+// Restore); the probability byte is written from the log-domain score by one
+// fused multiply-add ("ExpCast-FP8: eliminando o gargalo do softmax"). Page
+// "VC-Attention et FLUX 3 accélèrent la génération d'images sur Blackwell",
+// "Le compromis entre vitesse et fidélité": repair of the worst tokens.
+//
+// One CTA per (128-query tile, b*h). Warp roles:
+//   warp 0   TMA producer: Q once; K8 / V8 tiles through 3-stage rings; the
+//            bf16 block-mean tiles (one per 32 KV tiles); repair deltas.
+//   warp 1   allocates TMEM; lane 0 issues every tcgen05.mma and commit.
+//   warps 2-5  one thread per query row: online max, frames, ExpCast bytes,
+//            O rescale, row-sum bookkeeping, restore operands, repair, epilogue.
+// TMEM (512 columns x 128 lanes): S double buffer at columns [0,128) and
+// [128,256); the O accumulator at [256,384) followed by the row-sum columns
+// [384,400): the PV MMA uses N = 144 with a ones row appended to every V tile,
+// so column 384 receives l_t = sum_j p_ij of the decoded bytes of tile t.
+// O is kept in "code units": O_acc = sum p * code + sum_t l_t * mean_t/s + sum_R
+// p * delta/s, and the epilogue writes O = s_c * O_acc / l.
+#include "common.cuh"
+#include "sm100.cuh"
+#include "attn_fp8.cuh"
+#include "expcast.cuh"
+
+namespace vc {
+
+namespace {
+
+constexpr int KS = 3;  // K ring stages
+constexpr int VS = 3;  // V ring stages
+constexpr uint32_t SZ_TILE8 = 128 * 128;         // one 128x128 byte tile
+constexpr uint32_t SZ_VSTAGE = SZ_TILE8 + 2048;  // + 16 ones/zero rows
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = OFF_Q + SZ_TILE8;
+constexpr uint32_t OFF_V = OFF_K + KS * SZ_TILE8;
+constexpr uint32_t OFF_P = OFF_V + VS * SZ_VSTAGE;
+constexpr uint32_t OFF_AR = OFF_P + 2 * SZ_TILE8;
+constexpr uint32_t OFF_MU = OFF_AR + SZ_TILE8;
+constexpr uint32_t OFF_LB = OFF_MU + 2 * SZ_TILE8;
+constexpr uint32_t SMEM_USED = OFF_LB + 32 * 128 * 4;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // alignment slack
+static_assert(OFF_P % 1024 == 0 && OFF_AR % 1024 == 0 && OFF_MU % 1024 == 0, "tile alignment");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_L = 384;
+constexpr uint32_t IDESC_QK = idesc_make(0, 0, 128, 128, false, false);   // E4M3 x E4M3 -> f32
+constexpr uint32_t IDESC_PV = idesc_make(0, 0, 128, 144, false, false);   // + row-sum columns
+constexpr uint32_t IDESC_BF = idesc_make(1, 1, 128, 128, false, false);   // bf16 x bf16 -> f32
+
+struct Bars {
+  uint64_t q, kfull[KS], kempty[KS], vfull[VS], vempty[VS], mufull[2], muempty[2];
+  uint64_t sfull[2], pfull[2], pvdone, main, epi, repk, reps, repp, repdone, dt, fin;
+};
+
+__device__ __forceinline__ uint64_t desc128(const uint8_t *p) { return sdesc_sw128(smem_u32(p), 16, 1024); }
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+}  // namespace
+
+__global__ void __launch_bounds__(192, 1)
+    k_vc_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmMu,
+                  const __grid_constant__ CUtensorMap tmDT, const AttnFp8Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sQ = sm + OFF_Q;
+  uint8_t *sK = sm + OFF_K;
+  uint8_t *sV = sm + OFF_V;
+  uint8_t *sP = sm + OFF_P;
+  uint8_t *sAr = sm + OFF_AR;
+  uint8_t *sMu = sm + OFF_MU;
+  float *sLb = reinterpret_cast<float *>(sm + OFF_LB);  // [32 slots][128 rows]
+  __shared__ Bars bars;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+  __shared__ float s_vscale[128];
+  __shared__ float s_alphaR[128];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, bh = blockIdx.y;
+  const int T = p.Nb;
+  const int nrc = (p.R + 127) / 128;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    mbar_init(&bars.q, 1);
+    for (int i = 0; i < KS; ++i) { mbar_init(&bars.kfull[i], 1); mbar_init(&bars.kempty[i], 1); }
+    for (int i = 0; i < VS; ++i) { mbar_init(&bars.vfull[i], 1); mbar_init(&bars.vempty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.mufull[i], 1); mbar_init(&bars.muempty[i], 1);
+      mbar_init(&bars.sfull[i], 1); mbar_init(&bars.pfull[i], 128);
+    }
+    mbar_init(&bars.pvdone, 1); mbar_init(&bars.main, 1); mbar_init(&bars.epi, 128);
+    mbar_init(&bars.repk, 128); mbar_init(&bars.reps, 1); mbar_init(&bars.repp, 128);
+    mbar_init(&bars.repdone, 1); mbar_init(&bars.dt, 1); mbar_init(&bars.fin, 1);
+    fence_mbar_init();
+  }
+  if (warp >= 2) {
+    const int t = threadIdx.x - 64;  // 0..127
+    // ones rows appended to every V stage: row 128 is 1.0 (0x38) in every byte,
+    // rows 129..143 are zero (K-major, 128-byte swizzle, rows 128.. of the tile)
+    for (int i = t; i < VS * 16 * 8; i += 128) {
+      const int st = i / 128, rr = 128 + (i % 128) / 8, ch = i % 8;
+      const uint32_t v = rr == 128 ? 0x38383838u : 0u;
+      *reinterpret_cast<uint4 *>(sV + st * SZ_VSTAGE + sw128_off(rr, ch)) = make_uint4(v, v, v, v);
+    }
+    s_vscale[t] = p.vscale[static_cast<size_t>(bh) * 128 + t];
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) tmem_alloc(&s_tmem, 512);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  auto fail = [&]() {
+    s_abort = 1;
+    atomicOr(p.status, ST_TIMEOUT);
+  };
+  auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+    if (s_abort) return false;
+    if (!mbar_wait(bar, parity)) {
+      fail();
+      return false;
+    }
+    return true;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmMu);
+      mbar_arrive_expect_tx(&bars.q, SZ_TILE8);
+      tma_load_2d(sQ, &tmQ, &bars.q, 0, bh * p.Npad + qt * 128);
+      bool ok = true;
+      for (int t = 0; t < T && ok; ++t) {
+        if ((t & 31) == 0) {
+          const int X = t >> 5, s = X & 1;
+          ok = wait(&bars.muempty[s], ((X >> 1) & 1) ^ 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bars.mufull[s], SZ_TILE8);
+          tma_load_2d(sMu + s * SZ_TILE8, &tmMu, &bars.mufull[s], 0, (bh * p.nch32 + X) * 128);
+        }
+        const int s = t % KS;
+        const uint32_t ph = (t / KS) & 1;
+        ok = wait(&bars.kempty[s], ph ^ 1);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bars.kfull[s], SZ_TILE8);
+        tma_load_2d(sK + s * SZ_TILE8, &tmK, &bars.kfull[s], 0, bh * p.Npad + t * 128);
+        ok = wait(&bars.vempty[s], ph ^ 1);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bars.vfull[s], SZ_TILE8);
+        tma_load_2d(sV + s * SZ_VSTAGE, &tmV, &bars.vfull[s], t * 128, bh * 128);
+      }
+      if (ok && nrc > 0) {
+        ok = wait(&bars.main, 0);
+        for (int rc = 0; rc < nrc && ok; ++rc) {
+          if (rc > 0) ok = wait(&bars.repdone, (rc - 1) & 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bars.dt, 2 * SZ_TILE8);
+          tma_load_2d(sK, &tmDT, &bars.dt, rc * 128, bh * 128);
+          tma_load_2d(sK + SZ_TILE8, &tmDT, &bars.dt, rc * 128 + 64, bh * 128);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = wait(&bars.q, 0);
+      tc_fence_after();
+      auto issue_qk = [&](int t) -> bool {
+        const int s = t % KS;
+        if (!wait(&bars.kfull[s], (t / KS) & 1)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + TM_S0 + (t & 1) * 128;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f8_ss(d, desc128(sQ + 32 * kk), desc128(sK + s * SZ_TILE8 + 32 * kk), IDESC_QK, kk > 0);
+        mma_commit(&bars.kempty[s]);
+        mma_commit(&bars.sfull[t & 1]);
+        return true;
+      };
+      auto issue_restore = [&](int X) -> bool {
+        const int s = X & 1;
+        if (!wait(&bars.mufull[s], (X >> 1) & 1)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16_ss(tmem + TM_O, desc128(sAr + 32 * kk), desc128(sMu + s * SZ_TILE8 + 32 * kk), IDESC_BF, 1);
+        mma_commit(&bars.muempty[s]);
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      if (ok && T > 1) ok = issue_qk(1);
+      for (int t = 0; t < T && ok; ++t) {
+        ok = wait(&bars.pfull[t & 1], (t >> 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (t > 0 && (t & 31) == 0) {
+          ok = issue_restore((t >> 5) - 1);
+          if (!ok) break;
+        }
+        const int s = t % KS;
+        ok = wait(&bars.vfull[s], (t / KS) & 1);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f8_ss(tmem + TM_O, desc128(sP + (t & 1) * SZ_TILE8 + 32 * kk), desc128(sV + s * SZ_VSTAGE + 32 * kk),
+                    IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars.vempty[s]);
+        mma_commit(&bars.pvdone);
+        if (t + 2 < T) ok = issue_qk(t + 2);
+      }
+      if (ok) mma_commit(&bars.main);
+      if (ok) ok = wait(&bars.epi, 0);
+      if (ok) {
+        tc_fence_after();
+        ok = issue_restore((T - 1) >> 5);
+      }
+      for (int rc = 0; rc < nrc && ok; ++rc) {
+        ok = wait(&bars.repk, rc & 1);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f8_ss(tmem + TM_S0, desc128(sQ + 32 * kk), desc128(sV + 32 * kk), IDESC_QK, kk > 0);
+        mma_commit(&bars.reps);
+        ok = wait(&bars.repp, rc & 1) && wait(&bars.dt, rc & 1);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_f16_ss(tmem + TM_O, desc128(sP + (kk >> 2) * SZ_TILE8 + 32 * (kk & 3)),
+                     desc128(sK + (kk >> 2) * SZ_TILE8 + 32 * (kk & 3)), IDESC_BF, 1);
+        mma_commit(&bars.repdone);
+      }
+      if (ok) mma_commit(&bars.fin);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax rows
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const float sqs = p.sq[static_cast<size_t>(bh) * T + qt];
+    const float *skh = p.sk + static_cast<size_t>(bh) * T;
+    const int tail = p.N - (T - 1) * 128;  // valid keys in the last tile
+    float m = -INFINITY, F = -INFINITY, ltot = 0.0f;
+    bool ok = true;
+    // every lane waits; the outcome is made warp-uniform so that the
+    // .sync.aligned TMEM instructions below always see the whole warp
+    auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
+      const bool w = wait(bar, parity);
+      return __all_sync(0xFFFFFFFFu, w);
+    };
+
+    auto flush = [&](int nvalid) {
+      // A operand of the restore MMA: row r = [hi(l_0..l_31) | lo(l_0..l_31)] in bf16
+      uint32_t hw[16], lw[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float l0 = (2 * i < nvalid) ? sLb[(2 * i) * 128 + r] : 0.0f;
+        float l1 = (2 * i + 1 < nvalid) ? sLb[(2 * i + 1) * 128 + r] : 0.0f;
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(l0), h1 = __float2bfloat16_rn(l1);
+        const __nv_bfloat16 o0 = __float2bfloat16_rn(__fsub_rn(l0, __bfloat162float(h0)));
+        const __nv_bfloat16 o1 = __float2bfloat16_rn(__fsub_rn(l1, __bfloat162float(h1)));
+        hw[i] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+        lw[i] = static_cast<uint32_t>(__bfloat16_as_ushort(o0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(o1)) << 16);
+      }
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        *reinterpret_cast<uint4 *>(sAr + sw128_off(r, ch)) =
+            make_uint4(hw[4 * ch], hw[4 * ch + 1], hw[4 * ch + 2], hw[4 * ch + 3]);
+        *reinterpret_cast<uint4 *>(sAr + sw128_off(r, ch + 4)) =
+            make_uint4(lw[4 * ch], lw[4 * ch + 1], lw[4 * ch + 2], lw[4 * ch + 3]);
+      }
+    };
+
+    for (int t = 0; t < T && ok; ++t) {
+      const int b = t & 1;
+      ok = wwait(&bars.sfull[b], (t >> 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t v[32];
+        tmem_ld32(trow + TM_S0 + b * 128 + 32 * i, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s[32 * i + j] = __uint_as_float(v[j]);
+      }
+      const bool last = (t == T - 1) && (tail < 128);
+      float mx;
+      {
+        float mm[43];
+        if (last) {
+#pragma unroll
+          for (int j = 0; j < 128; ++j)
+            if (j >= tail) s[j] = -INFINITY;
+        }
+#pragma unroll
+        for (int j = 0; j < 42; ++j) mm[j] = max3(s[3 * j], s[3 * j + 1], s[3 * j + 2]);
+        mm[42] = fmaxf(s[126], s[127]);
+#pragma unroll
+        for (int j = 0; j < 14; ++j) mm[j] = max3(mm[3 * j], mm[3 * j + 1], mm[3 * j + 2]);
+        mm[14] = mm[42];
+#pragma unroll
+        for (int j = 0; j < 5; ++j) mm[j] = max3(mm[3 * j], mm[3 * j + 1], mm[3 * j + 2]);
+        mx = max3(mm[0], mm[1], fmaxf(mm[2], fmaxf(mm[3], mm[4])));
+      }
+      const float alpha = __fmul_rn(__fmul_rn(sqs, skh[t]), p.kappa);
+      m = fmaxf(m, __fmul_rn(mx, alpha));
+      const float Fn = 8.0f * ceilf(m * 0.125f);
+      if (t > 0) {
+        ok = wwait(&bars.pvdone, (t - 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const float lprev = __uint_as_float(tmem_ld1(trow + TM_L));
+        tmem_wait_ld();
+        tmem_st1(trow + TM_L, 0u);
+        const int slot = (t - 1) & 31;
+        sLb[slot * 128 + r] = lprev;
+        ltot += lprev;
+        const bool need = Fn != F;
+        if (__any_sync(0xFFFFFFFFu, need)) {
+          const int kshift = need ? static_cast<int>((Fn - F) * 0.125f) : 0;
+          const float sc = kshift > 126 ? 0.0f : __uint_as_float(static_cast<uint32_t>(127 - kshift) << 23);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t v[32];
+            tmem_ld32(trow + TM_O + 32 * i, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * sc);
+            tmem_st32(trow + TM_O + 32 * i, v);
+          }
+          ltot *= sc;
+          for (int sl = 0; sl <= slot; ++sl) sLb[sl * 128 + r] *= sc;
+        }
+        if (slot == 31) flush(32);
+        tmem_wait_st();
+      }
+      F = Fn;
+      const float al24 = alpha * TWO_M24;
+      const float c24 = (static_cast<float>(p.C) - F) * TWO_M24;
+      uint8_t *prow = sP + b * SZ_TILE8;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) w[q] = expcast4(&s[16 * ch + 4 * q], al24, c24);
+        if (last) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int j0 = 16 * ch + 4 * q;
+            uint32_t keep = 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (j0 + e < tail) keep |= 0xFFu << (8 * e);
+            w[q] &= keep;
+          }
+        }
+        *reinterpret_cast<uint4 *>(prow + sw128_off(r, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars.pfull[b]);
+    }
+
+    // ---------------------------------------------------------- end of the KV loop
+    if (ok) ok = wwait(&bars.main, 0);
+    if (ok) {
+      tc_fence_after();
+      const float lprev = __uint_as_float(tmem_ld1(trow + TM_L));
+      tmem_wait_ld();
+      const int slot = (T - 1) & 31;
+      sLb[slot * 128 + r] = lprev;
+      ltot += lprev;
+      flush(slot + 1);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars.epi);
+    }
+    // ---------------------------------------------------------- repair
+    const float c24f = (static_cast<float>(p.C) - F) * TWO_M24;
+    for (int rc = 0; rc < nrc && ok; ++rc) {
+      if (rc > 0) {
+        ok = wwait(&bars.repdone, (rc - 1) & 1);
+        if (!ok) break;
+      }
+      const int i = rc * 128 + r;
+      const int nval = min(128, p.R - rc * 128);
+      uint4 krow[8];
+      float al = 0.0f;
+      if (i < p.R) {
+        const int pos = p.rep_idx[static_cast<size_t>(bh) * p.R + i];
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.k8 + (static_cast<size_t>(bh) * p.Npad + pos) * 128);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) krow[ch] = src[ch];
+        al = __fmul_rn(__fmul_rn(sqs, skh[pos >> 7]), p.kappa);
+      } else {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) krow[ch] = make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4 *>(sV + sw128_off(r, ch)) = krow[ch];
+      s_alphaR[r] = al * TWO_M24;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars.repk);
+      softmax_bar();  // s_alphaR visible to every row
+      ok = wwait(&bars.reps, rc & 1);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t v[32];
+        tmem_ld32(trow + TM_S0 + 32 * q, v);
+        tmem_wait_ld();
+        // 32 scores -> 32 bf16 probabilities (two 16-byte chunks per 8 values)
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t outw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 32 * q + 8 * g + 2 * e;
+            const uint32_t h = expcast2(__uint_as_float(v[8 * g + 2 * e]), __uint_as_float(v[8 * g + 2 * e + 1]),
+                                        s_alphaR[j], s_alphaR[j + 1], c24f);
+            uint32_t b0 = h & 0xFFu, b1 = (h >> 16) & 0xFFu;
+            if (j >= nval) b0 = 0u;
+            if (j + 1 >= nval) b1 = 0u;
+            const float2 pv = e4m3x2_value(static_cast<uint16_t>(b0 | (b1 << 8)));
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(pv.x, pv.y);
+            outw[e] = *reinterpret_cast<const uint32_t *>(&pb);
+          }
+          const int jj = 32 * q + 8 * g;  // first key of this 16-byte chunk
+          *reinterpret_cast<uint4 *>(sP + (jj >> 6) * SZ_TILE8 + sw128_off(r, (jj & 63) >> 3)) =
+              make_uint4(outw[0], outw[1], outw[2], outw[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars.repp);
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok) ok = wwait(&bars.fin, 0);
+    if (ok) {
+      tc_fence_after();
+      const int row = qt * 128 + r;
+      uint16_t *orow = p.O + (static_cast<size_t>(bh) * p.N + row) * 128;
+      const float inv_ok = ltot;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t v[32];
+        tmem_ld32(trow + TM_O + 32 * i, v);
+        tmem_wait_ld();
+        if (row < p.N) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = 32 * i + 8 * g + 2 * e;
+              const float o0 = __fdiv_rn(__uint_as_float(v[8 * g + 2 * e]) * s_vscale[c], inv_ok);
+              const float o1 = __fdiv_rn(__uint_as_float(v[8 * g + 2 * e + 1]) * s_vscale[c + 1], inv_ok);
+              const __nv_bfloat162 ob = __floats2bfloat162_rn(o0, o1);
+              w[e] = *reinterpret_cast<const uint32_t *>(&ob);
+            }
+            *reinterpret_cast<uint4 *>(orow + 32 * i + 8 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+uint32_t attn_fp8_smem_bytes() { return SMEM_BYTES; }
+
+}  // namespace vc

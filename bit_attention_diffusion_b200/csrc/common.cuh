@@ -1,0 +1,65 @@
+// common.cuh - workspace layout, launch bookkeeping and small numeric helpers
+// shared by the kernels of libvcattn.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include "../../include/vc_attn.h"
+
+namespace vc {
+
+constexpr int D = 128;      // head dimension
+constexpr int TILE = 128;   // hardware block: rows of Q, keys of K/V, tokens of V-Smooth
+constexpr int CHUNK32 = 32; // KV tiles whose block means are restored by one bf16 MMA
+
+// Device status bits (workspace word).
+constexpr uint32_t ST_TIMEOUT = 1u;
+
+struct Shape {
+  int B, H, N, BH, Nb, Npad, k, iters, R, Rpad, nch32;
+  int km_nblk;   // k-means blocks per (b,h)
+  int km_cpb;    // 128-token chunks per k-means block
+  int kb_nchunk; // K-mean partial chunks per (b,h)
+  unsigned flags;
+};
+
+// Byte offsets of the workspace arrays (all 256-byte aligned).
+struct WsLayout {
+  size_t perm, labels, cent, km_psum, km_pcnt, km_counter;
+  size_t kbar_part, kbar;
+  size_t q8, sq, k8, sk;
+  size_t v8t, vscale, vexpo, vmean, amax_part, vq_counter, mut2, err;
+  size_t rep_idx, rep_delta, deltat;
+  size_t status;
+  size_t total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+Shape make_shape(int B, int H, int N, const vc_params &p, int repair_count);
+WsLayout make_layout(const Shape &s);
+
+// Bookkeeping: every launch in the library goes through this counter.
+void count_launch();
+
+// ---------------------------------------------------------------- numerics
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+__device__ __forceinline__ uint16_t f32_to_bf16_rn(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+// Two floats -> two E4M3 codes (round to nearest even, saturating), lo in byte 0.
+__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+  return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+// Exact value of two E4M3 codes (lo byte, hi byte).
+__device__ __forceinline__ float2 e4m3x2_value(uint16_t codes) {
+  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes), __NV_E4M3);
+  return __half22float2(*reinterpret_cast<__half2 *>(&h));
+}
+
+}  // namespace vc

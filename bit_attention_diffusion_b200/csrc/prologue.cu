@@ -1,0 +1,545 @@
+// prologue.cu - the HBM-bound steps before the attention kernel:
+//   V-Smooth Group   k-means over value tokens + stable sort into the permutation
+//   Q/K smoothing    per-(b,h) channel mean of K, 8-bit block quantization of Q, K'
+//   V-Smooth Demean  block means, per-channel power-of-two residual scale,
+//                    E4M3 residual codes (channel-major), token errors
+//   rho-repair       top-R tokens by error, bf16 correction of their residual
+// Sources: page "VC-Attention acelera atenção em modelos de vídeo de IA em até
+// 3,58× sem retreinamento", sections "V-Smooth: corrigindo outliers de valor"
+// (Group, Demean) and "Por que a atenção é o gargalo" (Q/K smoothing as prior
+// art); page "VC-Attention et FLUX 3 accélèrent la génération d'images sur
+// Blackwell", section "Le compromis entre vitesse et fidélité" (rho = 0.005).
+#include "common.cuh"
+#include "prologue.cuh"
+
+namespace vc {
+
+// ============================================================== k-means
+// Init c_j = V[floor(j*N/k)].
+__global__ void k_kmeans_init(const uint16_t *__restrict__ V, int N, int k, float *__restrict__ cent) {
+  const int bh = blockIdx.x;
+  for (int j = 0; j < k; ++j) {
+    const long long src = (static_cast<long long>(j) * N) / k;
+    cent[(static_cast<size_t>(bh) * k + j) * D + threadIdx.x] =
+        bf16_to_f32(V[(static_cast<size_t>(bh) * N + src) * D + threadIdx.x]);
+  }
+}
+
+// One Lloyd pass over `cpb` consecutive 128-token chunks per block: assign
+// labels (fp32 fma distances in channel order, ties to the lowest cluster) and,
+// when `accumulate`, the block's fp64 per-cluster sums; the last block of a
+// (b,h) reduces all blocks' sums in block order and writes the new centroids.
+constexpr int KM_ROW_WORDS = 66;  // 128 bf16 = 64 words, padded to 66 (bank spread)
+
+__global__ void __launch_bounds__(128) k_kmeans_pass(const uint16_t *__restrict__ V, int N, int k, int cpb,
+                                                     int nblk, float *__restrict__ cent,
+                                                     int32_t *__restrict__ labels, double *__restrict__ psum,
+                                                     int *__restrict__ pcnt, unsigned *__restrict__ counter,
+                                                     int accumulate) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint32_t *sv = reinterpret_cast<uint32_t *>(smem);                       // 128 x 66 words
+  float *scent = reinterpret_cast<float *>(smem + TILE * KM_ROW_WORDS * 4); // k x 128
+  double *ssum = reinterpret_cast<double *>(scent + k * D);                // k x 128
+  __shared__ int slab[TILE];
+  __shared__ int scnt[64];
+  __shared__ int s_last;
+
+  const int bh = blockIdx.y, blk = blockIdx.x, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const uint16_t *Vh = V + static_cast<size_t>(bh) * N * D;
+  float *cent_h = cent + static_cast<size_t>(bh) * k * D;
+
+  for (int i = tid; i < k * D; i += TILE) scent[i] = cent_h[i];
+  if (accumulate) {
+    for (int i = tid; i < k * D; i += TILE) ssum[i] = 0.0;
+    if (tid < 64) scnt[tid] = 0;
+  }
+  const int n_begin = blk * cpb * TILE;
+  const int n_end = min(N, n_begin + cpb * TILE);
+  for (int n0 = n_begin; n0 < n_end; n0 += TILE) {
+    const int cnt = min(TILE, n_end - n0);
+    __syncthreads();
+    // coalesced load of the chunk: a warp reads one 256-byte row, 8 bytes per lane
+    for (int r = warp; r < cnt; r += 4) {
+      const uint2 w = *reinterpret_cast<const uint2 *>(Vh + static_cast<size_t>(n0 + r) * D + 4 * lane);
+      sv[r * KM_ROW_WORDS + 2 * lane] = w.x;
+      sv[r * KM_ROW_WORDS + 2 * lane + 1] = w.y;
+    }
+    __syncthreads();
+    if (tid < cnt) {
+      const uint32_t *row = sv + tid * KM_ROW_WORDS;
+      int best = 0;
+      float bestd = 0.0f;
+      for (int j0 = 0; j0 < k; j0 += 8) {
+        float acc[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.0f;
+        for (int w = 0; w < 64; ++w) {
+          const uint32_t pr = row[w];
+          const float x0 = __uint_as_float(pr << 16), x1 = __uint_as_float(pr & 0xFFFF0000u);
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            if (j0 + jj < k) {
+              const float d0 = __fsub_rn(x0, scent[(j0 + jj) * D + 2 * w]);
+              acc[jj] = __fmaf_rn(d0, d0, acc[jj]);
+              const float d1 = __fsub_rn(x1, scent[(j0 + jj) * D + 2 * w + 1]);
+              acc[jj] = __fmaf_rn(d1, d1, acc[jj]);
+            }
+          }
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int j = j0 + jj;
+          if (j < k && (j == 0 || acc[jj] < bestd)) {
+            bestd = acc[jj];
+            best = j;
+          }
+        }
+      }
+      slab[tid] = best;
+      labels[static_cast<size_t>(bh) * N + n0 + tid] = best;
+    }
+    if (accumulate) {
+      __syncthreads();
+      // thread = channel: sums in token order, no write conflicts
+      const int c = tid;
+      const int wsel = c >> 1;
+      const bool hi = c & 1;
+      for (int r = 0; r < cnt; ++r) {
+        const uint32_t pr = sv[r * KM_ROW_WORDS + wsel];
+        const float x = hi ? __uint_as_float(pr & 0xFFFF0000u) : __uint_as_float(pr << 16);
+        ssum[slab[r] * D + c] += static_cast<double>(x);
+      }
+      if (tid == 0)
+        for (int r = 0; r < cnt; ++r) scnt[slab[r]] += 1;
+    }
+  }
+  if (!accumulate) return;
+  __syncthreads();
+  double *ps = psum + (static_cast<size_t>(bh) * nblk + blk) * k * D;
+  int *pc = pcnt + (static_cast<size_t>(bh) * nblk + blk) * k;
+  for (int i = tid; i < k * D; i += TILE) ps[i] = ssum[i];
+  if (tid < k) pc[tid] = scnt[tid];
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&counter[bh], 1u) == static_cast<unsigned>(nblk - 1));
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // last block of this (b,h): reduce in block order, new centroids
+  for (int j = 0; j < k; ++j) {
+    double s = 0.0;
+    long long n = 0;
+    for (int b = 0; b < nblk; ++b) {
+      s += __ldcg(psum + ((static_cast<size_t>(bh) * nblk + b) * k + j) * D + tid);
+      n += __ldcg(pcnt + (static_cast<size_t>(bh) * nblk + b) * k + j);
+    }
+    if (n > 0) cent_h[j * D + tid] = static_cast<float>(s / static_cast<double>(n));
+  }
+  if (tid == 0) counter[bh] = 0u;
+}
+
+// Stable counting sort of token indices by label, one block per (b,h): a
+// histogram gives each label's start; then rounds of 1024 tokens scatter in
+// order (rank among equal labels = earlier lanes of the warp + earlier warps).
+__global__ void __launch_bounds__(1024) k_perm_sort(const int32_t *__restrict__ labels, int N, int k,
+                                                    int32_t *__restrict__ perm) {
+  __shared__ int base[64];
+  __shared__ int tot[64];
+  __shared__ int wcnt[32][64];
+  const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int32_t *lab = labels + static_cast<size_t>(bh) * N;
+  int32_t *out = perm + static_cast<size_t>(bh) * N;
+  if (tid < 64) base[tid] = 0;
+  __syncthreads();
+  for (int n = tid; n < N; n += 1024) atomicAdd(&base[lab[n]], 1);
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int j = 0; j < k; ++j) {
+      const int c = base[j];
+      base[j] = run;
+      run += c;
+    }
+  }
+  for (int n0 = 0; n0 < N; n0 += 1024) {
+    for (int i = tid; i < 32 * 64; i += 1024) (&wcnt[0][0])[i] = 0;
+    __syncthreads();
+    const int n = n0 + tid;
+    const int L = n < N ? lab[n] : -1;
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, L);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (L >= 0 && rank == 0) wcnt[warp][L] = __popc(peers);
+    __syncthreads();
+    if (tid < k) {
+      int run = 0;
+      for (int w = 0; w < 32; ++w) {
+        const int c = wcnt[w][tid];
+        wcnt[w][tid] = run;
+        run += c;
+      }
+      tot[tid] = run;
+    }
+    __syncthreads();
+    if (L >= 0) out[base[L] + wcnt[warp][L] + rank] = n;
+    __syncthreads();
+    if (tid < k) base[tid] += tot[tid];
+  }
+}
+
+// ============================================================== Q/K smoothing + quantization
+// Partial fp64 channel sums of K over a row range (one block per (chunk, b,h)).
+__global__ void __launch_bounds__(128) k_kbar_partial(const uint16_t *__restrict__ K, int N, int nchunk,
+                                                      double *__restrict__ part) {
+  const int bh = blockIdx.y, ch = blockIdx.x, c = threadIdx.x;
+  const int rows = (N + nchunk - 1) / nchunk;
+  const int r0 = ch * rows, r1 = min(N, r0 + rows);
+  const uint16_t *Kh = K + static_cast<size_t>(bh) * N * D;
+  double s = 0.0;
+  for (int r = r0; r < r1; ++r) s += static_cast<double>(bf16_to_f32(Kh[static_cast<size_t>(r) * D + c]));
+  part[(static_cast<size_t>(bh) * nchunk + ch) * D + c] = s;
+}
+
+__global__ void __launch_bounds__(128) k_kbar_final(const double *__restrict__ part, int N, int nchunk,
+                                                    int ksmooth, float *__restrict__ kbar) {
+  const int bh = blockIdx.x, c = threadIdx.x;
+  double s = 0.0;
+  for (int ch = 0; ch < nchunk; ++ch) s += part[(static_cast<size_t>(bh) * nchunk + ch) * D + c];
+  kbar[static_cast<size_t>(bh) * D + c] = ksmooth ? static_cast<float>(s / static_cast<double>(N)) : 0.0f;
+}
+
+// Block quantization: z = 0 -> Q rows [128t, 128t+128) in original order;
+// z = 1 -> K rows perm[128t + r] minus the channel mean. scale = amax/448,
+// codes = E4M3(x * (448/amax)). 8 warps x 16 rows, 4 channels per lane.
+__global__ void __launch_bounds__(256) k_qk_quant(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
+                                                  const int32_t *__restrict__ perm, const float *__restrict__ kbar,
+                                                  int N, int Npad, uint8_t *__restrict__ q8, float *__restrict__ sq,
+                                                  uint8_t *__restrict__ k8, float *__restrict__ sk) {
+  __shared__ float wmax[8];
+  const int t = blockIdx.x, bh = blockIdx.y, z = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cnt = min(TILE, N - t * TILE);
+  const uint16_t *src = (z == 0 ? Q : K) + static_cast<size_t>(bh) * N * D;
+  float kb[4] = {0.f, 0.f, 0.f, 0.f};
+  if (z == 1) {
+    const float4 k4 = *reinterpret_cast<const float4 *>(kbar + static_cast<size_t>(bh) * D + 4 * lane);
+    kb[0] = k4.x; kb[1] = k4.y; kb[2] = k4.z; kb[3] = k4.w;
+  }
+  float x[16][4];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = warp * 16 + i;
+    if (r < cnt) {
+      const int p = t * TILE + r;
+      const int row = (z == 1 && perm != nullptr) ? perm[static_cast<size_t>(bh) * N + p] : p;
+      const uint2 w = *reinterpret_cast<const uint2 *>(src + static_cast<size_t>(row) * D + 4 * lane);
+      const float v[4] = {__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u),
+                          __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        x[i][e] = (z == 1) ? __fsub_rn(v[e], kb[e]) : v[e];
+        amax = fmaxf(amax, fabsf(x[i][e]));
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[i][e] = 0.0f;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if (lane == 0) wmax[warp] = amax;
+  __syncthreads();
+  amax = wmax[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, wmax[w]);
+  const float scale = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 448.0f);
+  const float mult = amax == 0.0f ? 0.0f : __fdiv_rn(448.0f, amax);
+  uint8_t *dst = (z == 0 ? q8 : k8) + (static_cast<size_t>(bh) * Npad + static_cast<size_t>(t) * TILE) * D;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = warp * 16 + i;
+    uint32_t packed = 0;
+    if (r < cnt) {
+      const uint32_t lo = e4m3x2(__fmul_rn(x[i][0], mult), __fmul_rn(x[i][1], mult));
+      const uint32_t hi = e4m3x2(__fmul_rn(x[i][2], mult), __fmul_rn(x[i][3], mult));
+      packed = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint32_t *>(dst + static_cast<size_t>(r) * D + 4 * lane) = packed;
+  }
+  if (tid == 0) (z == 0 ? sq : sk)[static_cast<size_t>(bh) * (Npad / TILE) + t] = scale;
+}
+
+// ============================================================== V demean + quantization
+constexpr int VQ_ROW_WORDS = 66;
+
+// Gather the block's rows (through perm) into shared memory, one warp per row.
+__device__ __forceinline__ void gather_rows(uint32_t *sv, const uint16_t *Vh, const int32_t *permh, int p0, int cnt) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
+  for (int r = warp; r < TILE; r += nw) {
+    uint2 w = make_uint2(0u, 0u);
+    if (r < cnt) {
+      const int row = permh ? permh[p0 + r] : p0 + r;
+      w = *reinterpret_cast<const uint2 *>(Vh + static_cast<size_t>(row) * D + 4 * lane);
+    }
+    sv[r * VQ_ROW_WORDS + 2 * lane] = w.x;
+    sv[r * VQ_ROW_WORDS + 2 * lane + 1] = w.y;
+  }
+}
+__device__ __forceinline__ float sv_get(const uint32_t *sv, int r, int c) {
+  const uint32_t w = sv[r * VQ_ROW_WORDS + (c >> 1)];
+  return (c & 1) ? __uint_as_float(w & 0xFFFF0000u) : __uint_as_float(w << 16);
+}
+
+// Pass 1: block means and per-block residual amax; the last block of a (b,h)
+// turns the channel amax into the power-of-two scale.
+__global__ void __launch_bounds__(128) k_quantv_pass1(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
+                                                      int N, int Nb, int demean, uint16_t *__restrict__ vmean,
+                                                      float *__restrict__ amax_part, float *__restrict__ vscale,
+                                                      int *__restrict__ vexpo, unsigned *__restrict__ counter) {
+  __shared__ uint32_t sv[TILE * VQ_ROW_WORDS];
+  __shared__ int s_last;
+  const int t = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+  const int p0 = t * TILE, cnt = min(TILE, N - p0);
+  gather_rows(sv, V + static_cast<size_t>(bh) * N * D, perm ? perm + static_cast<size_t>(bh) * N : nullptr, p0, cnt);
+  __syncthreads();
+  uint16_t mu = 0;
+  if (demean) {
+    double s = 0.0;
+    for (int r = 0; r < cnt; ++r) s += static_cast<double>(sv_get(sv, r, c));
+    mu = f32_to_bf16_rn(static_cast<float>(s / static_cast<double>(cnt)));
+  }
+  const float muf = bf16_to_f32(mu);
+  float amax = 0.0f;
+  for (int r = 0; r < cnt; ++r) amax = fmaxf(amax, fabsf(__fsub_rn(sv_get(sv, r, c), muf)));
+  vmean[(static_cast<size_t>(bh) * Nb + t) * D + c] = mu;
+  amax_part[(static_cast<size_t>(bh) * Nb + t) * D + c] = amax;
+  __threadfence();
+  __syncthreads();
+  if (c == 0) s_last = (atomicAdd(&counter[bh], 1u) == static_cast<unsigned>(Nb - 1));
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  float a = 0.0f;
+  for (int b = 0; b < Nb; ++b) a = fmaxf(a, __ldcg(amax_part + (static_cast<size_t>(bh) * Nb + b) * D + c));
+  int e = 0;
+  float s = 1.0f;
+  if (a > 0.0f) {
+    int E;
+    const float f = frexpf(a, &E);  // a = f * 2^E, f in [0.5, 1); 448 = 0.875 * 2^9
+    e = (f > 0.875f) ? E - 8 : E - 9;
+    s = ldexpf(1.0f, e);
+  }
+  vscale[static_cast<size_t>(bh) * D + c] = s;
+  vexpo[static_cast<size_t>(bh) * D + c] = e;
+  if (c == 0) counter[bh] = 0u;
+}
+
+// Pass 2: residual codes (written channel-major), per-token error, and the
+// bf16 block means pre-divided by the channel scale for the in-kernel restore
+// (mut2[bh][chunk][c][0..63]: slots 0..31 and 32..63 both hold tile
+// chunk*32 + slot; unused slots of the last chunk are zero).
+__global__ void __launch_bounds__(128) k_quantv_pass2(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
+                                                      int N, int Nb, int Npad, int nch32,
+                                                      const uint16_t *__restrict__ vmean,
+                                                      const float *__restrict__ vscale, const int *__restrict__ vexpo,
+                                                      uint8_t *__restrict__ v8t, float *__restrict__ err,
+                                                      uint16_t *__restrict__ mut2) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  uint32_t *sv = reinterpret_cast<uint32_t *>(dsm);          // TILE x VQ_ROW_WORDS words
+  uint8_t *codeT = dsm + TILE * VQ_ROW_WORDS * 4;              // D rows x 144 bytes
+  __shared__ float smu[D], smult[D], sscale[D];
+  const int t = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int p0 = t * TILE, cnt = min(TILE, N - p0);
+  gather_rows(sv, V + static_cast<size_t>(bh) * N * D, perm ? perm + static_cast<size_t>(bh) * N : nullptr, p0, cnt);
+  {
+    const int c = tid;
+    const uint16_t mu = vmean[(static_cast<size_t>(bh) * Nb + t) * D + c];
+    smu[c] = bf16_to_f32(mu);
+    const int e = vexpo[static_cast<size_t>(bh) * D + c];
+    smult[c] = ldexpf(1.0f, -e);
+    sscale[c] = vscale[static_cast<size_t>(bh) * D + c];
+    // block mean / scale for the restore MMA (exact: bf16 divided by a power of two)
+    const uint16_t ms = f32_to_bf16_rn(__fmul_rn(bf16_to_f32(mu), ldexpf(1.0f, -e)));
+    const int ch = t / CHUNK32, slot = t % CHUNK32;
+    uint16_t *m = mut2 + ((static_cast<size_t>(bh) * nch32 + ch) * D + c) * 64;
+    m[slot] = ms;
+    m[slot + 32] = ms;
+    if (t == Nb - 1)
+      for (int s2 = slot + 1; s2 < CHUNK32; ++s2) {
+        m[s2] = 0;
+        m[s2 + 32] = 0;
+      }
+  }
+  __syncthreads();
+  {
+    const int r = tid;
+    float acc = 0.0f;
+    for (int c = 0; c < D; c += 2) {
+      uint16_t codes = 0;
+      if (r < cnt) {
+        const float r0 = __fsub_rn(sv_get(sv, r, c), smu[c]);
+        const float r1 = __fsub_rn(sv_get(sv, r, c + 1), smu[c + 1]);
+        codes = e4m3x2(__fmul_rn(r0, smult[c]), __fmul_rn(r1, smult[c + 1]));
+        const float2 dq = e4m3x2_value(codes);
+        const float e0 = __fsub_rn(r0, __fmul_rn(dq.x, sscale[c]));
+        const float e1 = __fsub_rn(r1, __fmul_rn(dq.y, sscale[c + 1]));
+        acc = __fmaf_rn(e0, e0, acc);
+        acc = __fmaf_rn(e1, e1, acc);
+      }
+      codeT[c * 144 + r] = static_cast<uint8_t>(codes & 0xFF);
+      codeT[(c + 1) * 144 + r] = static_cast<uint8_t>(codes >> 8);
+    }
+    if (r < cnt) err[static_cast<size_t>(bh) * N + p0 + r] = acc;
+  }
+  __syncthreads();
+  {
+    const int c = tid;
+    uint8_t *dst = v8t + (static_cast<size_t>(bh) * D + c) * Npad + p0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      *reinterpret_cast<uint4 *>(dst + 16 * i) = *reinterpret_cast<const uint4 *>(codeT + c * 144 + 16 * i);
+  }
+}
+
+// ============================================================== repair selection
+// Top-R by error (float >= 0, so the bit pattern orders like the value), ties
+// to the lowest permuted position; output ascending. One block per (b,h):
+// radix select of the R-th largest key, then an ordered compaction.
+__global__ void __launch_bounds__(1024) k_repair_select(const float *__restrict__ err, int N, int R,
+                                                        int32_t *__restrict__ rep_idx) {
+  __shared__ unsigned hist[256];
+  __shared__ unsigned s_prefix, s_need;
+  __shared__ int wgt[32], weq[32];
+  __shared__ int s_base_gt, s_base_eq;
+  const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const unsigned *key = reinterpret_cast<const unsigned *>(err + static_cast<size_t>(bh) * N);
+  int32_t *out = rep_idx + static_cast<size_t>(bh) * R;
+  if (tid == 0) {
+    s_prefix = 0u;
+    s_need = static_cast<unsigned>(R);
+  }
+  unsigned mask = 0u;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    if (tid < 256) hist[tid] = 0u;
+    __syncthreads();
+    const unsigned prefix = s_prefix;
+    for (int n = tid; n < N; n += 1024) {
+      const unsigned kv = key[n];
+      if ((kv & mask) == prefix) atomicAdd(&hist[(kv >> shift) & 0xFFu], 1u);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      unsigned need = s_need, run = 0u;
+      int dsel = 0;
+      for (int dgt = 255; dgt >= 0; --dgt) {
+        if (run + hist[dgt] >= need) {
+          dsel = dgt;
+          break;
+        }
+        run += hist[dgt];
+      }
+      s_need = need - run;  // how many with exactly this digit prefix are still needed
+      s_prefix = prefix | (static_cast<unsigned>(dsel) << shift);
+    }
+    mask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  const unsigned T = s_prefix;   // the R-th largest key
+  const int need_eq = static_cast<int>(s_need);  // keys == T to take (lowest positions first)
+  if (tid == 0) {
+    s_base_gt = 0;
+    s_base_eq = 0;
+  }
+  __syncthreads();
+  for (int n0 = 0; n0 < N; n0 += 1024) {
+    const int n = n0 + tid;
+    const unsigned kv = n < N ? key[n] : 0u;
+    const bool gt = n < N && kv > T;
+    const bool eq = n < N && kv == T;
+    const unsigned bgt = __ballot_sync(0xFFFFFFFFu, gt), beq = __ballot_sync(0xFFFFFFFFu, eq);
+    if (lane == 0) {
+      wgt[warp] = __popc(bgt);
+      weq[warp] = __popc(beq);
+    }
+    __syncthreads();
+    int pre_gt = s_base_gt, pre_eq = s_base_eq;
+    for (int w = 0; w < warp; ++w) {
+      pre_gt += wgt[w];
+      pre_eq += weq[w];
+    }
+    const unsigned lt = (1u << lane) - 1u;
+    const int my_eq = pre_eq + __popc(beq & lt);
+    const bool take = gt || (eq && my_eq < need_eq);
+    // position in the ascending output = number of taken keys before n
+    const int taken_eq_before = min(my_eq, need_eq);
+    const int pos = pre_gt + __popc(bgt & lt) + taken_eq_before;
+    if (take) out[pos] = n;
+    __syncthreads();
+    if (tid == 0) {
+      int tg = 0, te = 0;
+      for (int w = 0; w < 32; ++w) {
+        tg += wgt[w];
+        te += weq[w];
+      }
+      s_base_gt += tg;
+      s_base_eq += te;
+    }
+    __syncthreads();
+  }
+}
+
+// delta = bf16(r - value(code)*scale) for every repaired token; also the
+// channel-major copy divided by the channel scale (deltat[bh][c][r], zero for
+// r in [R, Rpad)) that the attention kernel's repair MMA reads.
+__global__ void __launch_bounds__(256) k_repair_delta(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
+                                                      int N, int Nb, int R, int Rpad,
+                                                      const int32_t *__restrict__ rep_idx,
+                                                      const uint16_t *__restrict__ vmean,
+                                                      const float *__restrict__ vscale, const int *__restrict__ vexpo,
+                                                      uint16_t *__restrict__ rep_delta, uint16_t *__restrict__ deltat) {
+  const int bh = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + warp;
+  if (r >= Rpad) return;
+  if (r >= R) {
+    for (int i = 0; i < 4; ++i) deltat[(static_cast<size_t>(bh) * D + 4 * lane + i) * Rpad + r] = 0;
+    return;
+  }
+  const int p = rep_idx[static_cast<size_t>(bh) * R + r];
+  const int row = perm ? perm[static_cast<size_t>(bh) * N + p] : p;
+  const int t = p / TILE;
+  const uint2 w = *reinterpret_cast<const uint2 *>(V + (static_cast<size_t>(bh) * N + row) * D + 4 * lane);
+  const float v[4] = {__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u), __uint_as_float(w.y << 16),
+                      __uint_as_float(w.y & 0xFFFF0000u)};
+  float res[4], mult[4], sc[4];
+  for (int i = 0; i < 4; ++i) {
+    const int c = 4 * lane + i;
+    res[i] = __fsub_rn(v[i], bf16_to_f32(vmean[(static_cast<size_t>(bh) * Nb + t) * D + c]));
+    mult[i] = ldexpf(1.0f, -vexpo[static_cast<size_t>(bh) * D + c]);
+    sc[i] = vscale[static_cast<size_t>(bh) * D + c];
+  }
+  uint16_t dl[4];
+  for (int i = 0; i < 4; i += 2) {
+    const uint16_t codes = e4m3x2(__fmul_rn(res[i], mult[i]), __fmul_rn(res[i + 1], mult[i + 1]));
+    const float2 dq = e4m3x2_value(codes);
+    dl[i] = f32_to_bf16_rn(__fsub_rn(res[i], __fmul_rn(dq.x, sc[i])));
+    dl[i + 1] = f32_to_bf16_rn(__fsub_rn(res[i + 1], __fmul_rn(dq.y, sc[i + 1])));
+  }
+  uint2 o;
+  o.x = static_cast<uint32_t>(dl[0]) | (static_cast<uint32_t>(dl[1]) << 16);
+  o.y = static_cast<uint32_t>(dl[2]) | (static_cast<uint32_t>(dl[3]) << 16);
+  *reinterpret_cast<uint2 *>(rep_delta + (static_cast<size_t>(bh) * R + r) * D + 4 * lane) = o;
+  for (int i = 0; i < 4; ++i) {
+    const int c = 4 * lane + i;
+    deltat[(static_cast<size_t>(bh) * D + c) * Rpad + r] = f32_to_bf16_rn(__fmul_rn(bf16_to_f32(dl[i]), mult[i]));
+  }
+}
+
+// ============================================================== misc
+__global__ void k_identity_perm(int32_t *perm, int N, long long total) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < total) perm[i] = static_cast<int32_t>(i % N);
+}
+
+}  // namespace vc

@@ -1,0 +1,194 @@
+/*
+ * vc_attn.h - C ABI of libvcattn, VC-Attention FP8 for NVIDIA B200 (sm_100a).
+ *
+ * VC-Attention is a training-free, non-causal, quantized attention forward
+ * pass for diffusion transformers. Sources (web pages, by title and section):
+ *  [VCA]  "VC-Attention acelera atenção em modelos de vídeo de IA em até 3,58×
+ *         sem retreinamento": "Por que a atenção é o gargalo" (low-bit tensor
+ *         cores for QK^T and PV; Q/K smoothing is prior art), "V-Smooth:
+ *         corrigindo outliers de valor" (Group, Demean, Restore), "ExpCast-FP8:
+ *         eliminando o gargalo do softmax" (byte ~ 8*log2(p) + 56 by one FMA).
+ *  [IP73] "VC-Attention et FLUX 3 accélèrent la génération d'images sur
+ *         Blackwell", "Le compromis entre vitesse et fidélité" (repair budget
+ *         rho = 0.005 for the tokens with the largest quantization error).
+ *
+ * Conventions for every call:
+ *  - Tensors are dense, row-major, in device memory unless stated. Q, K, V
+ *    and O are bf16 [B, H, N, d] with d = 128 (any other d is
+ *    VC_ERR_UNSUPPORTED). Nb = ceil(N/128) blocks, Npad = 128*Nb.
+ *  - The caller owns and allocates every buffer, including the workspace
+ *    sized by vc_attn_workspace_bytes(); the library allocates nothing and
+ *    keeps no state between calls (the per-device tensor-map encoder entry
+ *    point is looked up once).
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *    asynchronous on it; argument errors are detected on the host before any
+ *    launch and nothing is launched then.
+ *  - Device pointers must be 16-byte aligned (TMA); the workspace 256-byte
+ *    aligned. B*H*Npad*d must be < 2^31.
+ *  - Inputs containing NaN/Inf give undefined (but bounded-time) results.
+ *  - Device-side waits are bounded; a wait that runs out sets a status word
+ *    in the workspace, read back with vc_attn_device_status().
+ */
+#ifndef VC_ATTN_H
+#define VC_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VC_OK = 0,
+  VC_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size or parameter */
+  VC_ERR_UNSUPPORTED = 2, /* d != 128, device not compute capability 10.0 */
+  VC_ERR_WORKSPACE = 3,   /* workspace smaller than vc_attn_workspace_bytes() */
+  VC_ERR_CUDA = 4,        /* a CUDA runtime call failed */
+  VC_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out */
+} vc_status;
+
+/* Method switches (vc_params.flags). */
+#define VC_VSMOOTH 1u /* V-Smooth: k-means grouping + block demean/restore */
+#define VC_REPAIR 2u  /* rho-repair of the worst-quantized value tokens */
+#define VC_KSMOOTH 8u /* subtract the per-(b,h) channel mean of K */
+
+typedef struct {
+  int k;             /* k-means clusters, 1..64 (default 8) */
+  int iters;         /* Lloyd iterations, 0..64 (default 3) */
+  float rho;         /* repair budget, [0, 1) (default 0.005); R = ceil(rho*N) */
+  float softmax_scale; /* 0 => 1/sqrt(d) */
+  int expcast_bias;  /* C: the running row maximum maps to byte C, 8..126 (default 120) */
+  unsigned flags;    /* VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH (default all) */
+} vc_params;
+
+/* Fill the defaults listed above. */
+void vc_params_default(vc_params *p);
+
+/* Human-readable name of a status code (static string). */
+const char *vc_status_str(vc_status s);
+
+/* Bytes of workspace vc_attn_fwd / vc_attn_cluster / vc_attn_quant_v need for
+ * this shape and these parameters (the largest of the three). 0 on bad args. */
+size_t vc_attn_workspace_bytes(int B, int H, int N, int d, const vc_params *p);
+
+/* Number of repair tokens per (b,h) for these parameters: ceil(rho*N) when
+ * VC_REPAIR is set, else 0 (rho*N evaluated in double from the float rho). */
+int vc_attn_repair_count(int N, const vc_params *p);
+
+/*
+ * V-Smooth Group ([VCA] "V-Smooth…", item Group): deterministic Lloyd k-means
+ * over the value tokens of every (b,h), then a stable sort of token indices by
+ * cluster label.
+ *   V        bf16 [B,H,N,d]                       in
+ *   perm     int32 [B,H,N] out: perm[p] = original index of the token at
+ *            permuted position p (K and V are both read through it)
+ *   centroids fp32 [B,H,k,d] out (final centroids), or NULL
+ * Init c_j = V[floor(j*N/k)]; distances are fp32, accumulated by fma in
+ * channel order; ties go to the lowest cluster; centroid = fp32(fp64 sum /
+ * count); an empty cluster keeps its centroid; `iters` rounds, then a final
+ * assignment. Bit-identical to the CPU oracle.
+ */
+vc_status vc_attn_cluster(const void *V, int B, int H, int N, int d, const vc_params *p, int32_t *perm,
+                          float *centroids, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Q/K smoothing + 8-bit quantization (prior art named in [VCA] "Por que a
+ * atenção é o gargalo"): K' = K - mean_n(K) per (b,h,channel) when
+ * VC_KSMOOTH is set; Q (original order) and K' (rows read through perm) are
+ * quantized per 128-row block to E4M3 with scale = amax/448.
+ *   Q, K  bf16 [B,H,N,d] in;  perm int32 [B,H,N] in (NULL = identity)
+ *   q8, k8 uint8 [B,H,Npad,d] out (E4M3 codes; padding rows are 0)
+ *   sq, sk fp32 [B,H,Nb] out (block scales)
+ */
+vc_status vc_attn_quant_qk(const void *Q, const void *K, const int32_t *perm, int B, int H, int N, int d,
+                           const vc_params *p, uint8_t *q8, float *sq, uint8_t *k8, float *sk, void *ws,
+                           size_t ws_bytes, void *stream);
+
+/*
+ * V-Smooth Demean + residual quantization ([VCA] "V-Smooth…", item Demean)
+ * and the rho-repair list ([IP73] "Le compromis…").
+ *   V           bf16 [B,H,N,d] in;  perm int32 [B,H,N] in (NULL = identity)
+ *   v8          uint8 [B,H,d,Npad] out: E4M3 residual codes, CHANNEL-MAJOR
+ *               (v8[b,h,c,p] is channel c of the token at permuted position
+ *               p); padding positions are 0
+ *   v_scale     fp32 [B,H,d] out: per-channel power-of-two scale, the least
+ *               2^e with max_p |r| <= 448 * 2^e (1 for an all-zero channel)
+ *   v_mean      bf16 [B,H,Nb,d] out: block means (0 without VC_VSMOOTH)
+ *   rep_idx     int32 [B,H,R] out: permuted positions of the R repaired
+ *               tokens, ascending (R = vc_attn_repair_count); may be NULL if R=0
+ *   rep_delta   bf16 [B,H,R,d] out: bf16(residual - dequantized code)
+ * Blocks are 128 consecutive permuted positions (tail block: the rest);
+ * mean = bf16(fp32(fp64 sum / count)); r = v - mean; code = E4M3(r * 2^-e);
+ * token error = sum_c (r - value(code)*scale)^2 (fp32, fma in channel order);
+ * the R largest errors are repaired (ties to the lowest position).
+ */
+vc_status vc_attn_quant_v(const void *V, const int32_t *perm, int B, int H, int N, int d, const vc_params *p,
+                          uint8_t *v8, float *v_scale, void *v_mean, int32_t *rep_idx, void *rep_delta,
+                          void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * The VC-Attention FP8 forward: O = attention(Q, K, V) for every (b,h).
+ *   Q, K, V  bf16 [B,H,N,d] in
+ *   perm     int32 [B,H,N] in, or NULL: cluster now when VC_VSMOOTH is set
+ *            (the pages run the grouping only in the first 25% of denoising
+ *            steps and reuse the permutation after), identity otherwise
+ *   O        bf16 [B,H,N,d] out, rows in the original query order
+ * Steps: K smoothing + Q/K quantization; V demean + per-channel E4M3
+ * residual + repair list; then one fused kernel per 128-query tile on the
+ * tcgen05 tensor cores: S = Q8 K8^T (FP8, fp32 in TMEM); online row max in
+ * "byte units" (8 * log2 of the probability) against the frame
+ * F = 8*ceil(max/8); ExpCast: byte = RNE(fp32(acc*alpha + C - F)) clamped at
+ * 0 - one fused multiply-add, no exponential; O += P V8 (FP8); the per-tile
+ * row sum l_t of the decoded bytes comes out of the same MMA (a ones column),
+ * and the block mean is restored as l_t * mean_t ([VCA] "V-Smooth…", item
+ * Restore) on the tensor cores in bf16; repair adds p * delta for the listed
+ * tokens; O = scale_c * acc / l.
+ */
+vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
+                      const int32_t *perm, const vc_params *p, void *O, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * In-library comparator: exact-softmax attention in BF16 on the tcgen05
+ * tensor cores (bf16 operands, fp32 accumulation, fp32 exp2 softmax).
+ * softmax_scale 0 => 1/sqrt(d). O bf16 [B,H,N,d].
+ */
+vc_status vc_attn_fwd_ref_bf16(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
+                               float softmax_scale, void *O, void *stream);
+
+/*
+ * ExpCast on the device, element-wise, exactly as the attention kernel
+ * computes it ([VCA] "ExpCast-FP8…"): out[i] = clamp(RNE(fp32(acc[i]*alpha[i]
+ * + c[i])), 0, ...) where the result must not exceed 126 (the kernel never
+ * produces more than C). n must be even; element pairs (2j, 2j+1) must share
+ * alpha and c (the kernel processes pairs). Device pointers.
+ */
+vc_status vc_attn_expcast(const float *acc, const float *alpha, const float *c, long long n, uint8_t *out,
+                          void *stream);
+
+/* Hardware E4M3 encoding (round to nearest even, saturating to +/-448) of n
+ * floats, as the quantization kernels use it. n even. Device pointers. */
+vc_status vc_attn_e4m3_encode(const float *x, long long n, uint8_t *out, void *stream);
+
+/* Read (synchronously, on `stream`) and clear the device status word kept in
+ * the workspace: VC_OK, or VC_ERR_TIMEOUT if a bounded device wait ran out.
+ * Every call that takes a workspace clears the word when it starts, so the
+ * word reports on the most recent such call. */
+vc_status vc_attn_device_status(void *ws, void *stream);
+
+/* Self test of the bounded device waits: launches one thread that waits on a
+ * barrier nothing arrives at, giving up after `limit_cycles` SM clock cycles
+ * (1 .. 2^32); it then records the timeout in the workspace status word the
+ * way the attention kernels do. Afterwards vc_attn_device_status(ws) returns
+ * VC_ERR_TIMEOUT. No GPU state is harmed; the kernel returns normally. */
+vc_status vc_attn_wait_selftest(void *ws, long long limit_cycles, void *stream);
+
+/* Number of kernels this library has launched in this process (for the
+ * bench's launch count). */
+unsigned long long vc_attn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VC_ATTN_H */

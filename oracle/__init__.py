@@ -77,6 +77,7 @@ def lib():
             L.orc_quant_v_head.argtypes = [P, P, i32, i32, i32, i32, P, P, P, P, P, P]
             L.orc_attn_vc_rows.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, f32, i32,
                                            P, i32, P, P, P]
+            L.orc_attn_exactv_rows.argtypes = [P, P, P, P, P, P, i32, i32, f32, i32, P, i32, P]
             L.orc_set_threads.argtypes = [i32]
             L.orc_get_threads.restype = i32
             L.orc_e4m3_encode_n.argtypes = [P, i64, P]
@@ -212,6 +213,21 @@ def attn_vc_rows(qk: dict, vq: dict, N: int, rows, softmax_scale: float = DEFAUL
                            int(N), d, float(kappa(softmax_scale)), int(C), _p(rows), rows.size,
                            _p(out), _p(out_l), _p(out_F))
     return out, out_l, out_F
+
+
+def attn_exactv_rows(qk: dict, v_bits, perm, N: int, rows, softmax_scale: float = DEFAULT_SCALE,
+                     C: int = DEFAULT_C):
+    """Diagnostic: the same probability bytes as the method, exact values.
+
+    ``out_method - out_exactv`` is the value-term error alone."""
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    v = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    pm = np.ascontiguousarray(perm, dtype=np.int32)
+    d = qk["q8"].shape[1]
+    out = np.empty((rows.size, d), np.float64)
+    lib().orc_attn_exactv_rows(_p(qk["q8"]), _p(qk["sq"]), _p(qk["k8"]), _p(qk["sk"]), _p(v), _p(pm), int(N), d,
+                               float(kappa(softmax_scale)), int(C), _p(rows), rows.size, _p(out))
+    return out
 
 
 # ---------------------------------------------------------------- whole path

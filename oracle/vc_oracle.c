@@ -286,6 +286,7 @@ void orc_quant_qk_head(const uint16_t *Q, const uint16_t *K, const int32_t *perm
  *   mu_t   = bf16(fp32(sum_fp64(v) / count))           (0 when demean is off)
  *   r      = fp32(v - mu_t)
  *   s_c    = 2^e_c, the least power of two with amax_c(r) <= 448 * 2^e_c [R]
+ *            (1 when every residual of the channel is zero)
  *   code   = E4M3(r * 2^-e_c)                           (exact scaling)
  *   err    = fp32(r - value(code) * s_c)
  *   e_p    = sum_c err^2, fmaf-accumulated in channel order from 0
@@ -295,8 +296,8 @@ static void pow2_scale(float amax, float *scale, int *expo)
 {
     int E;
     float f;
-    if (amax == 0.0f) {
-        *scale = 0.0f;
+    if (amax == 0.0f) {          /* all residuals zero: codes are 0, any scale works; take 1 */
+        *scale = 1.0f;
         *expo = 0;
         return;
     }
@@ -350,7 +351,7 @@ void orc_quant_v_head(const uint16_t *V, const int32_t *perm, int N, int d, int 
         float acc = 0.0f;
         for (int c = 0; c < d; ++c) {
             float r = res[(size_t)p * d + c];
-            uint8_t code = vscale[c] == 0.0f ? 0 : orc_e4m3_encode(ldexpf(r, -expo[c]));
+            uint8_t code = orc_e4m3_encode(ldexpf(r, -expo[c]));
             float deq = (float)(orc_e4m3_value(code) * (double)vscale[c]);
             float err = r - deq;
             v8[(size_t)p * d + c] = code;
@@ -492,6 +493,72 @@ void orc_attn_vc_rows(const uint8_t *q8, const float *sq, const uint8_t *k8, con
     free(kd);
     free(vd);
     free(mud);
+}
+
+/* Diagnostic (not a step of the method): the same online softmax and the same
+ * probability bytes as orc_attn_vc_rows, but the numerator uses the exact bf16
+ * values v_j (no quantization, no demean, no repair). The difference between
+ * the method's output and this one is the value-term error alone, which is the
+ * error V-Smooth and repair act on ([VCA] "Por que a atenção é o gargalo":
+ * after Q/K smoothing the value term dominates the output error). */
+void orc_attn_exactv_rows(const uint8_t *q8, const float *sq, const uint8_t *k8, const float *sk,
+                          const uint16_t *V, const int32_t *perm, int N, int d, float kappa, int C,
+                          const int32_t *rows, int nrows, double *out)
+{
+    int Nb = (N + TILE - 1) / TILE;
+    double *kd = (double *)malloc((size_t)N * d * sizeof(double));
+    double *vx = (double *)malloc((size_t)N * d * sizeof(double));
+    for (int j = 0; j < N; ++j)
+        for (int c = 0; c < d; ++c) {
+            kd[(size_t)j * d + c] = orc_e4m3_value(k8[(size_t)j * d + c]);
+            vx[(size_t)j * d + c] = (double)orc_bf16_value(V[(size_t)perm[j] * d + c]);
+        }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int ir = 0; ir < nrows; ++ir) {
+        int i = rows[ir];
+        double qd[TILE * 2];
+        double *num = (double *)calloc((size_t)d, sizeof(double));
+        float *acc = (float *)malloc((size_t)TILE * sizeof(float));
+        double l = 0.0;
+        float m = -INFINITY, F = -INFINITY;
+        float sqi = sq[i / TILE];
+        for (int c = 0; c < d; ++c)
+            qd[c] = orc_e4m3_value(q8[(size_t)i * d + c]);
+        for (int t = 0; t < Nb; ++t) {
+            int j0 = t * TILE, j1 = (j0 + TILE < N) ? j0 + TILE : N;
+            float alpha = (sqi * sk[t]) * kappa;
+            float Fnew;
+            for (int j = j0; j < j1; ++j) {
+                double s = 0.0;
+                for (int c = 0; c < d; ++c)
+                    s += qd[c] * kd[(size_t)j * d + c];
+                acc[j - j0] = (float)s;
+                float u = acc[j - j0] * alpha;
+                if (u > m)
+                    m = u;
+            }
+            Fnew = 8.0f * ceilf(m * 0.125f);
+            if (t > 0 && Fnew != F) {
+                double sc = ldexp(1.0, (int)((F - Fnew) / 8.0f));
+                for (int c = 0; c < d; ++c)
+                    num[c] *= sc;
+                l *= sc;
+            }
+            F = Fnew;
+            for (int j = j0; j < j1; ++j) {
+                double p = orc_e4m3_value((uint8_t)orc_expcast_byte(acc[j - j0], alpha, (float)C - F));
+                l += p;
+                for (int c = 0; c < d; ++c)
+                    num[c] += p * vx[(size_t)j * d + c];
+            }
+        }
+        for (int c = 0; c < d; ++c)
+            out[(size_t)ir * d + c] = num[c] / l;
+        free(num);
+        free(acc);
+    }
+    free(kd);
+    free(vx);
 }
 
 /* Thread control for the bench's CPU baseline (OpenMP over query rows). */

@@ -1,0 +1,106 @@
+"""CPU checks of the C-ABI boundary: the library loads, exports every function
+include/vc_attn.h declares, and rejects bad arguments on the host before any
+device work (these calls never reach a launch, so they run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_attention_diffusion_b200 import vcattn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "vc_attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(vc_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_attention_diffusion_b200 import build_lib
+    build_lib.build()
+    return vcattn.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert "vc_attn_fwd" in names and "vc_attn_cluster" in names and "vc_attn_quant_v" in names
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(vcattn.EXPORTED)
+
+
+def test_defaults_and_status_strings(L):
+    p = vcattn.params()
+    assert (p.k, p.iters, p.expcast_bias, p.flags) == (8, 3, 120, 11)
+    assert abs(p.rho - 0.005) < 1e-9
+    assert vcattn.status_str(0) == "ok"
+    assert "workspace" in vcattn.status_str(3)
+
+
+def test_repair_count_and_workspace_size(L):
+    p = vcattn.params()
+    assert [vcattn.vc_attn_repair_count(n, p) for n in (1024, 4256, 16544, 32928, 75600)] == \
+        [6, 22, 83, 165, 378]
+    assert vcattn.vc_attn_repair_count(1000, vcattn.params(flags=vcattn.VC_VSMOOTH)) == 0
+    ws = vcattn.vc_attn_workspace_bytes(1, 24, 16544, 128, p)
+    # at least the quantized Q, K, V (one byte per element) plus the permutation
+    assert ws >= 3 * 24 * 16640 * 128 + 24 * 16544 * 4
+    assert vcattn.vc_attn_workspace_bytes(1, 1, 100, 64, p) == 0
+    assert vcattn.vc_attn_workspace_bytes(1, 1, 0, 128, p) == 0
+
+
+FAKE = 1 << 20  # a 256-aligned non-null address; never dereferenced in these calls
+
+
+@pytest.mark.parametrize("case,status", [
+    (dict(d=64), vcattn.VC_ERR_UNSUPPORTED),
+    (dict(N=0), vcattn.VC_ERR_INVALID_ARG),
+    (dict(B=0), vcattn.VC_ERR_INVALID_ARG),
+    (dict(N=1 << 24, H=64), vcattn.VC_ERR_INVALID_ARG),      # B*H*Npad*d >= 2^31
+    (dict(ws=0), vcattn.VC_ERR_INVALID_ARG),
+    (dict(ws=FAKE + 16), vcattn.VC_ERR_INVALID_ARG),         # workspace not 256-aligned
+    (dict(ws_bytes=1024), vcattn.VC_ERR_WORKSPACE),
+    (dict(p=dict(k=0)), vcattn.VC_ERR_INVALID_ARG),
+    (dict(p=dict(k=65)), vcattn.VC_ERR_INVALID_ARG),
+    (dict(p=dict(rho=1.0)), vcattn.VC_ERR_INVALID_ARG),
+    (dict(p=dict(rho=-0.1)), vcattn.VC_ERR_INVALID_ARG),
+    (dict(p=dict(expcast_bias=127)), vcattn.VC_ERR_INVALID_ARG),
+    (dict(p=dict(flags=4)), vcattn.VC_ERR_INVALID_ARG),
+    (dict(p=dict(softmax_scale=-1.0)), vcattn.VC_ERR_INVALID_ARG),
+])
+def test_fwd_rejects_bad_arguments_on_host(L, case, status):
+    B, H, N, d = case.get("B", 1), case.get("H", 2), case.get("N", 256), case.get("d", 128)
+    p = vcattn.params(**case.get("p", {}))
+    ws = case.get("ws", FAKE)
+    ws_bytes = case.get("ws_bytes", 1 << 40)
+    st = vcattn.vc_attn_fwd(FAKE, FAKE, FAKE, B, H, N, d, None, p, FAKE, ws, ws_bytes, None)
+    assert st == status
+
+
+def test_ref_and_units_reject_bad_arguments_on_host(L):
+    assert vcattn.vc_attn_fwd_ref_bf16(FAKE, FAKE, FAKE, 1, 1, 128, 96, 0.0, FAKE, None) == vcattn.VC_ERR_UNSUPPORTED
+    assert vcattn.vc_attn_fwd_ref_bf16(FAKE + 8, FAKE, FAKE, 1, 1, 128, 128, 0.0, FAKE, None) == \
+        vcattn.VC_ERR_INVALID_ARG
+    assert vcattn.vc_attn_expcast(FAKE, FAKE, FAKE, 3, FAKE, None) == vcattn.VC_ERR_INVALID_ARG
+    assert vcattn.vc_attn_e4m3_encode(None, 4, FAKE, None) == vcattn.VC_ERR_INVALID_ARG
+    assert vcattn.vc_attn_wait_selftest(FAKE + 4, 100, None) == vcattn.VC_ERR_INVALID_ARG
+    assert vcattn.vc_attn_device_status(None, None) == vcattn.VC_ERR_INVALID_ARG
+    p = vcattn.params()
+    assert vcattn.vc_attn_cluster(FAKE, 1, 1, 256, 128, p, None, None, FAKE, 1 << 40, None) == \
+        vcattn.VC_ERR_INVALID_ARG
+    assert vcattn.vc_attn_quant_v(FAKE, None, 1, 1, 256, 128, p, FAKE, FAKE, FAKE, None, None, FAKE, 1 << 40,
+                                  None) == vcattn.VC_ERR_INVALID_ARG   # R > 0 needs rep_idx/rep_delta
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import importlib
+    mod = importlib.reload(vcattn)
+    monkeypatch.setattr(mod, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(mod, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        mod.lib()
+    importlib.reload(vcattn)

@@ -168,3 +168,16 @@ def test_random_inputs_error_band_vs_exact(orc):
     ex = orc.exact_attention_head(q, k, v, rows=rows)
     rel = np.linalg.norm(r["out"] - ex) / np.linalg.norm(ex)
     assert 0.02 < rel < 0.09, rel
+
+
+def test_exactv_diagnostic_equals_method_when_values_are_lossless(orc):
+    """The value-term diagnostic keeps the method's bytes and swaps in exact
+    values: in the lossless case (repair off, so the two off-grid tokens remain)
+    it differs from the method only by those tokens' residual error."""
+    q, k, v, perm, scale = _exact_case(orc, 25)
+    flags = orc.FLAG_VSMOOTH | orc.FLAG_REPAIR | orc.FLAG_KSMOOTH
+    r = orc.vc_attention_head(q, k, v, flags=flags, softmax_scale=scale, perm=perm)
+    ev = orc.attn_exactv_rows(r["qk"], v, r["perm"], 300, r["rows"], softmax_scale=scale)
+    assert np.allclose(ev, r["out"], rtol=1e-9, atol=1e-9)
+    r2 = orc.vc_attention_head(q, k, v, flags=flags & ~orc.FLAG_REPAIR, softmax_scale=scale, perm=perm)
+    assert not np.allclose(ev, r2["out"], rtol=1e-9, atol=1e-9)

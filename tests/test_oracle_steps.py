@@ -183,3 +183,16 @@ def test_kmeans_ties_go_to_lowest_cluster(orc):
     cent, lab = orc.kmeans_head(v, 8, 3)
     assert lab.tolist() == [0, 2, 4, 6]
     assert np.array_equal(orc.stable_sort_labels(lab, 8), np.arange(4))
+
+
+def test_quant_v_constant_channel_gets_unit_scale(orc):
+    """A channel whose residuals are all zero (constant within every block)
+    gets the power-of-two scale 1 and zero codes."""
+    rng = np.random.default_rng(20)
+    vf = rng.standard_normal((260, 128)).astype(np.float32)
+    vf[:, 7] = 3.0
+    v = synth.f32_to_bf16_bits(vf)
+    r = orc.quant_v_head(v, np.arange(260, dtype=np.int32), demean=True, R=0)
+    assert r["vscale"][7] == 1.0
+    assert np.all(r["v8"][:, 7] == 0)
+    assert np.all(orc.bf16_value(r["vmean"][:, 7]) == 3.0)

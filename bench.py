@@ -1,0 +1,409 @@
+#!/usr/bin/env python3
+"""Benchmark of the VC-Attention FP8 forward on B200.
+
+Workload: the 2048x2048 image-DiT joint-attention problem, B=1, H=24,
+N=16544 (16384 image + 160 text tokens), d=128, bf16 inputs drawn by
+bit_attention_diffusion_b200.synth (seeded synthetic data standing in for
+FLUX-3-style activations). One step = one vc_attn_fwd call over the whole hot
+path: V-Smooth clustering inside the call, Q/K smoothing + quantization, V
+demean + residual quantization + repair selection, and the fused FP8
+attention kernel. Metric: TFLOPS = 4*B*H*N^2*d / t (the pages' attention FLOP
+count), also as % of the measured FP8 dense peak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun: every rank owns one independent copy of the
+workload (heads are independent problems; no data-path collective), the step
+loop is bracketed by barriers and device syncs, times are CUDA-event device
+times and the job time is the max over ranks (weak scaling).
+
+--impl reference times the CPU oracle (oracle/, plain C + numpy) on the host
+cores on a bounded sample of the same workload, extrapolated to the metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "image2048_b1h24n16544"
+METRIC = "vc_attn_fwd TFLOPS (4N²dH/t) at N=16544,H=24,d=128; % of B200 FP8 peak"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [s for s, p in zip(sm, power) if p > 200] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(smax), "samples": len(sm),
+                "power_w_max": max(power), "reasons": sorted(reasons)}
+
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _to_dev(torch, bits):
+    import numpy as np
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def cpu_oracle_sample(wl, x, rows_per_head: int = 96, heads=(0,)):
+    """Time the oracle on a bounded sample and extrapolate to the workload.
+
+    For each sampled head: the full per-head prologue (k-means, quantization,
+    repair) plus `rows_per_head` query rows of the attention (all host cores).
+    Returns (TFLOPS extrapolated to the whole workload, cores, sample text,
+    seconds spent)."""
+    import numpy as np
+    import oracle
+    cores = oracle.set_threads(os.cpu_count() or 1)
+    t_pro = t_rows = 0.0
+    for h in heads:
+        q, k, v = x["q"][0, h], x["k"][0, h], x["v"][0, h]
+        t0 = time.perf_counter()
+        pro = oracle.head_prologue(q, k, v)
+        t1 = time.perf_counter()
+        rows = np.linspace(0, wl.N - 1, rows_per_head).astype(np.int32)
+        oracle.attn_vc_rows(pro["qk"], pro["vq"], wl.N, rows)
+        t2 = time.perf_counter()
+        t_pro += t1 - t0
+        t_rows += t2 - t1
+    nh = len(heads)
+    per_head = t_pro / nh + (t_rows / nh) * (wl.N / rows_per_head)
+    t_full = per_head * wl.B * wl.H
+    tflops = wl.flops / t_full / 1e12
+    sample = (f"{nh} head(s): full per-head prologue + {rows_per_head} of {wl.N} query rows each, "
+              f"extrapolated linearly in rows and heads to B={wl.B},H={wl.H} "
+              f"({t_pro + t_rows:.1f} s measured, {t_full:.0f} s extrapolated)")
+    return tflops, cores, sample, t_pro + t_rows
+
+
+def run_reference(args):
+    world, rank, _ = _dist_env()
+    if world > 1 and rank != 0:
+        return 0
+    from bit_attention_diffusion_b200 import synth
+    wl, x = synth.make_by_name(WORKLOAD)
+    vals = []
+    cores = 1
+    sample = ""
+    for i in range(args.warmup + args.steps):
+        tflops, cores, sample, secs = cpu_oracle_sample(wl, x, rows_per_head=16)
+        if i >= args.warmup:
+            vals.append(tflops)
+    v = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.flops / (v * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "B": wl.B, "H": wl.H, "N": wl.N, "d": 128},
+        "cpu_baseline": {"value": v, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------- GPU bench
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from bit_attention_diffusion_b200 import build_lib, synth, vcattn
+
+    world, rank, local = _dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    if rank == 0:
+        build_lib.build()
+    if world > 1:
+        dist.barrier()
+    vcattn.lib()
+    dev = torch.cuda.current_device()
+    stream = torch.cuda.current_stream()
+    sptr = stream.cuda_stream
+
+    wl, x = synth.make_by_name(WORKLOAD)
+    B, H, N, d = wl.B, wl.H, wl.N, 128
+    q, k, v = (_to_dev(torch, x[n]) for n in "qkv")
+    p = vcattn.params()
+    ws, ws_bytes = vcattn.workspace(B, H, N, p)
+    out = torch.empty_like(q)
+
+    def step(perm=None):
+        st = vcattn.vc_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d,
+                                None if perm is None else perm.data_ptr(), p, out.data_ptr(), ws.data_ptr(),
+                                ws_bytes, sptr)
+        if st != 0:
+            raise vcattn.VcError(st, "vc_attn_fwd")
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(val: float) -> float:
+        if world == 1:
+            return val
+        t = torch.tensor([val], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- main timed region: K full steps (clustering inside the call)
+    for _ in range(args.warmup):
+        step()
+    vcattn.vc_attn_profile(True)
+    barrier()
+    clocks = ClockSampler(dev)
+    clocks.start()
+    launches0 = vcattn.vc_attn_launch_count()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    launches = vcattn.vc_attn_launch_count() - launches0
+    clk = clocks.stop()
+    barrier()
+    ph_mean = vcattn.vc_attn_profile_read()  # mean over the timed steps (<= 64), read after the loop
+    vcattn.vc_attn_profile(False)
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_step = ms_total / args.steps
+    flops = wl.flops
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    if len(ph_mean) != 4:
+        ph_mean = [0.0, 0.0, 0.0, 0.0]
+    attn_ms = float(ph_mean[3])
+
+    if args.only_main:
+        if rank == 0:
+            print(json.dumps({"only_main": True, "ms_per_step": ms_step, "phases_ms": list(ph_mean),
+                              "gpu_launches": int(launches)}))
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
+
+    # ---- cached permutation (later denoising steps): clustering skipped
+    perm, _ = vcattn.cluster(v, p, ws=ws)
+    perm = perm.clone()
+    for _ in range(args.warmup):
+        step(perm)
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(perm)
+    e1.record(stream)
+    e1.synchronize()
+    ms_cached = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+
+    # ---- BF16 comparator kernel
+    for _ in range(args.warmup):
+        vcattn.fwd_ref_bf16(q, k, v, out=out)
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        vcattn.fwd_ref_bf16(q, k, v, out=out)
+    e1.record(stream)
+    e1.synchronize()
+    ms_ref = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+
+    # ---- end to end through the C ABI with host buffers
+    hq, hk, hv = (torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True) for _ in range(3))
+    for hbuf, n in zip((hq, hk, hv), "qkv"):
+        hbuf.copy_(torch.from_numpy(np.ascontiguousarray(x[n]).view(np.int16)).view(torch.bfloat16))
+    hout = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    e1.synchronize()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    bytes_in = 3 * q.numel() * 2
+    bytes_out = out.numel() * 2
+
+    peaks, peak_src = _peaks()
+    long_region = ms_total > 1000.0
+    bf16_peak = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops", FALLBACK_BF16_TFLOPS)
+    fp8_peak = 2.0 * bf16_peak  # dense FP8 = 2x dense BF16 (nominal ratio 4.5 : 2.25 PFLOP/s)
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12 if attn_ms > 0 else None
+    prof_path = os.path.join(ROOT, "profiles", "traffic.json")
+    traffic = None
+    try:
+        with open(prof_path) as f:
+            tj = json.load(f)
+        if tj.get("kernel_source_hash") == _kernel_hash():
+            traffic = tj.get("traffic_bytes_per_launch")
+    except Exception:
+        pass
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        tf, cores, sample, _ = cpu_oracle_sample(wl, x, rows_per_head=96)
+        cpu = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)", "data": "synthetic",
+            "pct_of_fp8_peak": 100.0 * (value / world) / fp8_peak,
+            "config": {"workload": WORKLOAD, "B": B, "H": H, "N": N, "d": d, "k": p.k, "iters": p.iters,
+                       "rho": round(p.rho, 6), "expcast_bias": p.expcast_bias,
+                       "step": "vc_attn_fwd with clustering in the call",
+                       "l2": "inputs larger than L2 (Q, K, V bf16 = 305 MB > 126 MB)",
+                       "parallelism": f"replicas x{world} (independent heads, no collective)"},
+            "phases_ms": {"cluster": float(ph_mean[0]), "quant_qk": float(ph_mean[1]),
+                          "quant_v_repair": float(ph_mean[2]), "attention": attn_ms},
+            "cached_perm": {"value": world * flops / (ms_cached * 1e-3) / 1e12, "unit": "TFLOPS",
+                            "ms_per_step": ms_cached},
+            "overhead_frac": {"with_clustering": (ms_step - attn_ms) / attn_ms if attn_ms else None,
+                              "cached_perm": (ms_cached - attn_ms) / attn_ms if attn_ms else None},
+            "ref_bf16": {"value": world * flops / (ms_ref * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms_ref,
+                         "pct_of_bf16_peak": 100.0 * (flops / (ms_ref * 1e-3) / 1e12) / bf16_peak},
+            "roofline": {"kernel": "k_vc_attn_fwd", "bound": "tensor", "achieved": attn_tflops,
+                         "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": (attn_tflops / fp8_peak) if attn_tflops else None,
+                         "traffic": traffic,
+                         "peak_source": f"{peak_src}: 2 x {'sustained' if long_region else 'burst'} "
+                                        f"cuBLAS bf16 ({bf16_peak:.1f} TFLOP/s)",
+                         "algorithmic": "4*B*H*N^2*d FLOP per launch"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms_e2e,
+                    "h2d_bytes_per_step": bytes_in, "d2h_bytes_per_step": bytes_out},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def _kernel_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("attn_fp8.cu", "attn_fp8.cuh", "expcast.cuh", "sm100.cuh"):
+        with open(os.path.join(ROOT, "bit_attention_diffusion_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    ap.add_argument("--only-main", action="store_true",
+                    help="warm-up + the timed main loop only (the small case profiler captures wrap)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -194,6 +194,21 @@ vc_status prep(int B, int H, int N, int d, const vc_params *p, void *ws, size_t 
   return VC_OK;
 }
 
+// Opt-in phase timing of vc_attn_fwd with CUDA events on the caller's stream:
+// a ring of PROF_RING calls, read (and averaged) once after the timed loop.
+constexpr int PROF_RING = 64;
+struct Prof {
+  bool on = false;
+  int dev = -1;
+  cudaEvent_t ev[PROF_RING][5] = {};
+  int calls = 0;  // calls recorded since profiling was switched on
+};
+Prof g_prof;
+
+void prof_mark(int i, cudaStream_t s) {
+  if (g_prof.on) cudaEventRecord(g_prof.ev[g_prof.calls % PROF_RING][i], s);
+}
+
 vc_status last_error() { return cudaGetLastError() == cudaSuccess ? VC_OK : VC_ERR_CUDA; }
 
 // Clear the completion counters and the status word at the start of a call.
@@ -366,16 +381,20 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
   const uint16_t *Qh = static_cast<const uint16_t *>(Q), *Kh = static_cast<const uint16_t *>(K),
                  *Vh = static_cast<const uint16_t *>(V);
   if ((st = clear_small(w, s)) != VC_OK) return st;
+  prof_mark(0, s);
   const int32_t *pm = perm;
   if (!pm && (sh.flags & VC_VSMOOTH)) {
     launch_cluster(sh, w, Vh, w.at<int32_t>(w.L.perm), w.at<float>(w.L.cent), s);
     pm = w.at<int32_t>(w.L.perm);
   }
+  prof_mark(1, s);
   uint8_t *q8 = w.at<uint8_t>(w.L.q8), *k8 = w.at<uint8_t>(w.L.k8), *v8t = w.at<uint8_t>(w.L.v8t);
   float *sq = w.at<float>(w.L.sq), *sk = w.at<float>(w.L.sk), *vscale = w.at<float>(w.L.vscale);
   int32_t *rep_idx = w.at<int32_t>(w.L.rep_idx);
   launch_quant_qk(sh, w, Qh, Kh, pm, q8, sq, k8, sk, s);
+  prof_mark(2, s);
   launch_quant_v(sh, w, Vh, pm, v8t, vscale, w.at<uint16_t>(w.L.vmean), rep_idx, w.at<uint16_t>(w.L.rep_delta), s);
+  prof_mark(3, s);
 
   CUtensorMap tq, tk, tv, tmu, tdt;
   const uint64_t rows = static_cast<uint64_t>(sh.BH) * sh.Npad;
@@ -410,7 +429,44 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
   ap.status = w.at<uint32_t>(w.L.status);
   k_vc_attn_fwd<<<dim3(sh.Nb, sh.BH), 192, attn_fp8_smem_bytes(), s>>>(tq, tk, tv, tmu, tdt, ap);
   count_launch();
+  prof_mark(4, s);
+  if (g_prof.on) ++g_prof.calls;
   return last_error();
+}
+
+vc_status vc_attn_profile(int on) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VC_ERR_CUDA;
+  if (on) {
+    if (g_prof.dev != dev) {
+      for (int c = 0; c < PROF_RING; ++c)
+        for (int i = 0; i < 5; ++i)
+          if (cudaEventCreate(&g_prof.ev[c][i]) != cudaSuccess) return VC_ERR_CUDA;
+      g_prof.dev = dev;
+    }
+    g_prof.on = true;
+  } else {
+    g_prof.on = false;
+  }
+  g_prof.calls = 0;
+  return VC_OK;
+}
+
+int vc_attn_profile_read(float *ms, int max_n) {
+  const int n = std::min(g_prof.calls, PROF_RING);
+  if (!ms || max_n < 4 || n == 0) return 0;
+  double acc[4] = {0, 0, 0, 0};
+  for (int c = 0; c < n; ++c) {
+    const int slot = (g_prof.calls - n + c) % PROF_RING;
+    if (cudaEventSynchronize(g_prof.ev[slot][4]) != cudaSuccess) return 0;
+    for (int i = 0; i < 4; ++i) {
+      float t = 0.0f;
+      if (cudaEventElapsedTime(&t, g_prof.ev[slot][i], g_prof.ev[slot][i + 1]) != cudaSuccess) return 0;
+      acc[i] += t;
+    }
+  }
+  for (int i = 0; i < 4; ++i) ms[i] = static_cast<float>(acc[i] / n);
+  return 4;
 }
 
 vc_status vc_attn_fwd_ref_bf16(const void *Q, const void *K, const void *V, int B, int H, int N, int d,

@@ -29,7 +29,7 @@ EXPORTED = [
     "vc_params_default", "vc_status_str", "vc_attn_workspace_bytes", "vc_attn_repair_count",
     "vc_attn_cluster", "vc_attn_quant_qk", "vc_attn_quant_v", "vc_attn_fwd", "vc_attn_fwd_ref_bf16",
     "vc_attn_expcast", "vc_attn_e4m3_encode", "vc_attn_device_status", "vc_attn_wait_selftest",
-    "vc_attn_launch_count",
+    "vc_attn_launch_count", "vc_attn_profile", "vc_attn_profile_read",
 ]
 
 
@@ -76,6 +76,9 @@ def lib():
             L.vc_attn_e4m3_encode.argtypes = [P, LL, P, P]
             L.vc_attn_device_status.argtypes = [P, P]
             L.vc_attn_wait_selftest.argtypes = [P, LL, P]
+            L.vc_attn_profile.argtypes = [I]
+            L.vc_attn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), I]
+            L.vc_attn_profile_read.restype = I
             L.vc_attn_launch_count.argtypes = []
             L.vc_attn_launch_count.restype = ctypes.c_ulonglong
             for n in EXPORTED:
@@ -142,6 +145,18 @@ def vc_attn_device_status(ws, stream) -> int:
 
 def vc_attn_wait_selftest(ws, limit_cycles, stream) -> int:
     return lib().vc_attn_wait_selftest(ws, int(limit_cycles), stream)
+
+
+def vc_attn_profile(on: bool) -> int:
+    return lib().vc_attn_profile(1 if on else 0)
+
+
+def vc_attn_profile_read() -> list:
+    """Phase durations (ms) of the last profiled vc_attn_fwd call:
+    [cluster, quant_qk, quant_v, attention]; [] if none was recorded."""
+    buf = (ctypes.c_float * 4)()
+    n = lib().vc_attn_profile_read(buf, 4)
+    return [float(buf[i]) for i in range(n)]
 
 
 def vc_attn_launch_count() -> int:

@@ -183,6 +183,19 @@ vc_status vc_attn_device_status(void *ws, void *stream);
  * VC_ERR_TIMEOUT. No GPU state is harmed; the kernel returns normally. */
 vc_status vc_attn_wait_selftest(void *ws, long long limit_cycles, void *stream);
 
+/* Opt-in phase timing for benchmarks (single-threaded use). While on, every
+ * vc_attn_fwd records CUDA events on its stream around its phases, with no
+ * host synchronization; the events (a ring of the last 64 calls) are created
+ * once per device when profiling is first switched on, and switching it on
+ * again restarts the count. vc_attn_profile_read() waits for the recorded
+ * calls and writes their mean phase durations in milliseconds to ms[0..3]:
+ * clustering (0 when a permutation was passed), Q/K quantization, V
+ * quantization + repair selection, and the fused attention kernel. Returns
+ * the number of values written (4), or 0 if nothing was recorded or
+ * max_n < 4. */
+vc_status vc_attn_profile(int on);
+int vc_attn_profile_read(float *ms, int max_n);
+
 /* Number of kernels this library has launched in this process (for the
  * bench's launch count). */
 unsigned long long vc_attn_launch_count(void);

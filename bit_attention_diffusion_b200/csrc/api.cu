@@ -504,3 +504,64 @@ vc_status vc_attn_device_status(void *ws, void *stream) {
 unsigned long long vc_attn_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"
+
+// ====================================================================== allocation-free clustering
+// For callers that cannot allocate device memory at the point where they
+// cluster (see vc_attn_cluster_noalloc in vc_attn.h): the clustering scratch
+// lives in a fixed device array that the library owns for the life of the
+// process on every device that loads it.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch for each device, looked up once per
+// device (with that device current) by cudaGetSymbolAddress. In host code the
+// symbol itself is only a host-side stand-in and must never be passed to a
+// kernel.
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[64] = {};
+
+vc_status noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VC_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return VC_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return VC_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return VC_OK;
+}
+
+}  // namespace
+
+extern "C" vc_status vc_attn_cluster_noalloc(const void *V, int B, int H, int N, int d, const vc_params *p,
+                                             int32_t *perm, float *centroids, void *stream) {
+  vc_status st = check_shape(B, H, N, d);
+  if (st != VC_OK) return st;
+  if ((st = check_params(p)) != VC_OK) return st;
+  if (!V || !perm || !centroids || !aligned(V, 16) || !aligned(perm, 16) || !aligned(centroids, 16))
+    return VC_ERR_INVALID_ARG;
+  Shape sh = make_shape(B, H, N, *p, vc_attn_repair_count(N, p));
+  WsLayout L = make_layout(sh);
+  // clustering touches only the leading regions of the layout (status,
+  // counters, permutation, labels, centroids, k-means partial sums)
+  const size_t need = L.kbar_part;
+  if (need > kNoAllocScratchBytes) return VC_ERR_WORKSPACE;
+  if ((st = check_device()) != VC_OK) return st;
+  void *scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != VC_OK) return st;
+  Ws w;
+  w.base = static_cast<uint8_t *>(scratch);
+  w.L = L;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the completion counters must start at zero; the array keeps the previous call's contents
+  if ((st = clear_small(w, s)) != VC_OK) return st;
+  launch_cluster(sh, w, static_cast<const uint16_t *>(V), perm, centroids, s);
+  return last_error();
+}
+
+extern "C" size_t vc_attn_cluster_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }

@@ -30,6 +30,7 @@ EXPORTED = [
     "vc_attn_cluster", "vc_attn_quant_qk", "vc_attn_quant_v", "vc_attn_fwd", "vc_attn_fwd_ref_bf16",
     "vc_attn_expcast", "vc_attn_e4m3_encode", "vc_attn_device_status", "vc_attn_wait_selftest",
     "vc_attn_launch_count", "vc_attn_profile", "vc_attn_profile_read",
+    "vc_attn_cluster_noalloc", "vc_attn_cluster_noalloc_max_bytes",
 ]
 
 
@@ -79,11 +80,15 @@ def lib():
             L.vc_attn_profile.argtypes = [I]
             L.vc_attn_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), I]
             L.vc_attn_profile_read.restype = I
+            L.vc_attn_cluster_noalloc.argtypes = [P, I, I, I, I, PP, P, P, P]
+            L.vc_attn_cluster_noalloc_max_bytes.argtypes = []
+            L.vc_attn_cluster_noalloc_max_bytes.restype = Z
             L.vc_attn_launch_count.argtypes = []
             L.vc_attn_launch_count.restype = ctypes.c_ulonglong
             for n in EXPORTED:
                 if n not in ("vc_params_default", "vc_status_str", "vc_attn_workspace_bytes",
-                             "vc_attn_repair_count", "vc_attn_launch_count"):
+                             "vc_attn_repair_count", "vc_attn_launch_count",
+                             "vc_attn_cluster_noalloc_max_bytes"):
                     getattr(L, n).restype = I
             _lib = L
     return _lib
@@ -112,6 +117,15 @@ def vc_attn_repair_count(N, p: VcParams) -> int:
 
 def vc_attn_cluster(V, B, H, N, d, p, perm, centroids, ws, ws_bytes, stream) -> int:
     return lib().vc_attn_cluster(V, B, H, N, d, ctypes.byref(p), perm, centroids, ws, ws_bytes, stream)
+
+
+def vc_attn_cluster_noalloc(V, B, H, N, d, p, perm, centroids, stream) -> int:
+    """vc_attn_cluster without a workspace (fixed 32 MiB library-owned scratch)."""
+    return lib().vc_attn_cluster_noalloc(V, B, H, N, d, ctypes.byref(p), perm, centroids, stream)
+
+
+def vc_attn_cluster_noalloc_max_bytes() -> int:
+    return int(lib().vc_attn_cluster_noalloc_max_bytes())
 
 
 def vc_attn_quant_qk(Q, K, perm, B, H, N, d, p, q8, sq, k8, sk, ws, ws_bytes, stream) -> int:

@@ -93,6 +93,36 @@ vc_status vc_attn_cluster(const void *V, int B, int H, int N, int d, const vc_pa
                           float *centroids, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * vc_attn_cluster without a workspace. The pages have no counterpart: this
+ * is a library convenience. It is for callers that cannot allocate device
+ * memory where they cluster - for example a plugin inside a host framework
+ * that owns every allocation and hands out no scratch, a deployment that
+ * forbids cudaMalloc after start-up so that memory use stays fixed, or code
+ * running where an allocation would synchronize the device. Such callers
+ * still pass V (input) and perm and centroids (outputs, centroids not NULL);
+ * the scratch (labels, k-means partial sums, completion counters) lives in a
+ * fixed 32 MiB array in device memory that the library reserves on every
+ * GPU that loads it, until the process exits.
+ *   Output: identical to vc_attn_cluster with the same arguments.
+ *   Limit: shapes whose clustering scratch exceeds 32 MiB (see
+ *   vc_attn_cluster_noalloc_max_bytes; about B*H*N <= 3.5 M tokens at k = 8,
+ *   the 720p video workload included) return VC_ERR_WORKSPACE before any
+ *   launch.
+ *   Set-up: the first call on each device looks up the array's device
+ *   address (cudaGetSymbolAddress) with that device current; make that first
+ *   call before any stream capture.
+ *   Calls allocate no memory (no cudaMalloc, cudaFree or allocating library
+ *   routine). All calls share the one array and each call starts by clearing
+ *   its counters; calls whose executions overlap on the GPU (other streams,
+ *   other host threads) race on it and must be serialized by the caller.
+ */
+vc_status vc_attn_cluster_noalloc(const void *V, int B, int H, int N, int d, const vc_params *p, int32_t *perm,
+                                  float *centroids, void *stream);
+
+/* Size in bytes of the fixed scratch array behind vc_attn_cluster_noalloc. */
+size_t vc_attn_cluster_noalloc_max_bytes(void);
+
+/*
  * Q/K smoothing + 8-bit quantization (prior art named in [VCA] "Por que a
  * atenção é o gargalo"): K' = K - mean_n(K) per (b,h,channel) when
  * VC_KSMOOTH is set; Q (original order) and K' (rows read through perm) are

@@ -225,9 +225,14 @@ void launch_cluster(const Shape &sh, const Ws &w, const uint16_t *V, int32_t *pe
   const size_t smem = KMEANS_SMEM_FIXED + static_cast<size_t>(sh.k) * D * 12;
   const dim3 grid(sh.km_nblk, sh.BH);
   for (int it = 0; it <= sh.iters; ++it) {
-    k_kmeans_pass<<<grid, 128, smem, s>>>(V, sh.N, sh.k, sh.km_cpb, sh.km_nblk, cent, labels,
+    if (sh.k <= 8)
+      k_kmeans_pass8<<<grid, 128, 0, s>>>(V, sh.N, sh.k, sh.km_cpb, sh.km_nblk, cent, labels,
                                           w.at<double>(w.L.km_psum), w.at<int>(w.L.km_pcnt),
                                           w.at<unsigned>(w.L.km_counter), it < sh.iters ? 1 : 0);
+    else
+      k_kmeans_pass<<<grid, 128, smem, s>>>(V, sh.N, sh.k, sh.km_cpb, sh.km_nblk, cent, labels,
+                                            w.at<double>(w.L.km_psum), w.at<int>(w.L.km_pcnt),
+                                            w.at<unsigned>(w.L.km_counter), it < sh.iters ? 1 : 0);
     count_launch();
   }
   k_perm_sort<<<sh.BH, 1024, 0, s>>>(labels, sh.N, sh.k, perm);
@@ -427,7 +432,7 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
   ap.k8 = k8;
   ap.O = static_cast<uint16_t *>(O);
   ap.status = w.at<uint32_t>(w.L.status);
-  k_vc_attn_fwd<<<dim3(sh.Nb, sh.BH), 192, attn_fp8_smem_bytes(), s>>>(tq, tk, tv, tmu, tdt, ap);
+  k_vc_attn_fwd<<<dim3(sh.Nb, sh.BH), 320, attn_fp8_smem_bytes(), s>>>(tq, tk, tv, tmu, tdt, ap);
   count_launch();
   prof_mark(4, s);
   if (g_prof.on) ++g_prof.calls;

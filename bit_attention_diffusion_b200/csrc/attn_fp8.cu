@@ -10,15 +10,22 @@
 // "Le compromis entre vitesse et fidélité": repair of the worst tokens.
 //
 // One CTA per (128-query tile, b*h). Warp roles:
-//   warp 0   TMA producer: Q once; K8 / V8 tiles through 3-stage rings; the
-//            bf16 block-mean tiles (one per 32 KV tiles); repair deltas.
-//   warp 1   allocates TMEM; lane 0 issues every tcgen05.mma and commit.
-//   warps 2-5  one thread per query row: online max, frames, ExpCast bytes,
-//            O rescale, row-sum bookkeeping, restore operands, repair, epilogue.
-// TMEM (512 columns x 128 lanes): S double buffer at columns [0,128) and
-// [128,256); the O accumulator at [256,384) followed by the row-sum columns
-// [384,400): the PV MMA uses N = 144 with a ones row appended to every V tile,
-// so column 384 receives l_t = sum_j p_ij of the decoded bytes of tile t.
+//   warp 0     TMA producer: Q once; K8 / V8 tiles through 3-stage rings; the
+//              bf16 block-mean tiles (one per 32 KV tiles); repair deltas.
+//   warp 1     allocates TMEM; lane 0 issues every tcgen05.mma and commit.
+//   warps 2-9  two warpgroups that take the KV tiles in turn (tile t goes to
+//              warpgroup t % 2), one thread per query row holding the whole
+//              row of its tile: scores, running max, frame, ExpCast bytes,
+//              O rescale when the frame moves, row-sum bookkeeping; at the end
+//              the last tile's warpgroup does the final restore and the repair,
+//              and both write the output.
+// TMEM (512 columns x 128 lanes): S double buffer at [0,256); O at [256,384);
+// two row-sum slots of 16 columns at [384,416). Per KV tile t the MMA issuer
+// runs O += P(t) V8(t), L[t%2] = P(t) E and S(t+2) = Q8 K8(t+2)^T, where E is
+// a constant block whose first row is all ones: column 0 of the slot receives
+// l_t = sum_j p_tj of the decoded bytes, overwritten (not accumulated). The
+// warpgroup of tile t reads l_t when it starts tile t+2: the commit that
+// signals S(t+2) also covers every earlier MMA.
 // O is kept in "code units": O_acc = sum p * code + sum_t l_t * mean_t/s + sum_R
 // p * delta/s, and the epilogue writes O = s_c * O_acc / l.
 #include "common.cuh"
@@ -26,34 +33,37 @@
 #include "attn_fp8.cuh"
 #include "expcast.cuh"
 
+#include <type_traits>
+
 namespace vc {
 
 namespace {
 
 constexpr int KS = 3;  // K ring stages
 constexpr int VS = 3;  // V ring stages
-constexpr uint32_t SZ_TILE8 = 128 * 128;         // one 128x128 byte tile
-constexpr uint32_t SZ_VSTAGE = SZ_TILE8 + 2048;  // + 16 ones/zero rows
+constexpr uint32_t SZ_TILE8 = 128 * 128;  // one 128x128 byte tile
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + SZ_TILE8;
 constexpr uint32_t OFF_V = OFF_K + KS * SZ_TILE8;
-constexpr uint32_t OFF_P = OFF_V + VS * SZ_VSTAGE;
+constexpr uint32_t OFF_P = OFF_V + VS * SZ_TILE8;
 constexpr uint32_t OFF_AR = OFF_P + 2 * SZ_TILE8;
 constexpr uint32_t OFF_MU = OFF_AR + SZ_TILE8;
-constexpr uint32_t OFF_LB = OFF_MU + 2 * SZ_TILE8;
+constexpr uint32_t OFF_E = OFF_MU + 2 * SZ_TILE8;  // 16 x 128-byte ones/zero block
+constexpr uint32_t OFF_LB = OFF_E + 2048;
 constexpr uint32_t SMEM_USED = OFF_LB + 32 * 128 * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // alignment slack
-static_assert(OFF_P % 1024 == 0 && OFF_AR % 1024 == 0 && OFF_MU % 1024 == 0, "tile alignment");
+static_assert(OFF_P % 1024 == 0 && OFF_AR % 1024 == 0 && OFF_MU % 1024 == 0 && OFF_E % 1024 == 0,
+              "tile alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_L = 384;
-constexpr uint32_t IDESC_QK = idesc_make(0, 0, 128, 128, false, false);   // E4M3 x E4M3 -> f32
-constexpr uint32_t IDESC_PV = idesc_make(0, 0, 128, 144, false, false);   // + row-sum columns
-constexpr uint32_t IDESC_BF = idesc_make(1, 1, 128, 128, false, false);   // bf16 x bf16 -> f32
+constexpr uint32_t IDESC_QK = idesc_make(0, 0, 128, 128, false, false);  // E4M3 x E4M3 -> f32, N = 128
+constexpr uint32_t IDESC_L = idesc_make(0, 0, 128, 16, false, false);    // row-sum MMA, N = 16
+constexpr uint32_t IDESC_BF = idesc_make(1, 1, 128, 128, false, false);  // bf16 x bf16 -> f32
 
 struct Bars {
   uint64_t q, kfull[KS], kempty[KS], vfull[VS], vempty[VS], mufull[2], muempty[2];
-  uint64_t sfull[2], pfull[2], pvdone, main, epi, repk, reps, repp, repdone, dt, fin;
+  uint64_t sfull[2], pfull[2], mxr[2], tdone[2], pvdone, main, epi, rdone, repk, reps, repp, repdone, dt, fin;
 };
 
 __device__ __forceinline__ uint64_t desc128(const uint8_t *p) { return sdesc_sw128(smem_u32(p), 16, 1024); }
@@ -64,11 +74,24 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
-__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Factor that moves a value from frame F_from to frame F_to >= F_from (both
+// multiples of 8 byte units): the exact power of two 2^((F_from - F_to)/8).
+__device__ __forceinline__ float frame_scale(float F_from, float F_to) {
+  const int k = static_cast<int>((F_to - F_from) * 0.125f);
+  return k > 126 ? 0.0f : __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
+}
+
+__device__ __forceinline__ void softmax_bar256() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void softmax_bar128(int g) { asm volatile("bar.sync %0, 128;" ::"r"(2 + g) : "memory"); }
+
+// Restore chunks. Chunk X (KV tiles 32X .. 32X+31) is flushed by the tail of
+// tile 32X+33, which reads l_{32X+31}; the chunks whose flush tile would lie
+// past the last tile (one or two) are flushed after the loop.
+__device__ __forceinline__ int first_epilogue_chunk(int T) { return T >= 34 ? (T - 34) / 32 + 1 : 0; }
 
 }  // namespace
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     k_vc_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmMu,
                   const __grid_constant__ CUtensorMap tmDT, const AttnFp8Params p) {
@@ -80,17 +103,20 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t *sP = sm + OFF_P;
   uint8_t *sAr = sm + OFF_AR;
   uint8_t *sMu = sm + OFF_MU;
+  uint8_t *sE = sm + OFF_E;
   float *sLb = reinterpret_cast<float *>(sm + OFF_LB);  // [32 slots][128 rows]
   __shared__ Bars bars;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ float s_vscale[128];
   __shared__ float s_alphaR[128];
+  __shared__ float s_m[128], s_F[128], s_ltot[128];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, bh = blockIdx.y;
   const int T = p.Nb;
   const int nrc = (p.R + 127) / 128;
+  const int X_epi0 = first_epilogue_chunk(T), X_epi1 = (T - 1) >> 5;
 
   if (threadIdx.x == 0) {
     s_abort = 0;
@@ -100,22 +126,22 @@ __global__ void __launch_bounds__(192, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.mufull[i], 1); mbar_init(&bars.muempty[i], 1);
       mbar_init(&bars.sfull[i], 1); mbar_init(&bars.pfull[i], 128);
+      mbar_init(&bars.mxr[i], 128); mbar_init(&bars.tdone[i], 128);
     }
-    mbar_init(&bars.pvdone, 1); mbar_init(&bars.main, 1); mbar_init(&bars.epi, 128);
+    mbar_init(&bars.pvdone, 1); mbar_init(&bars.main, 1); mbar_init(&bars.epi, 128); mbar_init(&bars.rdone, 1);
     mbar_init(&bars.repk, 128); mbar_init(&bars.reps, 1); mbar_init(&bars.repp, 128);
     mbar_init(&bars.repdone, 1); mbar_init(&bars.dt, 1); mbar_init(&bars.fin, 1);
     fence_mbar_init();
   }
   if (warp >= 2) {
-    const int t = threadIdx.x - 64;  // 0..127
-    // ones rows appended to every V stage: row 128 is 1.0 (0x38) in every byte,
-    // rows 129..143 are zero (K-major, 128-byte swizzle, rows 128.. of the tile)
-    for (int i = t; i < VS * 16 * 8; i += 128) {
-      const int st = i / 128, rr = 128 + (i % 128) / 8, ch = i % 8;
-      const uint32_t v = rr == 128 ? 0x38383838u : 0u;
-      *reinterpret_cast<uint4 *>(sV + st * SZ_VSTAGE + sw128_off(rr, ch)) = make_uint4(v, v, v, v);
+    const int t = threadIdx.x - 64;  // 0..255
+    // E: rows 0..15 of a K-major, 128-byte-swizzled B operand; row 0 = 1.0 (0x38)
+    if (t < 128) {
+      const int rr = t >> 3, ch = t & 7;
+      const uint32_t v = rr == 0 ? 0x38383838u : 0u;
+      *reinterpret_cast<uint4 *>(sE + sw128_off(rr, ch)) = make_uint4(v, v, v, v);
+      s_vscale[t] = p.vscale[static_cast<size_t>(bh) * 128 + t];
     }
-    s_vscale[t] = p.vscale[static_cast<size_t>(bh) * 128 + t];
     fence_proxy_async_smem();
   }
   if (warp == 1) tmem_alloc(&s_tmem, 512);
@@ -123,14 +149,11 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = s_tmem;
 
-  auto fail = [&]() {
-    s_abort = 1;
-    atomicOr(p.status, ST_TIMEOUT);
-  };
   auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
     if (s_abort) return false;
     if (!mbar_wait(bar, parity)) {
-      fail();
+      s_abort = 1;
+      atomicOr(p.status, ST_TIMEOUT);
       return false;
     }
     return true;
@@ -160,7 +183,7 @@ __global__ void __launch_bounds__(192, 1)
         ok = wait(&bars.vempty[s], ph ^ 1);
         if (!ok) break;
         mbar_arrive_expect_tx(&bars.vfull[s], SZ_TILE8);
-        tma_load_2d(sV + s * SZ_VSTAGE, &tmV, &bars.vfull[s], t * 128, bh * 128);
+        tma_load_2d(sV + s * SZ_TILE8, &tmV, &bars.vfull[s], t * 128, bh * 128);
       }
       if (ok && nrc > 0) {
         ok = wait(&bars.main, 0);
@@ -206,27 +229,34 @@ __global__ void __launch_bounds__(192, 1)
         ok = wait(&bars.pfull[t & 1], (t >> 1) & 1);
         if (!ok) break;
         tc_fence_after();
-        if (t > 0 && (t & 31) == 0) {
-          ok = issue_restore((t >> 5) - 1);
+        if (t >= 33 && ((t - 33) & 31) == 0) {
+          ok = issue_restore((t - 33) >> 5);
           if (!ok) break;
         }
         const int s = t % KS;
         ok = wait(&bars.vfull[s], (t / KS) & 1);
         if (!ok) break;
         tc_fence_after();
+        const uint8_t *pa = sP + (t & 1) * SZ_TILE8;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_f8_ss(tmem + TM_O, desc128(sP + (t & 1) * SZ_TILE8 + 32 * kk), desc128(sV + s * SZ_VSTAGE + 32 * kk),
-                    IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+          mma_f8_ss(tmem + TM_O, desc128(pa + 32 * kk), desc128(sV + s * SZ_TILE8 + 32 * kk), IDESC_QK,
+                    (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f8_ss(tmem + TM_L + 16 * (t & 1), desc128(pa + 32 * kk), desc128(sE + 32 * kk), IDESC_L, kk > 0);
         mma_commit(&bars.vempty[s]);
         mma_commit(&bars.pvdone);
         if (t + 2 < T) ok = issue_qk(t + 2);
       }
       if (ok) mma_commit(&bars.main);
-      if (ok) ok = wait(&bars.epi, 0);
-      if (ok) {
+      // the restore chunks flushed after the loop, in order
+      for (int X = X_epi0, e = 0; X <= X_epi1 && ok; ++X, ++e) {
+        ok = wait(&bars.epi, e & 1);
+        if (!ok) break;
         tc_fence_after();
-        ok = issue_restore((T - 1) >> 5);
+        ok = issue_restore(X);
+        if (ok) mma_commit(&bars.rdone);
       }
       for (int rc = 0; rc < nrc && ok; ++rc) {
         ok = wait(&bars.repk, rc & 1);
@@ -249,21 +279,28 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax rows
+    // Warpgroup g (warps 2+4g .. 5+4g) takes the tiles t with t % 2 == g;
+    // thread row r = 32*(warp%4) + lane. Shared per-row state, handed from
+    // tile to tile in order: s_m / s_F (running max and frame; mxr[t%2]) and
+    // s_ltot / sLb (row sum and staged l_t, both in the current frame;
+    // tdone[t%2]).
+    const int g = (warp - 2) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const float sqs = p.sq[static_cast<size_t>(bh) * T + qt];
     const float *skh = p.sk + static_cast<size_t>(bh) * T;
     const int tail = p.N - (T - 1) * 128;  // valid keys in the last tile
-    float m = -INFINITY, F = -INFINITY, ltot = 0.0f;
     bool ok = true;
+    float F_own = 0.0f;   // frame of this warpgroup's latest tile
+    float F_hand = 0.0f;  // frame handed over to this warpgroup's latest tile
+    float sk_next = skh[g < T ? g : 0];
     // every lane waits; the outcome is made warp-uniform so that the
     // .sync.aligned TMEM instructions below always see the whole warp
     auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
       const bool w = wait(bar, parity);
       return __all_sync(0xFFFFFFFFu, w);
     };
-
     auto flush = [&](int nvalid) {
       // A operand of the restore MMA: row r = [hi(l_0..l_31) | lo(l_0..l_31)] in bf16
       uint32_t hw[16], lw[16];
@@ -286,29 +323,33 @@ __global__ void __launch_bounds__(192, 1)
       }
     };
 
-    for (int t = 0; t < T && ok; ++t) {
+    // One KV tile t (t % 2 == g). LAST: the ragged last tile (keys >= tail masked).
+    auto tile = [&](int t, auto last_tag) -> bool {
+      constexpr bool LAST = decltype(last_tag)::value;
       const int b = t & 1;
-      ok = wwait(&bars.sfull[b], (t >> 1) & 1);
-      if (!ok) break;
+      const float skt = sk_next;
+      if (t + 2 < T) sk_next = skh[t + 2];  // this warpgroup's next tile
+      if (!wwait(&bars.sfull[b], (t >> 1) & 1)) return false;
       tc_fence_after();
+      // S(t) and, from the row-sum slot this tile reuses, l_{t-2} (complete:
+      // the commit behind sfull covers every earlier MMA)
+      uint32_t sr[128];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        tmem_ld32(trow + TM_S0 + b * 128 + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * i]));
+      const uint32_t lraw = tmem_ld1(trow + TM_L + 16 * b);
+      tmem_wait_ld();
       float s[128];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint32_t v[32];
-        tmem_ld32(trow + TM_S0 + b * 128 + 32 * i, v);
-        tmem_wait_ld();
+      for (int j = 0; j < 128; ++j) s[j] = __uint_as_float(sr[j]);
+      if constexpr (LAST) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) s[32 * i + j] = __uint_as_float(v[j]);
+        for (int j = 0; j < 128; ++j)
+          if (j >= tail) s[j] = -INFINITY;
       }
-      const bool last = (t == T - 1) && (tail < 128);
       float mx;
       {
         float mm[43];
-        if (last) {
-#pragma unroll
-          for (int j = 0; j < 128; ++j)
-            if (j >= tail) s[j] = -INFINITY;
-        }
 #pragma unroll
         for (int j = 0; j < 42; ++j) mm[j] = max3(s[3 * j], s[3 * j + 1], s[3 * j + 2]);
         mm[42] = fmaxf(s[126], s[127]);
@@ -319,85 +360,132 @@ __global__ void __launch_bounds__(192, 1)
         for (int j = 0; j < 5; ++j) mm[j] = max3(mm[3 * j], mm[3 * j + 1], mm[3 * j + 2]);
         mx = max3(mm[0], mm[1], fmaxf(mm[2], fmaxf(mm[3], mm[4])));
       }
-      const float alpha = __fmul_rn(__fmul_rn(sqs, skh[t]), p.kappa);
-      m = fmaxf(m, __fmul_rn(mx, alpha));
-      const float Fn = 8.0f * ceilf(m * 0.125f);
+      const float alpha = __fmul_rn(__fmul_rn(sqs, skt), p.kappa);
+      // running max and frame, taken over from tile t-1's warpgroup
+      float m_prev = -INFINITY, F_prev = -INFINITY;
       if (t > 0) {
-        ok = wwait(&bars.pvdone, (t - 1) & 1);
-        if (!ok) break;
+        if (!wwait(&bars.mxr[(t - 1) & 1], ((t - 1) >> 1) & 1)) return false;
+        m_prev = s_m[r];
+        F_prev = s_F[r];
+      }
+      const float m = fmaxf(m_prev, __fmul_rn(mx, alpha));
+      const float Fn = 8.0f * ceilf(m * 0.125f);
+      if (t == 0) F_prev = Fn;
+      s_m[r] = m;  // for tile t+1 (after the last tile, s_F holds the final frame)
+      s_F[r] = Fn;
+      if (t + 1 < T) mbar_arrive(&bars.mxr[b]);
+      // bytes against the frame Fn, to P buffer t&1 (its previous reader
+      // PV(t-2) completed before S(t) was signalled)
+      {
+        const float al24 = alpha * TWO_M24;
+        const float c24 = (static_cast<float>(p.C) - Fn) * TWO_M24;
+        uint8_t *prow = sP + b * SZ_TILE8;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) w[q] = expcast4(&s[16 * ch + 4 * q], al24, c24);
+          if constexpr (LAST) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int j0 = 16 * ch + 4 * q;
+              uint32_t keep = 0u;
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (j0 + e < tail) keep |= 0xFFu << (8 * e);
+              w[q] &= keep;
+            }
+          }
+          *reinterpret_cast<uint4 *>(prow + sw128_off(r, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      // tail, in tile order after tile t-1's tail
+      if (t > 0 && !wwait(&bars.tdone[(t - 1) & 1], ((t - 1) >> 1) & 1)) return false;
+      const bool need = Fn != F_prev;
+      const float sc = need ? frame_scale(F_prev, Fn) : 1.0f;
+      if (__any_sync(0xFFFFFFFFu, need)) {
+        // O holds PV(0..t-1) in frame F_prev: rescale it before PV(t)
+        if (!wwait(&bars.pvdone, (t - 1) & 1)) return false;
         tc_fence_after();
-        const float lprev = __uint_as_float(tmem_ld1(trow + TM_L));
+        uint32_t o[128];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          tmem_ld32(trow + TM_O + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&o[32 * i]));
         tmem_wait_ld();
-        tmem_st1(trow + TM_L, 0u);
-        const int slot = (t - 1) & 31;
-        sLb[slot * 128 + r] = lprev;
-        ltot += lprev;
-        const bool need = Fn != F;
-        if (__any_sync(0xFFFFFFFFu, need)) {
-          const int kshift = need ? static_cast<int>((Fn - F) * 0.125f) : 0;
-          const float sc = kshift > 126 ? 0.0f : __uint_as_float(static_cast<uint32_t>(127 - kshift) << 23);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t v[32];
-            tmem_ld32(trow + TM_O + 32 * i, v);
-            tmem_wait_ld();
+        for (int j = 0; j < 128; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * sc);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * sc);
-            tmem_st32(trow + TM_O + 32 * i, v);
-          }
-          ltot *= sc;
-          for (int sl = 0; sl <= slot; ++sl) sLb[sl * 128 + r] *= sc;
-        }
-        if (slot == 31) flush(32);
+        for (int i = 0; i < 4; ++i)
+          tmem_st32(trow + TM_O + 32 * i, *reinterpret_cast<const uint32_t(*)[32]>(&o[32 * i]));
         tmem_wait_st();
+        if (need)
+          for (int sl = 0; sl < 32; ++sl) sLb[sl * 128 + r] *= sc;
       }
-      F = Fn;
-      const float al24 = alpha * TWO_M24;
-      const float c24 = (static_cast<float>(p.C) - F) * TWO_M24;
-      uint8_t *prow = sP + b * SZ_TILE8;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) w[q] = expcast4(&s[16 * ch + 4 * q], al24, c24);
-        if (last) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int j0 = 16 * ch + 4 * q;
-            uint32_t keep = 0u;
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (j0 + e < tail) keep |= 0xFFu << (8 * e);
-            w[q] &= keep;
-          }
-        }
-        *reinterpret_cast<uint4 *>(prow + sw128_off(r, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+      float lt = (t > 0 ? s_ltot[r] : 0.0f) * sc;
+      if (t >= 2) {
+        // l_{t-2}: this warpgroup's previous tile, computed in frame F_own
+        const float lo = __uint_as_float(lraw) * frame_scale(F_own, Fn);
+        const int slot = (t - 2) & 31;
+        sLb[slot * 128 + r] = lo;
+        lt += lo;
+        if (slot == 31) flush(32);
       }
+      s_ltot[r] = lt;
+      F_own = Fn;
+      F_hand = F_prev;
       fence_proxy_async_smem();
       tc_fence_before();
+      mbar_arrive(&bars.tdone[b]);
       mbar_arrive(&bars.pfull[b]);
-    }
+      return true;
+    };
+
+    const bool ragged = tail < 128;
+    for (int t = g; t < T - 1 && ok; t += 2) ok = tile(t, std::false_type{});
+    if (ok && ((T - 1) & 1) == g)
+      ok = ragged ? tile(T - 1, std::true_type{}) : tile(T - 1, std::false_type{});
 
     // ---------------------------------------------------------- end of the KV loop
-    if (ok) ok = wwait(&bars.main, 0);
-    if (ok) {
+    // The warpgroup of the last tile adds l_{T-2} and l_{T-1} to the row sum
+    // and flushes the remaining one or two restore chunks; then it runs the
+    // repair; then both warpgroups write half of the output columns each.
+    const bool fin_wg = ((T - 1) & 1) == g;
+    if (ok && fin_wg) ok = wwait(&bars.main, 0);
+    const float F_fin = F_own;  // frame of the last tile (meaningful in fin_wg)
+    if (ok && fin_wg) {
       tc_fence_after();
-      const float lprev = __uint_as_float(tmem_ld1(trow + TM_L));
-      tmem_wait_ld();
-      const int slot = (T - 1) & 31;
-      sLb[slot * 128 + r] = lprev;
-      ltot += lprev;
-      flush(slot + 1);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bars.epi);
+      float lt = s_ltot[r];
+      int e = 0;
+      for (int u = (T >= 2 ? T - 2 : 0); u <= T - 1; ++u) {
+        // l_u is in slot u%2, computed in frame F_{T-1} (own last tile) or
+        // F_{T-2} (the frame handed over to the last tile)
+        const float lu_raw = __uint_as_float(tmem_ld1(trow + TM_L + 16 * (u & 1)));
+        tmem_wait_ld();
+        const float lo = lu_raw * frame_scale(u == T - 1 ? F_own : F_hand, F_fin);
+        const int slot = u & 31;
+        sLb[slot * 128 + r] = lo;
+        lt += lo;
+        if (slot == 31 || u == T - 1) {
+          if (e > 0) {  // the restore of the previous flush must have read sAr
+            ok = wwait(&bars.rdone, (e - 1) & 1);
+            if (!ok) break;
+          }
+          flush(slot + 1);
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(&bars.epi);
+          ++e;
+        }
+      }
+      s_ltot[r] = lt;
     }
-    // ---------------------------------------------------------- repair
-    const float c24f = (static_cast<float>(p.C) - F) * TWO_M24;
-    for (int rc = 0; rc < nrc && ok; ++rc) {
-      if (rc > 0) {
-        ok = wwait(&bars.repdone, (rc - 1) & 1);
-        if (!ok) break;
+    // ---------------------------------------------------------- repair (the last tile's warpgroup)
+    const float c24f = (static_cast<float>(p.C) - F_fin) * TWO_M24;
+    for (int rc = 0; rc < nrc && fin_wg; ++rc) {
+      if (ok && rc > 0) ok = wwait(&bars.repdone, (rc - 1) & 1);
+      if (!ok) {
+        softmax_bar128(g);  // keep this warpgroup's barrier sequence on failure
+        continue;
       }
       const int i = rc * 128 + r;
       const int nval = min(128, p.R - rc * 128);
@@ -419,9 +507,9 @@ __global__ void __launch_bounds__(192, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars.repk);
-      softmax_bar();  // s_alphaR visible to every row
+      softmax_bar128(g);  // s_alphaR visible to every row of this warpgroup
       ok = wwait(&bars.reps, rc & 1);
-      if (!ok) break;
+      if (!ok) continue;  // one barrier per iteration on every path
       tc_fence_after();
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -430,12 +518,12 @@ __global__ void __launch_bounds__(192, 1)
         tmem_wait_ld();
         // 32 scores -> 32 bf16 probabilities (two 16-byte chunks per 8 values)
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
+        for (int gg = 0; gg < 4; ++gg) {
           uint32_t outw[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int j = 32 * q + 8 * g + 2 * e;
-            const uint32_t h = expcast2(__uint_as_float(v[8 * g + 2 * e]), __uint_as_float(v[8 * g + 2 * e + 1]),
+            const int j = 32 * q + 8 * gg + 2 * e;
+            const uint32_t h = expcast2(__uint_as_float(v[8 * gg + 2 * e]), __uint_as_float(v[8 * gg + 2 * e + 1]),
                                         s_alphaR[j], s_alphaR[j + 1], c24f);
             uint32_t b0 = h & 0xFFu, b1 = (h >> 16) & 0xFFu;
             if (j >= nval) b0 = 0u;
@@ -444,7 +532,7 @@ __global__ void __launch_bounds__(192, 1)
             const __nv_bfloat162 pb = __floats2bfloat162_rn(pv.x, pv.y);
             outw[e] = *reinterpret_cast<const uint32_t *>(&pb);
           }
-          const int jj = 32 * q + 8 * g;  // first key of this 16-byte chunk
+          const int jj = 32 * q + 8 * gg;  // first key of this 16-byte chunk
           *reinterpret_cast<uint4 *>(sP + (jj >> 6) * SZ_TILE8 + sw128_off(r, (jj & 63) >> 3)) =
               make_uint4(outw[0], outw[1], outw[2], outw[3]);
         }
@@ -453,31 +541,33 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(&bars.repp);
     }
-    // ---------------------------------------------------------- epilogue
+    // ---------------------------------------------------------- epilogue (each warpgroup 64 columns)
     if (ok) ok = wwait(&bars.fin, 0);
+    softmax_bar256();  // s_ltot final, from the last tile's warpgroup
     if (ok) {
       tc_fence_after();
+      const int c0 = g * 64;
       const int row = qt * 128 + r;
       uint16_t *orow = p.O + (static_cast<size_t>(bh) * p.N + row) * 128;
-      const float inv_ok = ltot;
+      const float lrow = s_ltot[r];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 2; ++i) {
         uint32_t v[32];
-        tmem_ld32(trow + TM_O + 32 * i, v);
+        tmem_ld32(trow + TM_O + c0 + 32 * i, v);
         tmem_wait_ld();
         if (row < p.N) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
+          for (int gg = 0; gg < 4; ++gg) {
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int c = 32 * i + 8 * g + 2 * e;
-              const float o0 = __fdiv_rn(__uint_as_float(v[8 * g + 2 * e]) * s_vscale[c], inv_ok);
-              const float o1 = __fdiv_rn(__uint_as_float(v[8 * g + 2 * e + 1]) * s_vscale[c + 1], inv_ok);
+              const int c = c0 + 32 * i + 8 * gg + 2 * e;
+              const float o0 = __fdiv_rn(__uint_as_float(v[8 * gg + 2 * e]) * s_vscale[c], lrow);
+              const float o1 = __fdiv_rn(__uint_as_float(v[8 * gg + 2 * e + 1]) * s_vscale[c + 1], lrow);
               const __nv_bfloat162 ob = __floats2bfloat162_rn(o0, o1);
               w[e] = *reinterpret_cast<const uint32_t *>(&ob);
             }
-            *reinterpret_cast<uint4 *>(orow + 32 * i + 8 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4 *>(orow + c0 + 32 * i + 8 * gg) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }

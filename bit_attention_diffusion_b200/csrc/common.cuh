@@ -9,7 +9,7 @@
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
-#include "../../include/vc_attn.h"
+#include "vc_attn.h"
 
 namespace vc {
 

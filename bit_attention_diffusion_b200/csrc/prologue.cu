@@ -130,11 +130,149 @@ __global__ void __launch_bounds__(128) k_kmeans_pass(const uint16_t *__restrict_
   for (int j = 0; j < k; ++j) {
     double s = 0.0;
     long long n = 0;
-    for (int b = 0; b < nblk; ++b) {
+#pragma unroll 16
+    for (int b = 0; b < nblk; ++b) {  // loads batched by the unroll, sums kept in block order
       s += __ldcg(psum + ((static_cast<size_t>(bh) * nblk + b) * k + j) * D + tid);
       n += __ldcg(pcnt + (static_cast<size_t>(bh) * nblk + b) * k + j);
     }
     if (n > 0) cent_h[j * D + tid] = static_cast<float>(s / static_cast<double>(n));
+  }
+  if (tid == 0) counter[bh] = 0u;
+}
+
+// Fast path of the Lloyd pass for k <= 8, same arithmetic per (token,
+// cluster) as k_kmeans_pass: d = fp32(v - c) and acc = fma(d, d, acc) in
+// channel order, two clusters per packed f32x2 instruction (each lane rounds
+// exactly like the scalar instruction). Centroids sit channel-major in shared
+// memory ([c][8]) so one 16-byte load brings four clusters of a channel; the
+// fp64 sums run in registers of the channel's thread behind a label switch
+// that is uniform across the warp (all lanes read the same token).
+constexpr int KM8_ROW_WORDS = 68;  // 272-byte rows: 16-byte aligned, spread over banks
+
+__device__ __forceinline__ void sub_fma2(float x, float c0, float c1, float &a0, float &a1) {
+  asm("{\n\t.reg .b64 xx, cc, dd, aa;\n\t"
+      "mov.b64 xx, {%2, %2};\n\tmov.b64 cc, {%3, %4};\n\tmov.b64 aa, {%0, %1};\n\t"
+      "sub.rn.f32x2 dd, xx, cc;\n\t"
+      "fma.rn.f32x2 aa, dd, dd, aa;\n\t"
+      "mov.b64 {%0, %1}, aa;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x), "f"(c0), "f"(c1));
+}
+
+__global__ void __launch_bounds__(128) k_kmeans_pass8(const uint16_t *__restrict__ V, int N, int k, int cpb,
+                                                      int nblk, float *__restrict__ cent,
+                                                      int32_t *__restrict__ labels, double *__restrict__ psum,
+                                                      int *__restrict__ pcnt, unsigned *__restrict__ counter,
+                                                      int accumulate) {
+  __shared__ __align__(16) uint32_t sv[TILE * KM8_ROW_WORDS];
+  __shared__ __align__(16) float scent[D * 8];  // [c][j], j >= k padded with +inf-distance values
+  __shared__ int slab[TILE];
+  __shared__ int scnt[8];
+  __shared__ int s_last;
+  const int bh = blockIdx.y, blk = blockIdx.x, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const uint16_t *Vh = V + static_cast<size_t>(bh) * N * D;
+  float *cent_h = cent + static_cast<size_t>(bh) * k * D;
+  for (int i = tid; i < D * 8; i += TILE) {
+    const int c = i >> 3, j = i & 7;
+    scent[i] = j < k ? cent_h[j * D + c] : 0.0f;
+  }
+  if (tid < 8) scnt[tid] = 0;
+  double acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0, acc4 = 0, acc5 = 0, acc6 = 0, acc7 = 0;
+  const int n_begin = blk * cpb * TILE;
+  const int n_end = min(N, n_begin + cpb * TILE);
+  for (int n0 = n_begin; n0 < n_end; n0 += TILE) {
+    const int cnt = min(TILE, n_end - n0);
+    __syncthreads();
+    // coalesced chunk load: 16 lanes per 256-byte row, two rows per warp per step
+    for (int r = warp * 2 + (lane >> 4); r < cnt; r += 8) {
+      const uint4 w = *reinterpret_cast<const uint4 *>(Vh + static_cast<size_t>(n0 + r) * D + 8 * (lane & 15));
+      *reinterpret_cast<uint4 *>(&sv[r * KM8_ROW_WORDS + 4 * (lane & 15)]) = w;
+    }
+    __syncthreads();
+    if (tid < cnt) {
+      float a[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = 0.0f;
+      const uint32_t *row = sv + tid * KM8_ROW_WORDS;
+#pragma unroll 2
+      for (int g = 0; g < 16; ++g) {  // 8 channels per 16-byte load
+        const uint4 w = *reinterpret_cast<const uint4 *>(row + 4 * g);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = 8 * g + 2 * h + e;
+            const float x = e ? __uint_as_float(ws[h] & 0xFFFF0000u) : __uint_as_float(ws[h] << 16);
+            const float4 cA = *reinterpret_cast<const float4 *>(&scent[c * 8]);
+            const float4 cB = *reinterpret_cast<const float4 *>(&scent[c * 8 + 4]);
+            sub_fma2(x, cA.x, cA.y, a[0], a[1]);
+            sub_fma2(x, cA.z, cA.w, a[2], a[3]);
+            sub_fma2(x, cB.x, cB.y, a[4], a[5]);
+            sub_fma2(x, cB.z, cB.w, a[6], a[7]);
+          }
+        }
+      }
+      int best = 0;
+      float bestd = a[0];
+#pragma unroll
+      for (int j = 1; j < 8; ++j)
+        if (j < k && a[j] < bestd) {
+          bestd = a[j];
+          best = j;
+        }
+      slab[tid] = best;
+      labels[static_cast<size_t>(bh) * N + n0 + tid] = best;
+    }
+    if (accumulate) {
+      __syncthreads();
+      const int c = tid;
+      for (int r = 0; r < cnt; ++r) {
+        const uint32_t pr = sv[r * KM8_ROW_WORDS + (c >> 1)];
+        const double x = static_cast<double>((c & 1) ? __uint_as_float(pr & 0xFFFF0000u) : __uint_as_float(pr << 16));
+        switch (slab[r]) {  // uniform across the warp
+          case 0: acc0 += x; break;
+          case 1: acc1 += x; break;
+          case 2: acc2 += x; break;
+          case 3: acc3 += x; break;
+          case 4: acc4 += x; break;
+          case 5: acc5 += x; break;
+          case 6: acc6 += x; break;
+          default: acc7 += x; break;
+        }
+      }
+      if (tid < 8) {
+        int n = 0;
+        for (int r = 0; r < cnt; ++r) n += (slab[r] == tid);
+        scnt[tid] += n;
+      }
+    }
+  }
+  if (!accumulate) return;
+  double *ps = psum + (static_cast<size_t>(bh) * nblk + blk) * k * D;
+  int *pc = pcnt + (static_cast<size_t>(bh) * nblk + blk) * k;
+  const double accs[8] = {acc0, acc1, acc2, acc3, acc4, acc5, acc6, acc7};
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < k) ps[j * D + tid] = accs[j];
+  __syncthreads();
+  if (tid < k) pc[tid] = scnt[tid];
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&counter[bh], 1u) == static_cast<unsigned>(nblk - 1));
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int j = 0; j < k; ++j) {
+    double sum = 0.0;
+    long long n = 0;
+#pragma unroll 16
+    for (int b = 0; b < nblk; ++b) {  // loads batched by the unroll, sums kept in block order
+      sum += __ldcg(psum + ((static_cast<size_t>(bh) * nblk + b) * k + j) * D + tid);
+      n += __ldcg(pcnt + (static_cast<size_t>(bh) * nblk + b) * k + j);
+    }
+    if (n > 0) cent_h[j * D + tid] = static_cast<float>(sum / static_cast<double>(n));
   }
   if (tid == 0) counter[bh] = 0u;
 }
@@ -322,6 +460,7 @@ __global__ void __launch_bounds__(128) k_quantv_pass1(const uint16_t *__restrict
   if (!s_last) return;
   __threadfence();
   float a = 0.0f;
+#pragma unroll 32
   for (int b = 0; b < Nb; ++b) a = fmaxf(a, __ldcg(amax_part + (static_cast<size_t>(bh) * Nb + b) * D + c));
   int e = 0;
   float s = 1.0f;

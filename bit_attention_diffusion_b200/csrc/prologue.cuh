@@ -7,6 +7,8 @@ namespace vc {
 __global__ void k_kmeans_init(const uint16_t *V, int N, int k, float *cent);
 __global__ void k_kmeans_pass(const uint16_t *V, int N, int k, int cpb, int nblk, float *cent, int32_t *labels,
                               double *psum, int *pcnt, unsigned *counter, int accumulate);
+__global__ void k_kmeans_pass8(const uint16_t *V, int N, int k, int cpb, int nblk, float *cent, int32_t *labels,
+                               double *psum, int *pcnt, unsigned *counter, int accumulate);
 __global__ void k_perm_sort(const int32_t *labels, int N, int k, int32_t *perm);
 __global__ void k_kbar_partial(const uint16_t *K, int N, int nchunk, double *part);
 __global__ void k_kbar_final(const double *part, int N, int nchunk, int ksmooth, float *kbar);

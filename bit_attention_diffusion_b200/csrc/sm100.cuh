@@ -45,15 +45,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Wait for the phase of `parity` to complete; false if it did not within the limit.
+
+// Wait for the phase of `parity` to complete; false if it did not within the
+// limit. try_wait suspends the thread in hardware for a short while when the
+// phase is not complete yet; the clock is read only every 256 tries so the
+// loop stays a few instructions long.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           long long limit = VC_WAIT_LIMIT_CYCLES) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const long long t0 = clock64();
+  uint32_t n = 0;
   while (true) {
     if (mbar_try_wait(a, parity)) return true;
-    if (clock64() - t0 > limit) return false;
+    if ((++n & 255u) == 0u && clock64() - t0 > limit) return false;
   }
 }
 

@@ -189,3 +189,13 @@ def test_vsmooth_lowers_value_term_error_on_outlier_channel(torch):
     full = np.sqrt(acc["full"][0] / acc["full"][1])
     plain = np.sqrt(acc["plain"][0] / acc["plain"][1])
     assert full < 0.75 * plain, (full, plain)
+
+
+@pytest.mark.parametrize("N", [4097, 4200, 4224, 8300])
+def test_fwd_restore_chunk_boundaries(torch, N):
+    """KV-tile counts where the block-mean restore chunks (32 tiles each) end
+    right at the last tile (two chunks restored after the loop) or one past it."""
+    x = synth.make_inputs(synth.custom(1, 2, N, seed=600 + N))
+    out = _run_gpu(torch, x, vcattn.params())
+    rel, worst = _compare(x, out, [(0, 0), (0, 1)], lambda n: _sampled_rows(n, 48), oracle.FLAGS_DEFAULT)
+    assert rel <= TOL and worst <= 2 * TOL, (rel, worst)

@@ -29,7 +29,7 @@ def _inputs(B, H, N, seed=0):
 
 
 @pytest.mark.parametrize("B,H,N", SHAPES)
-@pytest.mark.parametrize("k,iters", [(8, 3), (3, 1), (1, 2)])
+@pytest.mark.parametrize("k,iters", [(8, 3), (3, 1), (1, 2), (12, 2)])
 def test_cluster_bit_exact(torch, B, H, N, k, iters):
     x = _inputs(B, H, N)
     p = vcattn.params(k=k, iters=iters)

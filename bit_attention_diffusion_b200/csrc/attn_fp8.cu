@@ -10,7 +10,7 @@
 // "Le compromis entre vitesse et fidélité": repair of the worst tokens.
 //
 // One CTA per (128-query tile, b*h). Warp roles:
-//   warp 0     TMA producer: Q once; K8 / V8 tiles through 3-stage rings; the
+//   warp 0     TMA producer: Q once; K8 / V8 tiles through 4-stage rings; the
 //              bf16 block-mean tiles (one per 32 KV tiles); repair deltas.
 //   warp 1     allocates TMEM; lane 0 issues every tcgen05.mma and commit.
 //   warps 2-9  two warpgroups that take the KV tiles in turn (tile t goes to
@@ -20,7 +20,9 @@
 //              the last tile's warpgroup does the final restore and the repair,
 //              and both write the output.
 // TMEM (512 columns x 128 lanes): S double buffer at [0,256); O at [256,384);
-// two row-sum slots of 16 columns at [384,416). Per KV tile t the MMA issuer
+// two row-sum slots of 16 columns at [384,416); the probability bytes P, double
+// buffered, 32 columns each (4 bytes per column) at [416,480), read by the PV
+// and row-sum MMAs as their A operand straight from TMEM. Per KV tile t the MMA issuer
 // runs O += P(t) V8(t), L[t%2] = P(t) E and S(t+2) = Q8 K8(t+2)^T, where E is
 // a constant block whose first row is all ones: column 0 of the slot receives
 // l_t = sum_j p_tj of the decoded bytes, overwritten (not accumulated). The
@@ -39,34 +41,79 @@ namespace vc {
 
 namespace {
 
-constexpr int KS = 3;  // K ring stages
-constexpr int VS = 3;  // V ring stages
+constexpr int KS = 4;  // K ring stages
+constexpr int VS = 4;  // V ring stages
 constexpr uint32_t SZ_TILE8 = 128 * 128;  // one 128x128 byte tile
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + SZ_TILE8;
 constexpr uint32_t OFF_V = OFF_K + KS * SZ_TILE8;
-constexpr uint32_t OFF_P = OFF_V + VS * SZ_TILE8;
-constexpr uint32_t OFF_AR = OFF_P + 2 * SZ_TILE8;
+constexpr uint32_t OFF_AR = OFF_V + VS * SZ_TILE8;
 constexpr uint32_t OFF_MU = OFF_AR + SZ_TILE8;
 constexpr uint32_t OFF_E = OFF_MU + 2 * SZ_TILE8;  // 16 x 128-byte ones/zero block
 constexpr uint32_t OFF_LB = OFF_E + 2048;
 constexpr uint32_t SMEM_USED = OFF_LB + 32 * 128 * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // alignment slack
-static_assert(OFF_P % 1024 == 0 && OFF_AR % 1024 == 0 && OFF_MU % 1024 == 0 && OFF_E % 1024 == 0,
+static_assert(OFF_AR % 1024 == 0 && OFF_MU % 1024 == 0 && OFF_E % 1024 == 0,
               "tile alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_L = 384;
+constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_L = 384, TM_P = 416;
 constexpr uint32_t IDESC_QK = idesc_make(0, 0, 128, 128, false, false);  // E4M3 x E4M3 -> f32, N = 128
 constexpr uint32_t IDESC_L = idesc_make(0, 0, 128, 16, false, false);    // row-sum MMA, N = 16
 constexpr uint32_t IDESC_BF = idesc_make(1, 1, 128, 128, false, false);  // bf16 x bf16 -> f32
 
 struct Bars {
-  uint64_t q, kfull[KS], kempty[KS], vfull[VS], vempty[VS], mufull[2], muempty[2];
+  uint64_t q, kvfull[KS], kempty[KS], vempty[VS], mufull[2], muempty[2];
   uint64_t sfull[2], pfull[2], mxr[2], tdone[2], pvdone, main, epi, rdone, repk, reps, repp, repdone, dt, fin;
 };
 
 __device__ __forceinline__ uint64_t desc128(const uint8_t *p) { return sdesc_sw128(smem_u32(p), 16, 1024); }
+
+// tcgen05 MMA with the A operand read from TMEM (M = 128 lanes; K = 32 bytes
+// per instruction = 8 columns of 4 packed E4M3 values) and B from shared memory.
+__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The MMA issuer warp runs converged; these execute the tcgen05 instruction
+// only where `leader` is nonzero (one elected lane), so every operand can be
+// computed once per warp in uniform registers.
+__device__ __forceinline__ void mma_f8_ss_el(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc,
+                                             uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(leader)
+      : "memory");
+}
+__device__ __forceinline__ void mma_f8_ts_el(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc,
+                                             uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(leader)
+      : "memory");
+}
+__device__ __forceinline__ void mma_f16_ss_el(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc,
+                                              uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(leader)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_el(uint64_t *bar, uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
+      "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar)),
+      "r"(leader)
+      : "memory");
+}
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
@@ -100,7 +147,6 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t *sQ = sm + OFF_Q;
   uint8_t *sK = sm + OFF_K;
   uint8_t *sV = sm + OFF_V;
-  uint8_t *sP = sm + OFF_P;
   uint8_t *sAr = sm + OFF_AR;
   uint8_t *sMu = sm + OFF_MU;
   uint8_t *sE = sm + OFF_E;
@@ -121,8 +167,11 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     s_abort = 0;
     mbar_init(&bars.q, 1);
-    for (int i = 0; i < KS; ++i) { mbar_init(&bars.kfull[i], 1); mbar_init(&bars.kempty[i], 1); }
-    for (int i = 0; i < VS; ++i) { mbar_init(&bars.vfull[i], 1); mbar_init(&bars.vempty[i], 1); }
+    for (int i = 0; i < KS; ++i) {
+      mbar_init(&bars.kvfull[i], 1);
+      mbar_init(&bars.kempty[i], 1);
+      mbar_init(&bars.vempty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.mufull[i], 1); mbar_init(&bars.muempty[i], 1);
       mbar_init(&bars.sfull[i], 1); mbar_init(&bars.pfull[i], 128);
@@ -176,14 +225,12 @@ __global__ void __launch_bounds__(320, 1)
         }
         const int s = t % KS;
         const uint32_t ph = (t / KS) & 1;
-        ok = wait(&bars.kempty[s], ph ^ 1);
+        ok = wait(&bars.kempty[s], ph ^ 1) && wait(&bars.vempty[s], ph ^ 1);
         if (!ok) break;
-        mbar_arrive_expect_tx(&bars.kfull[s], SZ_TILE8);
-        tma_load_2d(sK + s * SZ_TILE8, &tmK, &bars.kfull[s], 0, bh * p.Npad + t * 128);
-        ok = wait(&bars.vempty[s], ph ^ 1);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bars.vfull[s], SZ_TILE8);
-        tma_load_2d(sV + s * SZ_TILE8, &tmV, &bars.vfull[s], t * 128, bh * 128);
+        // K(t) and V(t) on one barrier: the issuer waits once, before QK(t)
+        mbar_arrive_expect_tx(&bars.kvfull[s], 2 * SZ_TILE8);
+        tma_load_2d(sK + s * SZ_TILE8, &tmK, &bars.kvfull[s], 0, bh * p.Npad + t * 128);
+        tma_load_2d(sV + s * SZ_TILE8, &tmV, &bars.kvfull[s], t * 128, bh * 128);
       }
       if (ok && nrc > 0) {
         ok = wait(&bars.main, 0);
@@ -198,85 +245,93 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      bool ok = wait(&bars.q, 0);
+    // The whole warp runs the issue loop converged, so the descriptors are
+    // warp-uniform (precomputed once; a 32-byte step along K adds 2 to the
+    // address field, a 16 KB tile step adds 1024); lane 0 alone executes the
+    // tcgen05 instructions.
+    const uint32_t leader = lane == 0 ? 1u : 0u;
+    auto mwait = [&](uint64_t *bar, uint32_t parity) -> bool {
+      const bool w = wait(bar, parity);
+      return __all_sync(0xFFFFFFFFu, w);
+    };
+    const uint64_t dQ = desc128(sQ), dK = desc128(sK), dV = desc128(sV), dE = desc128(sE);
+    const uint64_t dAr = desc128(sAr), dMu = desc128(sMu);
+    constexpr uint64_t KSTEP = 32 >> 4, TSTEP = SZ_TILE8 >> 4;
+    bool ok = mwait(&bars.q, 0);
+    tc_fence_after();
+    auto issue_qk = [&](int t) -> bool {
+      const int s = t % KS;
+      if (!mwait(&bars.kvfull[s], (t / KS) & 1)) return false;
       tc_fence_after();
-      auto issue_qk = [&](int t) -> bool {
-        const int s = t % KS;
-        if (!wait(&bars.kfull[s], (t / KS) & 1)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + TM_S0 + (t & 1) * 128;
+      const uint32_t d = tmem + TM_S0 + (t & 1) * 128;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f8_ss(d, desc128(sQ + 32 * kk), desc128(sK + s * SZ_TILE8 + 32 * kk), IDESC_QK, kk > 0);
-        mma_commit(&bars.kempty[s]);
-        mma_commit(&bars.sfull[t & 1]);
-        return true;
-      };
-      auto issue_restore = [&](int X) -> bool {
-        const int s = X & 1;
-        if (!wait(&bars.mufull[s], (X >> 1) & 1)) return false;
-        tc_fence_after();
+      for (int kk = 0; kk < 4; ++kk)
+        mma_f8_ss_el(d, dQ + KSTEP * kk, dK + TSTEP * s + KSTEP * kk, IDESC_QK, kk > 0, leader);
+      mma_commit_el(&bars.kempty[s], leader);
+      mma_commit_el(&bars.sfull[t & 1], leader);
+      return true;
+    };
+    auto issue_restore = [&](int X) -> bool {
+      const int s = X & 1;
+      if (!mwait(&bars.mufull[s], (X >> 1) & 1)) return false;
+      tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f16_ss(tmem + TM_O, desc128(sAr + 32 * kk), desc128(sMu + s * SZ_TILE8 + 32 * kk), IDESC_BF, 1);
-        mma_commit(&bars.muempty[s]);
-        return true;
-      };
-      if (ok) ok = issue_qk(0);
-      if (ok && T > 1) ok = issue_qk(1);
-      for (int t = 0; t < T && ok; ++t) {
-        ok = wait(&bars.pfull[t & 1], (t >> 1) & 1);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_f16_ss_el(tmem + TM_O, dAr + KSTEP * kk, dMu + TSTEP * s + KSTEP * kk, IDESC_BF, 1, leader);
+      mma_commit_el(&bars.muempty[s], leader);
+      return true;
+    };
+    if (ok) ok = issue_qk(0);
+    if (ok && T > 1) ok = issue_qk(1);
+    for (int t = 0; t < T && ok; ++t) {
+      ok = mwait(&bars.pfull[t & 1], (t >> 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      if (t >= 33 && ((t - 33) & 31) == 0) {
+        ok = issue_restore((t - 33) >> 5);
         if (!ok) break;
-        tc_fence_after();
-        if (t >= 33 && ((t - 33) & 31) == 0) {
-          ok = issue_restore((t - 33) >> 5);
-          if (!ok) break;
-        }
-        const int s = t % KS;
-        ok = wait(&bars.vfull[s], (t / KS) & 1);
-        if (!ok) break;
-        tc_fence_after();
-        const uint8_t *pa = sP + (t & 1) * SZ_TILE8;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f8_ss(tmem + TM_O, desc128(pa + 32 * kk), desc128(sV + s * SZ_TILE8 + 32 * kk), IDESC_QK,
-                    (t > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f8_ss(tmem + TM_L + 16 * (t & 1), desc128(pa + 32 * kk), desc128(sE + 32 * kk), IDESC_L, kk > 0);
-        mma_commit(&bars.vempty[s]);
-        mma_commit(&bars.pvdone);
-        if (t + 2 < T) ok = issue_qk(t + 2);
       }
-      if (ok) mma_commit(&bars.main);
-      // the restore chunks flushed after the loop, in order
-      for (int X = X_epi0, e = 0; X <= X_epi1 && ok; ++X, ++e) {
-        ok = wait(&bars.epi, e & 1);
-        if (!ok) break;
-        tc_fence_after();
-        ok = issue_restore(X);
-        if (ok) mma_commit(&bars.rdone);
-      }
-      for (int rc = 0; rc < nrc && ok; ++rc) {
-        ok = wait(&bars.repk, rc & 1);
-        if (!ok) break;
-        tc_fence_after();
+      // V(t) arrived with K(t), which issue_qk(t) waited for
+      const int s = t % KS;
+      const uint32_t pa = tmem + TM_P + 32 * (t & 1);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f8_ss(tmem + TM_S0, desc128(sQ + 32 * kk), desc128(sV + 32 * kk), IDESC_QK, kk > 0);
-        mma_commit(&bars.reps);
-        ok = wait(&bars.repp, rc & 1) && wait(&bars.dt, rc & 1);
-        if (!ok) break;
-        tc_fence_after();
+      for (int kk = 0; kk < 4; ++kk)
+        mma_f8_ts_el(tmem + TM_O, pa + 8 * kk, dV + TSTEP * s + KSTEP * kk, IDESC_QK, (t > 0 || kk > 0) ? 1u : 0u,
+                     leader);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_f16_ss(tmem + TM_O, desc128(sP + (kk >> 2) * SZ_TILE8 + 32 * (kk & 3)),
-                     desc128(sK + (kk >> 2) * SZ_TILE8 + 32 * (kk & 3)), IDESC_BF, 1);
-        mma_commit(&bars.repdone);
-      }
-      if (ok) mma_commit(&bars.fin);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_f8_ts_el(tmem + TM_L + 16 * (t & 1), pa + 8 * kk, dE + KSTEP * kk, IDESC_L, kk > 0, leader);
+      mma_commit_el(&bars.vempty[s], leader);
+      mma_commit_el(&bars.pvdone, leader);
+      if (t + 2 < T) ok = issue_qk(t + 2);
     }
+    if (ok) mma_commit_el(&bars.main, leader);
+    // the restore chunks flushed after the loop, in order
+    for (int X = X_epi0, e = 0; X <= X_epi1 && ok; ++X, ++e) {
+      ok = mwait(&bars.epi, e & 1);
+      if (!ok) break;
+      tc_fence_after();
+      ok = issue_restore(X);
+      if (ok) mma_commit_el(&bars.rdone, leader);
+    }
+    for (int rc = 0; rc < nrc && ok; ++rc) {
+      ok = mwait(&bars.repk, rc & 1);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_f8_ss_el(tmem + TM_S0, dQ + KSTEP * kk, dV + KSTEP * kk, IDESC_QK, kk > 0, leader);
+      mma_commit_el(&bars.reps, leader);
+      ok = mwait(&bars.repp, rc & 1) && mwait(&bars.dt, rc & 1);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_f16_ss_el(tmem + TM_O, dV + TSTEP * (1 + (kk >> 2)) + KSTEP * (kk & 3),
+                      dK + TSTEP * (kk >> 2) + KSTEP * (kk & 3), IDESC_BF, 1, leader);
+      mma_commit_el(&bars.repdone, leader);
+    }
+    if (ok) mma_commit_el(&bars.fin, leader);
   } else {
     // ------------------------------------------------------------ softmax rows
     // Warpgroup g (warps 2+4g .. 5+4g) takes the tiles t with t % 2 == g;
@@ -374,30 +429,26 @@ __global__ void __launch_bounds__(320, 1)
       s_m[r] = m;  // for tile t+1 (after the last tile, s_F holds the final frame)
       s_F[r] = Fn;
       if (t + 1 < T) mbar_arrive(&bars.mxr[b]);
-      // bytes against the frame Fn, to P buffer t&1 (its previous reader
-      // PV(t-2) completed before S(t) was signalled)
+      // bytes against the frame Fn, to the TMEM P buffer t&1 (its previous
+      // readers PV(t-2) / L(t-2) completed before S(t) was signalled): one
+      // 32-column store of the row's 128 bytes, 4 per column
       {
         const float al24 = alpha * TWO_M24;
         const float c24 = (static_cast<float>(p.C) - Fn) * TWO_M24;
-        uint8_t *prow = sP + b * SZ_TILE8;
+        uint32_t w[32];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t w[4];
+        for (int q = 0; q < 32; ++q) w[q] = expcast4(&s[4 * q], al24, c24);
+        if constexpr (LAST) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) w[q] = expcast4(&s[16 * ch + 4 * q], al24, c24);
-          if constexpr (LAST) {
+          for (int q = 0; q < 32; ++q) {
+            uint32_t keep = 0u;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int j0 = 16 * ch + 4 * q;
-              uint32_t keep = 0u;
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (j0 + e < tail) keep |= 0xFFu << (8 * e);
-              w[q] &= keep;
-            }
+            for (int e = 0; e < 4; ++e)
+              if (4 * q + e < tail) keep |= 0xFFu << (8 * e);
+            w[q] &= keep;
           }
-          *reinterpret_cast<uint4 *>(prow + sw128_off(r, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        tmem_st32(trow + TM_P + 32 * b, w);
       }
       // tail, in tile order after tile t-1's tail
       if (t > 0 && !wwait(&bars.tdone[(t - 1) & 1], ((t - 1) >> 1) & 1)) return false;
@@ -433,6 +484,7 @@ __global__ void __launch_bounds__(320, 1)
       s_ltot[r] = lt;
       F_own = Fn;
       F_hand = F_prev;
+      tmem_wait_st();  // the P bytes (and any O rescale) are in TMEM
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars.tdone[b]);
@@ -533,7 +585,7 @@ __global__ void __launch_bounds__(320, 1)
             outw[e] = *reinterpret_cast<const uint32_t *>(&pb);
           }
           const int jj = 32 * q + 8 * gg;  // first key of this 16-byte chunk
-          *reinterpret_cast<uint4 *>(sP + (jj >> 6) * SZ_TILE8 + sw128_off(r, (jj & 63) >> 3)) =
+          *reinterpret_cast<uint4 *>(sV + SZ_TILE8 + (jj >> 6) * SZ_TILE8 + sw128_off(r, (jj & 63) >> 3)) =
               make_uint4(outw[0], outw[1], outw[2], outw[3]);
         }
       }

@@ -432,7 +432,7 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
   ap.k8 = k8;
   ap.O = static_cast<uint16_t *>(O);
   ap.status = w.at<uint32_t>(w.L.status);
-  k_vc_attn_fwd<<<dim3(sh.Nb, sh.BH), 320, attn_fp8_smem_bytes(), s>>>(tq, tk, tv, tmu, tdt, ap);
+  k_vc_attn_fwd<<<dim3(sh.Nb, sh.BH), 352, attn_fp8_smem_bytes(), s>>>(tq, tk, tv, tmu, tdt, ap);
   count_launch();
   prof_mark(4, s);
   if (g_prof.on) ++g_prof.calls;

@@ -10,10 +10,15 @@
 // "Le compromis entre vitesse et fidélité": repair of the worst tokens.
 //
 // One CTA per (128-query tile, b*h). Warp roles:
-//   warp 0     TMA producer: Q once; K8 / V8 tiles through 4-stage rings; the
-//              bf16 block-mean tiles (one per 32 KV tiles); repair deltas.
-//   warp 1     allocates TMEM; lane 0 issues every tcgen05.mma and commit.
-//   warps 2-9  two warpgroups that take the KV tiles in turn (tile t goes to
+//   warp 0     TMA producers: lane 0 Q once, the K8 tiles through a 4-stage
+//              ring, then the repair deltas; lane 1 the V8 tiles through a
+//              4-stage ring and the bf16 block-mean tiles (one per 32 KV tiles).
+//   warp 1     allocates TMEM; issues PV, the row sums, the block-mean
+//              restores and the repair products.
+//   warp 2     issues QK^T. Two issuing warps keep the tensor pipe fed: a wait
+//              by one of them (~100 cycles even on a completed barrier while
+//              MMAs run) overlaps the other's MMAs.
+//   warps 3-10 two warpgroups that take the KV tiles in turn (tile t goes to
 //              warpgroup t % 2), one thread per query row holding the whole
 //              row of its tile: scores, running max, frame, ExpCast bytes,
 //              O rescale when the frame moves, row-sum bookkeeping; at the end
@@ -23,11 +28,13 @@
 // two row-sum slots of 16 columns at [384,416); the probability bytes P, double
 // buffered, 32 columns each (4 bytes per column) at [416,480), read by the PV
 // and row-sum MMAs as their A operand straight from TMEM. Per KV tile t the MMA issuer
-// runs O += P(t) V8(t), L[t%2] = P(t) E and S(t+2) = Q8 K8(t+2)^T, where E is
-// a constant block whose first row is all ones: column 0 of the slot receives
-// l_t = sum_j p_tj of the decoded bytes, overwritten (not accumulated). The
-// warpgroup of tile t reads l_t when it starts tile t+2: the commit that
-// signals S(t+2) also covers every earlier MMA.
+// runs S(t+2) = Q8 K8(t+2)^T as soon as the warpgroup of tile t has read S(t)
+// out of the buffer, then O += P(t) V8(t) and L[t%2] = P(t) E once the bytes
+// are in, where E is a constant block whose first row is all ones: column 0
+// of the slot receives l_t = sum_j p_tj of the decoded bytes, overwritten (not
+// accumulated). pvdone[t%2] signals that PV(t) and L(t) are complete: the
+// warpgroup waits for it in tile t+2 before it reuses the P buffer and reads
+// l_t out of the slot.
 // O is kept in "code units": O_acc = sum p * code + sum_t l_t * mean_t/s + sum_R
 // p * delta/s, and the epilogue writes O = s_c * O_acc / l.
 #include "common.cuh"
@@ -63,8 +70,9 @@ constexpr uint32_t IDESC_L = idesc_make(0, 0, 128, 16, false, false);    // row-
 constexpr uint32_t IDESC_BF = idesc_make(1, 1, 128, 128, false, false);  // bf16 x bf16 -> f32
 
 struct Bars {
-  uint64_t q, kvfull[KS], kempty[KS], vempty[VS], mufull[2], muempty[2];
-  uint64_t sfull[2], pfull[2], mxr[2], tdone[2], pvdone, main, epi, rdone, repk, reps, repp, repdone, dt, fin;
+  uint64_t q, kfull[KS], kempty[KS], vfull[VS], vempty[VS], mufull[2], muempty[2];
+  uint64_t sfull[2], sfree[2], pfull[2], mxr[2], tdone[2], pvdone[2], main, epi, rdone, repk, reps, repp, repdone, dt,
+      fin;
 };
 
 __device__ __forceinline__ uint64_t desc128(const uint8_t *p) { return sdesc_sw128(smem_u32(p), 16, 1024); }
@@ -80,39 +88,14 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
-// The MMA issuer warp runs converged; these execute the tcgen05 instruction
-// only where `leader` is nonzero (one elected lane), so every operand can be
-// computed once per warp in uniform registers.
-__device__ __forceinline__ void mma_f8_ss_el(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc,
-                                             uint32_t leader) {
+// One lane of a converged warp, chosen by elect.sync: the tcgen05 MMA groups
+// are issued under this predicate so that the warp stays converged around them.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
   asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
-      "@q tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(leader)
-      : "memory");
-}
-__device__ __forceinline__ void mma_f8_ts_el(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc,
-                                             uint32_t leader) {
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
-      "@q tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(leader)
-      : "memory");
-}
-__device__ __forceinline__ void mma_f16_ss_el(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc,
-                                              uint32_t leader) {
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
-      "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(leader)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit_el(uint64_t *bar, uint32_t leader) {
-  asm volatile(
-      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
-      "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar)),
-      "r"(leader)
-      : "memory");
+      "{\n\t.reg .b32 rx;\n\t.reg .pred px;\n\telect.sync rx|px, 0xffffffff;\n\t@px mov.s32 %0, 1;\n\t}"
+      : "+r"(pred));
+  return pred != 0;
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -138,7 +121,7 @@ __device__ __forceinline__ int first_epilogue_chunk(int T) { return T >= 34 ? (T
 
 }  // namespace
 
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     k_vc_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmMu,
                   const __grid_constant__ CUtensorMap tmDT, const AttnFp8Params p) {
@@ -168,22 +151,26 @@ __global__ void __launch_bounds__(320, 1)
     s_abort = 0;
     mbar_init(&bars.q, 1);
     for (int i = 0; i < KS; ++i) {
-      mbar_init(&bars.kvfull[i], 1);
+      mbar_init(&bars.kfull[i], 1);
       mbar_init(&bars.kempty[i], 1);
+    }
+    for (int i = 0; i < VS; ++i) {
+      mbar_init(&bars.vfull[i], 1);
       mbar_init(&bars.vempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.mufull[i], 1); mbar_init(&bars.muempty[i], 1);
-      mbar_init(&bars.sfull[i], 1); mbar_init(&bars.pfull[i], 128);
-      mbar_init(&bars.mxr[i], 128); mbar_init(&bars.tdone[i], 128);
+      mbar_init(&bars.sfull[i], 1); mbar_init(&bars.sfree[i], 128); mbar_init(&bars.pfull[i], 128);
+      mbar_init(&bars.mxr[i], 128); mbar_init(&bars.tdone[i], 128); mbar_init(&bars.pvdone[i], 1);
     }
-    mbar_init(&bars.pvdone, 1); mbar_init(&bars.main, 1); mbar_init(&bars.epi, 128); mbar_init(&bars.rdone, 1);
+    mbar_init(&bars.main, 2);  // one commit from each issuing warp
+    mbar_init(&bars.epi, 128); mbar_init(&bars.rdone, 1);
     mbar_init(&bars.repk, 128); mbar_init(&bars.reps, 1); mbar_init(&bars.repp, 128);
     mbar_init(&bars.repdone, 1); mbar_init(&bars.dt, 1); mbar_init(&bars.fin, 1);
     fence_mbar_init();
   }
-  if (warp >= 2) {
-    const int t = threadIdx.x - 64;  // 0..255
+  if (warp >= 3) {
+    const int t = threadIdx.x - 96;  // 0..255
     // E: rows 0..15 of a K-major, 128-byte-swizzled B operand; row 0 = 1.0 (0x38)
     if (t < 128) {
       const int rr = t >> 3, ch = t & 7;
@@ -198,7 +185,10 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = s_tmem;
 
+  // One try_wait on the fast path; the abort flag (set by a warp whose wait
+  // ran out) is read only when the phase is not complete yet.
   auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+    if (mbar_try_wait(smem_u32(bar), parity)) return true;
     if (s_abort) return false;
     if (!mbar_wait(bar, parity)) {
       s_abort = 1;
@@ -210,27 +200,20 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Lane 0 streams Q and the K tiles (then the repair deltas), lane 1 the V
+    // tiles and the block-mean chunks: a K stage is freed by QK(t), long before
+    // the V stage of the same tile is freed by PV(t).
     if (lane == 0) {
-      prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmMu);
+      prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmDT);
       mbar_arrive_expect_tx(&bars.q, SZ_TILE8);
       tma_load_2d(sQ, &tmQ, &bars.q, 0, bh * p.Npad + qt * 128);
       bool ok = true;
       for (int t = 0; t < T && ok; ++t) {
-        if ((t & 31) == 0) {
-          const int X = t >> 5, s = X & 1;
-          ok = wait(&bars.muempty[s], ((X >> 1) & 1) ^ 1);
-          if (!ok) break;
-          mbar_arrive_expect_tx(&bars.mufull[s], SZ_TILE8);
-          tma_load_2d(sMu + s * SZ_TILE8, &tmMu, &bars.mufull[s], 0, (bh * p.nch32 + X) * 128);
-        }
         const int s = t % KS;
-        const uint32_t ph = (t / KS) & 1;
-        ok = wait(&bars.kempty[s], ph ^ 1) && wait(&bars.vempty[s], ph ^ 1);
+        ok = wait(&bars.kempty[s], ((t / KS) & 1) ^ 1);
         if (!ok) break;
-        // K(t) and V(t) on one barrier: the issuer waits once, before QK(t)
-        mbar_arrive_expect_tx(&bars.kvfull[s], 2 * SZ_TILE8);
-        tma_load_2d(sK + s * SZ_TILE8, &tmK, &bars.kvfull[s], 0, bh * p.Npad + t * 128);
-        tma_load_2d(sV + s * SZ_TILE8, &tmV, &bars.kvfull[s], t * 128, bh * 128);
+        mbar_arrive_expect_tx(&bars.kfull[s], SZ_TILE8);
+        tma_load_2d(sK + s * SZ_TILE8, &tmK, &bars.kfull[s], 0, bh * p.Npad + t * 128);
       }
       if (ok && nrc > 0) {
         ok = wait(&bars.main, 0);
@@ -242,14 +225,29 @@ __global__ void __launch_bounds__(320, 1)
           tma_load_2d(sK + SZ_TILE8, &tmDT, &bars.dt, rc * 128 + 64, bh * 128);
         }
       }
+    } else if (lane == 1) {
+      prefetch_tmap(&tmV); prefetch_tmap(&tmMu);
+      bool ok = true;
+      for (int t = 0; t < T && ok; ++t) {
+        if ((t & 31) == 0) {
+          const int X = t >> 5, s = X & 1;
+          ok = wait(&bars.muempty[s], ((X >> 1) & 1) ^ 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bars.mufull[s], SZ_TILE8);
+          tma_load_2d(sMu + s * SZ_TILE8, &tmMu, &bars.mufull[s], 0, (bh * p.nch32 + X) * 128);
+        }
+        const int s = t % VS;
+        ok = wait(&bars.vempty[s], ((t / VS) & 1) ^ 1);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bars.vfull[s], SZ_TILE8);
+        tma_load_2d(sV + s * SZ_TILE8, &tmV, &bars.vfull[s], t * 128, bh * 128);
+      }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // The whole warp runs the issue loop converged, so the descriptors are
-    // warp-uniform (precomputed once; a 32-byte step along K adds 2 to the
-    // address field, a 16 KB tile step adds 1024); lane 0 alone executes the
-    // tcgen05 instructions.
-    const uint32_t leader = lane == 0 ? 1u : 0u;
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Both warps run converged; descriptors are warp-uniform (a 32-byte step
+    // along K adds 2 to the address field, a 16 KB tile step adds 1024), and
+    // each group of tcgen05 instructions is issued by one elected lane.
     auto mwait = [&](uint64_t *bar, uint32_t parity) -> bool {
       const bool w = wait(bar, parity);
       return __all_sync(0xFFFFFFFFu, w);
@@ -257,89 +255,113 @@ __global__ void __launch_bounds__(320, 1)
     const uint64_t dQ = desc128(sQ), dK = desc128(sK), dV = desc128(sV), dE = desc128(sE);
     const uint64_t dAr = desc128(sAr), dMu = desc128(sMu);
     constexpr uint64_t KSTEP = 32 >> 4, TSTEP = SZ_TILE8 >> 4;
-    bool ok = mwait(&bars.q, 0);
-    tc_fence_after();
-    auto issue_qk = [&](int t) -> bool {
-      const int s = t % KS;
-      if (!mwait(&bars.kvfull[s], (t / KS) & 1)) return false;
-      tc_fence_after();
-      const uint32_t d = tmem + TM_S0 + (t & 1) * 128;
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f8_ss_el(d, dQ + KSTEP * kk, dK + TSTEP * s + KSTEP * kk, IDESC_QK, kk > 0, leader);
-      mma_commit_el(&bars.kempty[s], leader);
-      mma_commit_el(&bars.sfull[t & 1], leader);
-      return true;
-    };
-    auto issue_restore = [&](int X) -> bool {
-      const int s = X & 1;
-      if (!mwait(&bars.mufull[s], (X >> 1) & 1)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f16_ss_el(tmem + TM_O, dAr + KSTEP * kk, dMu + TSTEP * s + KSTEP * kk, IDESC_BF, 1, leader);
-      mma_commit_el(&bars.muempty[s], leader);
-      return true;
-    };
-    if (ok) ok = issue_qk(0);
-    if (ok && T > 1) ok = issue_qk(1);
-    for (int t = 0; t < T && ok; ++t) {
-      ok = mwait(&bars.pfull[t & 1], (t >> 1) & 1);
-      if (!ok) break;
-      tc_fence_after();
-      if (t >= 33 && ((t - 33) & 31) == 0) {
-        ok = issue_restore((t - 33) >> 5);
+    bool ok = true;
+    if (warp == 2) {
+      // S(t) = Q8 K8(t)^T into S buffer t%2, once the warpgroup of tile t-2
+      // has read S(t-2) out of it
+      ok = mwait(&bars.q, 0);
+      for (int t = 0; t < T && ok; ++t) {
+        const int s = t % KS;
+        if (t >= 2) ok = mwait(&bars.sfree[t & 1], ((t - 2) >> 1) & 1);
+        ok = ok && mwait(&bars.kfull[s], (t / KS) & 1);
         if (!ok) break;
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t d = tmem + TM_S0 + (t & 1) * 128;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) mma_f8_ss(d, dQ + KSTEP * kk, dK + TSTEP * s + KSTEP * kk, IDESC_QK, kk > 0);
+          mma_commit(&bars.kempty[s]);
+          mma_commit(&bars.sfull[t & 1]);
+        }
+        __syncwarp();
       }
-      // V(t) arrived with K(t), which issue_qk(t) waited for
-      const int s = t % KS;
-      const uint32_t pa = tmem + TM_P + 32 * (t & 1);
+      if (ok && elect_one()) mma_commit(&bars.main);
+      __syncwarp();
+    } else {
+      auto issue_restore = [&](int X) -> bool {
+        const int s = X & 1;
+        if (!mwait(&bars.mufull[s], (X >> 1) & 1)) return false;
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f8_ts_el(tmem + TM_O, pa + 8 * kk, dV + TSTEP * s + KSTEP * kk, IDESC_QK, (t > 0 || kk > 0) ? 1u : 0u,
-                     leader);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16_ss(tmem + TM_O, dAr + KSTEP * kk, dMu + TSTEP * s + KSTEP * kk, IDESC_BF, 1);
+          mma_commit(&bars.muempty[s]);
+        }
+        __syncwarp();
+        return true;
+      };
+      for (int t = 0; t < T && ok; ++t) {
+        ok = mwait(&bars.pfull[t & 1], (t >> 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (t >= 33 && ((t - 33) & 31) == 0) {
+          ok = issue_restore((t - 33) >> 5);
+          if (!ok) break;
+        }
+        const int s = t % VS;
+        ok = mwait(&bars.vfull[s], (t / VS) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t pa = tmem + TM_P + 32 * (t & 1);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f8_ts_el(tmem + TM_L + 16 * (t & 1), pa + 8 * kk, dE + KSTEP * kk, IDESC_L, kk > 0, leader);
-      mma_commit_el(&bars.vempty[s], leader);
-      mma_commit_el(&bars.pvdone, leader);
-      if (t + 2 < T) ok = issue_qk(t + 2);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f8_ts(tmem + TM_O, pa + 8 * kk, dV + TSTEP * s + KSTEP * kk, IDESC_QK, (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f8_ts(tmem + TM_L + 16 * (t & 1), pa + 8 * kk, dE + KSTEP * kk, IDESC_L, kk > 0);
+          mma_commit(&bars.vempty[s]);
+          mma_commit(&bars.pvdone[t & 1]);
+        }
+        __syncwarp();
+      }
+      if (ok && elect_one()) mma_commit(&bars.main);
+      __syncwarp();
+      // the restore chunks flushed after the loop, in order
+      for (int X = X_epi0, e = 0; X <= X_epi1 && ok; ++X, ++e) {
+        ok = mwait(&bars.epi, e & 1);
+        if (!ok) break;
+        tc_fence_after();
+        ok = issue_restore(X);
+        if (ok && elect_one()) mma_commit(&bars.rdone);
+        __syncwarp();
+      }
+      // repair: the warpgroup's K rows and bf16 probabilities arrive after
+      // `main`, so every QK^T and PV of the loop has completed
+      for (int rc = 0; rc < nrc && ok; ++rc) {
+        ok = mwait(&bars.repk, rc & 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tmem + TM_S0, dQ + KSTEP * kk, dV + KSTEP * kk, IDESC_QK, kk > 0);
+          mma_commit(&bars.reps);
+        }
+        __syncwarp();
+        ok = mwait(&bars.repp, rc & 1) && mwait(&bars.dt, rc & 1);
+        if (!ok) break;
+        tc_fence_after();
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_f16_ss(tmem + TM_O, dV + TSTEP * (1 + (kk >> 2)) + KSTEP * (kk & 3),
+                       dK + TSTEP * (kk >> 2) + KSTEP * (kk & 3), IDESC_BF, 1);
+          mma_commit(&bars.repdone);
+        }
+        __syncwarp();
+      }
+      if (ok && elect_one()) mma_commit(&bars.fin);
+      __syncwarp();
     }
-    if (ok) mma_commit_el(&bars.main, leader);
-    // the restore chunks flushed after the loop, in order
-    for (int X = X_epi0, e = 0; X <= X_epi1 && ok; ++X, ++e) {
-      ok = mwait(&bars.epi, e & 1);
-      if (!ok) break;
-      tc_fence_after();
-      ok = issue_restore(X);
-      if (ok) mma_commit_el(&bars.rdone, leader);
-    }
-    for (int rc = 0; rc < nrc && ok; ++rc) {
-      ok = mwait(&bars.repk, rc & 1);
-      if (!ok) break;
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f8_ss_el(tmem + TM_S0, dQ + KSTEP * kk, dV + KSTEP * kk, IDESC_QK, kk > 0, leader);
-      mma_commit_el(&bars.reps, leader);
-      ok = mwait(&bars.repp, rc & 1) && mwait(&bars.dt, rc & 1);
-      if (!ok) break;
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_f16_ss_el(tmem + TM_O, dV + TSTEP * (1 + (kk >> 2)) + KSTEP * (kk & 3),
-                      dK + TSTEP * (kk >> 2) + KSTEP * (kk & 3), IDESC_BF, 1, leader);
-      mma_commit_el(&bars.repdone, leader);
-    }
-    if (ok) mma_commit_el(&bars.fin, leader);
   } else {
     // ------------------------------------------------------------ softmax rows
-    // Warpgroup g (warps 2+4g .. 5+4g) takes the tiles t with t % 2 == g;
+    // Warpgroup g (warps 3+4g .. 6+4g) takes the tiles t with t % 2 == g;
     // thread row r = 32*(warp%4) + lane. Shared per-row state, handed from
     // tile to tile in order: s_m / s_F (running max and frame; mxr[t%2]) and
     // s_ltot / sLb (row sum and staged l_t, both in the current frame;
     // tdone[t%2]).
-    const int g = (warp - 2) >> 2;
+    const int g = (warp - 3) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
@@ -386,14 +408,13 @@ __global__ void __launch_bounds__(320, 1)
       if (t + 2 < T) sk_next = skh[t + 2];  // this warpgroup's next tile
       if (!wwait(&bars.sfull[b], (t >> 1) & 1)) return false;
       tc_fence_after();
-      // S(t) and, from the row-sum slot this tile reuses, l_{t-2} (complete:
-      // the commit behind sfull covers every earlier MMA)
       uint32_t sr[128];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         tmem_ld32(trow + TM_S0 + b * 128 + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * i]));
-      const uint32_t lraw = tmem_ld1(trow + TM_L + 16 * b);
       tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars.sfree[b]);  // the issuer may now compute S(t+2) into this buffer
       float s[128];
 #pragma unroll
       for (int j = 0; j < 128; ++j) s[j] = __uint_as_float(sr[j]);
@@ -429,9 +450,16 @@ __global__ void __launch_bounds__(320, 1)
       s_m[r] = m;  // for tile t+1 (after the last tile, s_F holds the final frame)
       s_F[r] = Fn;
       if (t + 1 < T) mbar_arrive(&bars.mxr[b]);
-      // bytes against the frame Fn, to the TMEM P buffer t&1 (its previous
-      // readers PV(t-2) / L(t-2) completed before S(t) was signalled): one
-      // 32-column store of the row's 128 bytes, 4 per column
+      // P buffer t&1 and row-sum slot t&1 were last used by PV(t-2) and
+      // L(t-2): wait for them, then take l_{t-2} from the slot
+      uint32_t lraw = 0u;
+      if (t >= 2) {
+        if (!wwait(&bars.pvdone[b], ((t - 2) >> 1) & 1)) return false;
+        tc_fence_after();
+        lraw = tmem_ld1(trow + TM_L + 16 * b);
+      }
+      // bytes against the frame Fn: one 32-column store of the row's 128
+      // bytes, 4 per column
       {
         const float al24 = alpha * TWO_M24;
         const float c24 = (static_cast<float>(p.C) - Fn) * TWO_M24;
@@ -456,7 +484,7 @@ __global__ void __launch_bounds__(320, 1)
       const float sc = need ? frame_scale(F_prev, Fn) : 1.0f;
       if (__any_sync(0xFFFFFFFFu, need)) {
         // O holds PV(0..t-1) in frame F_prev: rescale it before PV(t)
-        if (!wwait(&bars.pvdone, (t - 1) & 1)) return false;
+        if (!wwait(&bars.pvdone[(t - 1) & 1], ((t - 1) >> 1) & 1)) return false;
         tc_fence_after();
         uint32_t o[128];
 #pragma unroll
@@ -473,6 +501,7 @@ __global__ void __launch_bounds__(320, 1)
           for (int sl = 0; sl < 32; ++sl) sLb[sl * 128 + r] *= sc;
       }
       float lt = (t > 0 ? s_ltot[r] : 0.0f) * sc;
+      tmem_wait_ld();  // lraw
       if (t >= 2) {
         // l_{t-2}: this warpgroup's previous tile, computed in frame F_own
         const float lo = __uint_as_float(lraw) * frame_scale(F_own, Fn);

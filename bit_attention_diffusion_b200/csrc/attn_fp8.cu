@@ -24,17 +24,18 @@
 //              O rescale when the frame moves, row-sum bookkeeping; at the end
 //              the last tile's warpgroup does the final restore and the repair,
 //              and both write the output.
-// TMEM (512 columns x 128 lanes): S double buffer at [0,256); O at [256,384);
-// two row-sum slots of 16 columns at [384,416); the probability bytes P, double
-// buffered, 32 columns each (4 bytes per column) at [416,480), read by the PV
-// and row-sum MMAs as their A operand straight from TMEM. Per KV tile t the MMA issuer
-// runs S(t+2) = Q8 K8(t+2)^T as soon as the warpgroup of tile t has read S(t)
-// out of the buffer, then O += P(t) V8(t) and L[t%2] = P(t) E once the bytes
-// are in, where E is a constant block whose first row is all ones: column 0
-// of the slot receives l_t = sum_j p_tj of the decoded bytes, overwritten (not
-// accumulated). pvdone[t%2] signals that PV(t) and L(t) are complete: the
-// warpgroup waits for it in tile t+2 before it reuses the P buffer and reads
-// l_t out of the slot.
+// TMEM (512 columns x 128 lanes): S double buffer at [0,256); the odd-tile
+// row-sum column at 256; O at [272,400); the even-tile row-sum column at 400;
+// the probability bytes P, double buffered, 32 columns each (4 bytes per
+// column) at [416,480), read by the PV MMA as its A operand straight from
+// TMEM. The issuers run S(t) = Q8 K8(t)^T as soon as the warpgroup of tile t-2
+// has read S(t-2) out of the buffer, and PV(t) once the bytes are in. PV is
+// one N = 144 product: its B operand is the V tile plus a 16-row block E whose
+// first row is all ones, placed after V for even tiles (D = [O | l_even]) and
+// before V for odd tiles (D = [l_odd | O]), so each tile parity accumulates
+// l_t = sum_j p_tj of the decoded bytes into a column of its own. The
+// warpgroup of tile t reads l_{t-2} there once PV(t-2) is complete
+// (pvdone[(t-2)%4]) and resets it before PV(t).
 // O is kept in "code units": O_acc = sum p * code + sum_t l_t * mean_t/s + sum_R
 // p * delta/s, and the epilogue writes O = s_c * O_acc / l.
 #include "common.cuh"
@@ -51,28 +52,35 @@ namespace {
 constexpr int KS = 4;  // K ring stages
 constexpr int VS = 4;  // V ring stages
 constexpr uint32_t SZ_TILE8 = 128 * 128;  // one 128x128 byte tile
+constexpr uint32_t SZ_EBLK = 2048;         // 16 rows x 128 bytes: row 0 ones, rows 1-15 zero
+// V ring: [V0][E][V1][V2][E][V3]. The PV MMA of an even stage reads N = 144
+// rows V(128) + E(16) and writes [O | l_even]; an odd stage reads E(16) + V(128)
+// and writes [l_odd | O]: one E block serves both neighbours.
+__host__ __device__ constexpr uint32_t voff(int s) { return s * SZ_TILE8 + ((s + 1) >> 1) * SZ_EBLK; }
+constexpr uint32_t SZ_VRING = VS * SZ_TILE8 + (VS / 2) * SZ_EBLK;
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + SZ_TILE8;
 constexpr uint32_t OFF_V = OFF_K + KS * SZ_TILE8;
-constexpr uint32_t OFF_AR = OFF_V + VS * SZ_TILE8;
+constexpr uint32_t OFF_AR = OFF_V + SZ_VRING;
 constexpr uint32_t OFF_MU = OFF_AR + SZ_TILE8;
-constexpr uint32_t OFF_E = OFF_MU + 2 * SZ_TILE8;  // 16 x 128-byte ones/zero block
-constexpr uint32_t OFF_LB = OFF_E + 2048;
+constexpr uint32_t OFF_LB = OFF_MU + 2 * SZ_TILE8;
 constexpr uint32_t SMEM_USED = OFF_LB + 32 * 128 * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // alignment slack
-static_assert(OFF_AR % 1024 == 0 && OFF_MU % 1024 == 0 && OFF_E % 1024 == 0,
+static_assert(VS == 4 && voff(1) % 1024 == 0 && voff(3) % 1024 == 0 && OFF_AR % 1024 == 0 && OFF_MU % 1024 == 0,
               "tile alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_L = 384, TM_P = 416;
+// TMEM columns: S double buffer [0,256); l_odd at 256 (257..271 unused);
+// O [272,400); l_even at 400 (401..415 unused); P double buffer [416,480).
+constexpr uint32_t TM_S0 = 0, TM_LO = 256, TM_O = 272, TM_LE = 400, TM_P = 416;
 constexpr uint32_t IDESC_QK = idesc_make(0, 0, 128, 128, false, false);  // E4M3 x E4M3 -> f32, N = 128
-constexpr uint32_t IDESC_L = idesc_make(0, 0, 128, 16, false, false);    // row-sum MMA, N = 16
+constexpr uint32_t IDESC_PV = idesc_make(0, 0, 128, 144, false, false);  // PV with the row-sum rows, N = 144
 constexpr uint32_t IDESC_BF = idesc_make(1, 1, 128, 128, false, false);  // bf16 x bf16 -> f32
 
 struct Bars {
   uint64_t q, kfull[KS], kempty[KS], vfull[VS], vempty[VS], mufull[2], muempty[2];
-  uint64_t sfull[2], sfree[2], pfull[2], mxr[2], tdone[2], pvdone[2], main, epi, rdone, repk, reps, repp, repdone, dt,
-      fin;
+  uint64_t sfull[2], sfree[2], pfull[2], mxr[2], tdone[2], pvdone[4], lflush, main, epi, rdone, repk, reps, repp,
+      repdone, dt, fin;
 };
 
 __device__ __forceinline__ uint64_t desc128(const uint8_t *p) { return sdesc_sw128(smem_u32(p), 16, 1024); }
@@ -132,7 +140,6 @@ __global__ void __launch_bounds__(352, 1)
   uint8_t *sV = sm + OFF_V;
   uint8_t *sAr = sm + OFF_AR;
   uint8_t *sMu = sm + OFF_MU;
-  uint8_t *sE = sm + OFF_E;
   float *sLb = reinterpret_cast<float *>(sm + OFF_LB);  // [32 slots][128 rows]
   __shared__ Bars bars;
   __shared__ uint32_t s_tmem;
@@ -161,8 +168,10 @@ __global__ void __launch_bounds__(352, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.mufull[i], 1); mbar_init(&bars.muempty[i], 1);
       mbar_init(&bars.sfull[i], 1); mbar_init(&bars.sfree[i], 128); mbar_init(&bars.pfull[i], 128);
-      mbar_init(&bars.mxr[i], 128); mbar_init(&bars.tdone[i], 128); mbar_init(&bars.pvdone[i], 1);
+      mbar_init(&bars.mxr[i], 128); mbar_init(&bars.tdone[i], 128);
     }
+    for (int i = 0; i < 4; ++i) mbar_init(&bars.pvdone[i], 1);
+    mbar_init(&bars.lflush, 128);
     mbar_init(&bars.main, 2);  // one commit from each issuing warp
     mbar_init(&bars.epi, 128); mbar_init(&bars.rdone, 1);
     mbar_init(&bars.repk, 128); mbar_init(&bars.reps, 1); mbar_init(&bars.repp, 128);
@@ -171,13 +180,15 @@ __global__ void __launch_bounds__(352, 1)
   }
   if (warp >= 3) {
     const int t = threadIdx.x - 96;  // 0..255
-    // E: rows 0..15 of a K-major, 128-byte-swizzled B operand; row 0 = 1.0 (0x38)
-    if (t < 128) {
-      const int rr = t >> 3, ch = t & 7;
+    // the two E blocks of the V ring: rows 0..15 of a K-major, 128-byte-swizzled
+    // B operand; row 0 = 1.0 (0x38) for every key, rows 1..15 zero
+    {
+      const int rr = (t >> 3) & 15, ch = t & 7;
+      uint8_t *eblk = sV + voff(2 * (t >> 7)) + SZ_TILE8;
       const uint32_t v = rr == 0 ? 0x38383838u : 0u;
-      *reinterpret_cast<uint4 *>(sE + sw128_off(rr, ch)) = make_uint4(v, v, v, v);
-      s_vscale[t] = p.vscale[static_cast<size_t>(bh) * 128 + t];
+      *reinterpret_cast<uint4 *>(eblk + sw128_off(rr, ch)) = make_uint4(v, v, v, v);
     }
+    if (t < 128) s_vscale[t] = p.vscale[static_cast<size_t>(bh) * 128 + t];
     fence_proxy_async_smem();
   }
   if (warp == 1) tmem_alloc(&s_tmem, 512);
@@ -240,7 +251,7 @@ __global__ void __launch_bounds__(352, 1)
         ok = wait(&bars.vempty[s], ((t / VS) & 1) ^ 1);
         if (!ok) break;
         mbar_arrive_expect_tx(&bars.vfull[s], SZ_TILE8);
-        tma_load_2d(sV + s * SZ_TILE8, &tmV, &bars.vfull[s], t * 128, bh * 128);
+        tma_load_2d(sV + voff(s), &tmV, &bars.vfull[s], t * 128, bh * 128);
       }
     }
   } else if (warp == 1 || warp == 2) {
@@ -252,7 +263,7 @@ __global__ void __launch_bounds__(352, 1)
       const bool w = wait(bar, parity);
       return __all_sync(0xFFFFFFFFu, w);
     };
-    const uint64_t dQ = desc128(sQ), dK = desc128(sK), dV = desc128(sV), dE = desc128(sE);
+    const uint64_t dQ = desc128(sQ), dK = desc128(sK), dV = desc128(sV);
     const uint64_t dAr = desc128(sAr), dMu = desc128(sMu);
     constexpr uint64_t KSTEP = 32 >> 4, TSTEP = SZ_TILE8 >> 4;
     bool ok = true;
@@ -294,25 +305,31 @@ __global__ void __launch_bounds__(352, 1)
       for (int t = 0; t < T && ok; ++t) {
         ok = mwait(&bars.pfull[t & 1], (t >> 1) & 1);
         if (!ok) break;
-        tc_fence_after();
-        if (t >= 33 && ((t - 33) & 31) == 0) {
-          ok = issue_restore((t - 33) >> 5);
-          if (!ok) break;
-        }
         const int s = t % VS;
         ok = mwait(&bars.vfull[s], (t / VS) & 1);
         if (!ok) break;
         tc_fence_after();
         if (elect_one()) {
+          // even tile: B = V(t) + E, D = [O | l_even]; odd: B = E + V(t), D = [l_odd | O]
           const uint32_t pa = tmem + TM_P + 32 * (t & 1);
+          const uint32_t d = tmem + ((t & 1) ? TM_LO : TM_O);
+          const uint64_t bv = dV + ((voff(s) - (s & 1) * SZ_EBLK) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_f8_ts(tmem + TM_O, pa + 8 * kk, dV + TSTEP * s + KSTEP * kk, IDESC_QK, (t > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f8_ts(tmem + TM_L + 16 * (t & 1), pa + 8 * kk, dE + KSTEP * kk, IDESC_L, kk > 0);
+            mma_f8_ts(d, pa + 8 * kk, bv + KSTEP * kk, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
+        // block means of chunk X = (t-33)/32: their row sums were staged by the
+        // tail of tile t in the frame of tile t, which O holds right after PV(t)
+        if (t >= 33 && ((t - 33) & 31) == 0) {
+          const int X = (t - 33) >> 5;
+          ok = mwait(&bars.lflush, X & 1);
+          if (ok) ok = issue_restore(X);
+          if (!ok) break;
+        }
+        if (elect_one()) {
           mma_commit(&bars.vempty[s]);
-          mma_commit(&bars.pvdone[t & 1]);
+          mma_commit(&bars.pvdone[t & 3]);
         }
         __syncwarp();
       }
@@ -365,6 +382,7 @@ __global__ void __launch_bounds__(352, 1)
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const uint32_t lcol = g == 0 ? TM_LE : TM_LO;  // this warpgroup's row-sum column
     const float sqs = p.sq[static_cast<size_t>(bh) * T + qt];
     const float *skh = p.sk + static_cast<size_t>(bh) * T;
     const int tail = p.N - (T - 1) * 128;  // valid keys in the last tile
@@ -450,13 +468,18 @@ __global__ void __launch_bounds__(352, 1)
       s_m[r] = m;  // for tile t+1 (after the last tile, s_F holds the final frame)
       s_F[r] = Fn;
       if (t + 1 < T) mbar_arrive(&bars.mxr[b]);
-      // P buffer t&1 and row-sum slot t&1 were last used by PV(t-2) and
-      // L(t-2): wait for them, then take l_{t-2} from the slot
+      const bool need = Fn != F_prev;
+      const float sc = need ? frame_scale(F_prev, Fn) : 1.0f;
+      const bool anyneed = __any_sync(0xFFFFFFFFu, need);
+      // PV(t-2) is complete: P buffer t&1 is free, and this warpgroup's
+      // row-sum column holds l_{t-2} alone (reset here for l_t)
       uint32_t lraw = 0u;
       if (t >= 2) {
-        if (!wwait(&bars.pvdone[b], ((t - 2) >> 1) & 1)) return false;
+        if (!wwait(&bars.pvdone[(t - 2) & 3], ((t - 2) >> 2) & 1)) return false;
         tc_fence_after();
-        lraw = tmem_ld1(trow + TM_L + 16 * b);
+        lraw = tmem_ld1(trow + lcol);
+        tmem_wait_ld();
+        tmem_st1(trow + lcol, 0u);
       }
       // bytes against the frame Fn: one 32-column store of the row's 128
       // bytes, 4 per column
@@ -478,13 +501,9 @@ __global__ void __launch_bounds__(352, 1)
         }
         tmem_st32(trow + TM_P + 32 * b, w);
       }
-      // tail, in tile order after tile t-1's tail
-      if (t > 0 && !wwait(&bars.tdone[(t - 1) & 1], ((t - 1) >> 1) & 1)) return false;
-      const bool need = Fn != F_prev;
-      const float sc = need ? frame_scale(F_prev, Fn) : 1.0f;
-      if (__any_sync(0xFFFFFFFFu, need)) {
+      if (anyneed) {
         // O holds PV(0..t-1) in frame F_prev: rescale it before PV(t)
-        if (!wwait(&bars.pvdone[(t - 1) & 1], ((t - 1) >> 1) & 1)) return false;
+        if (!wwait(&bars.pvdone[(t - 1) & 3], ((t - 1) >> 2) & 1)) return false;
         tc_fence_after();
         uint32_t o[128];
 #pragma unroll
@@ -496,31 +515,43 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           tmem_st32(trow + TM_O + 32 * i, *reinterpret_cast<const uint32_t(*)[32]>(&o[32 * i]));
-        tmem_wait_st();
-        if (need)
-          for (int sl = 0; sl < 32; ++sl) sLb[sl * 128 + r] *= sc;
       }
+      tmem_wait_st();  // the P bytes, the column reset and any O rescale are in TMEM
+      tc_fence_before();
+      mbar_arrive(&bars.pfull[b]);
+      // row-sum bookkeeping, in tile order after tile t-1's
+      if (t > 0 && !wwait(&bars.tdone[(t - 1) & 1], ((t - 1) >> 1) & 1)) return false;
+      if (need)
+        for (int sl = 0; sl < 32; ++sl) sLb[sl * 128 + r] *= sc;
       float lt = (t > 0 ? s_ltot[r] : 0.0f) * sc;
-      tmem_wait_ld();  // lraw
+      bool flushed = false;
       if (t >= 2) {
         // l_{t-2}: this warpgroup's previous tile, computed in frame F_own
         const float lo = __uint_as_float(lraw) * frame_scale(F_own, Fn);
         const int slot = (t - 2) & 31;
         sLb[slot * 128 + r] = lo;
         lt += lo;
-        if (slot == 31) flush(32);
+        if (slot == 31) {
+          flush(32);
+          flushed = true;
+        }
       }
       s_ltot[r] = lt;
       F_own = Fn;
       F_hand = F_prev;
-      tmem_wait_st();  // the P bytes (and any O rescale) are in TMEM
-      fence_proxy_async_smem();
-      tc_fence_before();
+      if (flushed) {  // the restore of this chunk follows PV(t)
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars.lflush);
+      }
       mbar_arrive(&bars.tdone[b]);
-      mbar_arrive(&bars.pfull[b]);
       return true;
     };
 
+    // this warpgroup's row-sum column starts at zero: the first odd PV
+    // accumulates onto it (the first even PV overwrites)
+    tmem_st1(trow + lcol, 0u);
+    tmem_wait_st();
     const bool ragged = tail < 128;
     for (int t = g; t < T - 1 && ok; t += 2) ok = tile(t, std::false_type{});
     if (ok && ((T - 1) & 1) == g)
@@ -538,9 +569,9 @@ __global__ void __launch_bounds__(352, 1)
       float lt = s_ltot[r];
       int e = 0;
       for (int u = (T >= 2 ? T - 2 : 0); u <= T - 1; ++u) {
-        // l_u is in slot u%2, computed in frame F_{T-1} (own last tile) or
+        // l_u is in the row-sum column of parity u%2, computed in frame F_{T-1} (own last tile) or
         // F_{T-2} (the frame handed over to the last tile)
-        const float lu_raw = __uint_as_float(tmem_ld1(trow + TM_L + 16 * (u & 1)));
+        const float lu_raw = __uint_as_float(tmem_ld1(trow + ((u & 1) ? TM_LO : TM_LE)));
         tmem_wait_ld();
         const float lo = lu_raw * frame_scale(u == T - 1 ? F_own : F_hand, F_fin);
         const int slot = u & 31;

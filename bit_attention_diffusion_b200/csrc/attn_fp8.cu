@@ -13,7 +13,7 @@
 //   warp 0     TMA producers: lane 0 Q once, the K8 tiles through a 4-stage
 //              ring, then the repair deltas; lane 1 the V8 tiles through a
 //              4-stage ring and the bf16 block-mean tiles (one per 32 KV tiles).
-//   warp 1     allocates TMEM; issues PV, the row sums, the block-mean
+//   warp 1     allocates TMEM; issues PV (with the row sums), the block-mean
 //              restores and the repair products.
 //   warp 2     issues QK^T. Two issuing warps keep the tensor pipe fed: a wait
 //              by one of them (~100 cycles even on a completed barrier while
@@ -24,18 +24,18 @@
 //              O rescale when the frame moves, row-sum bookkeeping; at the end
 //              the last tile's warpgroup does the final restore and the repair,
 //              and both write the output.
-// TMEM (512 columns x 128 lanes): S double buffer at [0,256); the odd-tile
-// row-sum column at 256; O at [272,400); the even-tile row-sum column at 400;
-// the probability bytes P, double buffered, 32 columns each (4 bytes per
-// column) at [416,480), read by the PV MMA as its A operand straight from
-// TMEM. The issuers run S(t) = Q8 K8(t)^T as soon as the warpgroup of tile t-2
-// has read S(t-2) out of the buffer, and PV(t) once the bytes are in. PV is
-// one N = 144 product: its B operand is the V tile plus a 16-row block E whose
-// first row is all ones, placed after V for even tiles (D = [O | l_even]) and
-// before V for odd tiles (D = [l_odd | O]), so each tile parity accumulates
-// l_t = sum_j p_tj of the decoded bytes into a column of its own. The
-// warpgroup of tile t reads l_{t-2} there once PV(t-2) is complete
-// (pvdone[(t-2)%4]) and resets it before PV(t).
+// TMEM (512 columns x 128 lanes): S double buffer at [0,256); O at [272,400);
+// row-sum columns at 256, 257 (odd tiles) and 400, 401 (even tiles); the
+// probability bytes P in three slots of 32 columns (4 bytes per column) at
+// [416,512), read by the PV MMA as its A operand straight from TMEM. The
+// issuers run S(t) = Q8 K8(t)^T as soon as the warpgroup of tile t-2 has read
+// S(t-2) out of the buffer, and PV(t) once the bytes are in. PV is one N = 144
+// product: its B operand is the V tile plus a 16-row block E with one row of
+// ones, placed after V for even tiles (D = [O | 400..415]) and before V for
+// odd tiles (D = [256..271 | O]), so that l_t = sum_j p_tj of the decoded
+// bytes accumulates into column 400 + (t/2)%2 or 256 + (t/2)%2. The warpgroup
+// of tile t reads l_{t-2} there once PV(t-2) is complete (pvdone[(t-2)%8]),
+// after it has handed the bytes of tile t to the issuer.
 // O is kept in "code units": O_acc = sum p * code + sum_t l_t * mean_t/s + sum_R
 // p * delta/s, and the epilogue writes O = s_c * O_acc / l.
 #include "common.cuh"
@@ -70,17 +70,23 @@ static_assert(VS == 4 && voff(1) % 1024 == 0 && voff(3) % 1024 == 0 && OFF_AR % 
               "tile alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// TMEM columns: S double buffer [0,256); l_odd at 256 (257..271 unused);
-// O [272,400); l_even at 400 (401..415 unused); P double buffer [416,480).
+// TMEM columns: S double buffer [0,256); row sums of odd tiles at 256 + (t/2)%2
+// (258..271 unused); O [272,400); row sums of even tiles at 400 + (t/2)%2
+// (402..415 unused); P in three slots of 32 columns at [416,512). A row-sum
+// column accumulates l_t over the tiles t that map to it (every fourth tile);
+// the other PV products of its parity add exact zeros to it, so the value read
+// between PV(t) and PV(t+4) is stable and l_t is the difference of two reads.
 constexpr uint32_t TM_S0 = 0, TM_LO = 256, TM_O = 272, TM_LE = 400, TM_P = 416;
+constexpr int NPD = 8;  // PV completion barriers, indexed t % 8
+__device__ __forceinline__ uint32_t lcol_of(int t) { return ((t & 1) ? TM_LO : TM_LE) + ((t >> 1) & 1); }
 constexpr uint32_t IDESC_QK = idesc_make(0, 0, 128, 128, false, false);  // E4M3 x E4M3 -> f32, N = 128
 constexpr uint32_t IDESC_PV = idesc_make(0, 0, 128, 144, false, false);  // PV with the row-sum rows, N = 144
 constexpr uint32_t IDESC_BF = idesc_make(1, 1, 128, 128, false, false);  // bf16 x bf16 -> f32
 
 struct Bars {
   uint64_t q, kfull[KS], kempty[KS], vfull[VS], vempty[VS], mufull[2], muempty[2];
-  uint64_t sfull[2], sfree[2], pfull[2], mxr[2], tdone[2], pvdone[4], lflush, main, epi, rdone, repk, reps, repp,
-      repdone, dt, fin;
+  uint64_t sfull[2], sfree[2], pfull[2], mxr[2], pvdone[NPD], bk, lflush, wgdone, main, epi, rdone, repk, reps,
+      repp, repdone, dt, fin;
 };
 
 __device__ __forceinline__ uint64_t desc128(const uint8_t *p) { return sdesc_sw128(smem_u32(p), 16, 1024); }
@@ -146,7 +152,7 @@ __global__ void __launch_bounds__(352, 1)
   __shared__ volatile int s_abort;
   __shared__ float s_vscale[128];
   __shared__ float s_alphaR[128];
-  __shared__ float s_m[128], s_F[128], s_ltot[128];
+  __shared__ float s_F[128], s_ltot[128], s_lto[128], s_lprev[2][128];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, bh = blockIdx.y;
@@ -168,10 +174,10 @@ __global__ void __launch_bounds__(352, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.mufull[i], 1); mbar_init(&bars.muempty[i], 1);
       mbar_init(&bars.sfull[i], 1); mbar_init(&bars.sfree[i], 128); mbar_init(&bars.pfull[i], 128);
-      mbar_init(&bars.mxr[i], 128); mbar_init(&bars.tdone[i], 128);
+      mbar_init(&bars.mxr[i], 128);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&bars.pvdone[i], 1);
-    mbar_init(&bars.lflush, 128);
+    for (int i = 0; i < NPD; ++i) mbar_init(&bars.pvdone[i], 1);
+    mbar_init(&bars.bk, 128); mbar_init(&bars.lflush, 128); mbar_init(&bars.wgdone, 128);
     mbar_init(&bars.main, 2);  // one commit from each issuing warp
     mbar_init(&bars.epi, 128); mbar_init(&bars.rdone, 1);
     mbar_init(&bars.repk, 128); mbar_init(&bars.reps, 1); mbar_init(&bars.repp, 128);
@@ -181,11 +187,13 @@ __global__ void __launch_bounds__(352, 1)
   if (warp >= 3) {
     const int t = threadIdx.x - 96;  // 0..255
     // the two E blocks of the V ring: rows 0..15 of a K-major, 128-byte-swizzled
-    // B operand; row 0 = 1.0 (0x38) for every key, rows 1..15 zero
+    // B operand, all zero except one row of 1.0 (0x38) for every key: row 0 in
+    // the block of stages 0/1, row 1 in the block of stages 2/3, so that tiles
+    // t and t+2 put their row sums into different columns
     {
-      const int rr = (t >> 3) & 15, ch = t & 7;
-      uint8_t *eblk = sV + voff(2 * (t >> 7)) + SZ_TILE8;
-      const uint32_t v = rr == 0 ? 0x38383838u : 0u;
+      const int rr = (t >> 3) & 15, ch = t & 7, blk = t >> 7;
+      uint8_t *eblk = sV + voff(2 * blk) + SZ_TILE8;
+      const uint32_t v = rr == blk ? 0x38383838u : 0u;
       *reinterpret_cast<uint4 *>(eblk + sw128_off(rr, ch)) = make_uint4(v, v, v, v);
     }
     if (t < 128) s_vscale[t] = p.vscale[static_cast<size_t>(bh) * 128 + t];
@@ -303,15 +311,17 @@ __global__ void __launch_bounds__(352, 1)
         return true;
       };
       for (int t = 0; t < T && ok; ++t) {
-        ok = mwait(&bars.pfull[t & 1], (t >> 1) & 1);
-        if (!ok) break;
+        // V(t) lands long before the bytes: check it first, so that PV(t) goes
+        // out as soon as pfull(t) completes
         const int s = t % VS;
         ok = mwait(&bars.vfull[s], (t / VS) & 1);
+        if (!ok) break;
+        ok = mwait(&bars.pfull[t & 1], (t >> 1) & 1);
         if (!ok) break;
         tc_fence_after();
         if (elect_one()) {
           // even tile: B = V(t) + E, D = [O | l_even]; odd: B = E + V(t), D = [l_odd | O]
-          const uint32_t pa = tmem + TM_P + 32 * (t & 1);
+          const uint32_t pa = tmem + TM_P + 32 * (t % 3);
           const uint32_t d = tmem + ((t & 1) ? TM_LO : TM_O);
           const uint64_t bv = dV + ((voff(s) - (s & 1) * SZ_EBLK) >> 4);
 #pragma unroll
@@ -329,7 +339,7 @@ __global__ void __launch_bounds__(352, 1)
         }
         if (elect_one()) {
           mma_commit(&bars.vempty[s]);
-          mma_commit(&bars.pvdone[t & 3]);
+          mma_commit(&bars.pvdone[t % NPD]);
         }
         __syncwarp();
       }
@@ -374,21 +384,24 @@ __global__ void __launch_bounds__(352, 1)
   } else {
     // ------------------------------------------------------------ softmax rows
     // Warpgroup g (warps 3+4g .. 6+4g) takes the tiles t with t % 2 == g;
-    // thread row r = 32*(warp%4) + lane. Shared per-row state, handed from
-    // tile to tile in order: s_m / s_F (running max and frame; mxr[t%2]) and
-    // s_ltot / sLb (row sum and staged l_t, both in the current frame;
-    // tdone[t%2]).
+    // thread row r = 32*(warp%4) + lane. The frame is handed from tile to tile
+    // in order through s_F (mxr[t%2]). Row sums stay with the warpgroup that
+    // owns the tile: lt_own (registers) and its own slots of sLb (slot t%32 of
+    // every tile t of parity g), all in the frame of its latest tile; the two
+    // warpgroups meet only where a chunk of 32 row sums is flushed for the
+    // block-mean restore, and at the end.
     const int g = (warp - 3) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    const uint32_t lcol = g == 0 ? TM_LE : TM_LO;  // this warpgroup's row-sum column
     const float sqs = p.sq[static_cast<size_t>(bh) * T + qt];
     const float *skh = p.sk + static_cast<size_t>(bh) * T;
     const int tail = p.N - (T - 1) * 128;  // valid keys in the last tile
     bool ok = true;
     float F_own = 0.0f;   // frame of this warpgroup's latest tile
     float F_hand = 0.0f;  // frame handed over to this warpgroup's latest tile
+    float lt_own = 0.0f;  // sum of l_u over this warpgroup's tiles read so far, in frame F_own
+    float lprev0 = 0.0f, lprev1 = 0.0f;  // last values read from this warpgroup's two row-sum columns
     float sk_next = skh[g < T ? g : 0];
     // every lane waits; the outcome is made warp-uniform so that the
     // .sync.aligned TMEM instructions below always see the whole warp
@@ -396,13 +409,16 @@ __global__ void __launch_bounds__(352, 1)
       const bool w = wait(bar, parity);
       return __all_sync(0xFFFFFFFFu, w);
     };
-    auto flush = [&](int nvalid) {
-      // A operand of the restore MMA: row r = [hi(l_0..l_31) | lo(l_0..l_31)] in bf16
+    // A operand of the restore MMA: row r = [hi(l_0..l_31) | lo(l_0..l_31)] in
+    // bf16; the slots of the other warpgroup's parity are scaled by sc_other
+    // into this warpgroup's frame
+    auto flush = [&](int nvalid, float sc_other) {
+      const float sc0 = g == 0 ? 1.0f : sc_other, sc1 = g == 1 ? 1.0f : sc_other;
       uint32_t hw[16], lw[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        float l0 = (2 * i < nvalid) ? sLb[(2 * i) * 128 + r] : 0.0f;
-        float l1 = (2 * i + 1 < nvalid) ? sLb[(2 * i + 1) * 128 + r] : 0.0f;
+        float l0 = (2 * i < nvalid) ? sLb[(2 * i) * 128 + r] * sc0 : 0.0f;
+        float l1 = (2 * i + 1 < nvalid) ? sLb[(2 * i + 1) * 128 + r] * sc1 : 0.0f;
         const __nv_bfloat16 h0 = __float2bfloat16_rn(l0), h1 = __float2bfloat16_rn(l1);
         const __nv_bfloat16 o0 = __float2bfloat16_rn(__fsub_rn(l0, __bfloat162float(h0)));
         const __nv_bfloat16 o1 = __float2bfloat16_rn(__fsub_rn(l1, __bfloat162float(h1)));
@@ -455,32 +471,22 @@ __global__ void __launch_bounds__(352, 1)
         mx = max3(mm[0], mm[1], fmaxf(mm[2], fmaxf(mm[3], mm[4])));
       }
       const float alpha = __fmul_rn(__fmul_rn(sqs, skt), p.kappa);
-      // running max and frame, taken over from tile t-1's warpgroup
-      float m_prev = -INFINITY, F_prev = -INFINITY;
+      // frame, taken over from tile t-1's warpgroup: F_t = max(F_{t-1}, 8 ceil(m_t / 8))
+      // with m_t this tile's scaled row max, i.e. 8 ceil(running max / 8)
+      float F_prev = -INFINITY;
       if (t > 0) {
         if (!wwait(&bars.mxr[(t - 1) & 1], ((t - 1) >> 1) & 1)) return false;
-        m_prev = s_m[r];
         F_prev = s_F[r];
       }
-      const float m = fmaxf(m_prev, __fmul_rn(mx, alpha));
-      const float Fn = 8.0f * ceilf(m * 0.125f);
+      const float Fn = fmaxf(F_prev, 8.0f * ceilf(__fmul_rn(mx, alpha) * 0.125f));
       if (t == 0) F_prev = Fn;
-      s_m[r] = m;  // for tile t+1 (after the last tile, s_F holds the final frame)
-      s_F[r] = Fn;
+      s_F[r] = Fn;  // for tile t+1 (after the last tile it holds the final frame)
       if (t + 1 < T) mbar_arrive(&bars.mxr[b]);
       const bool need = Fn != F_prev;
       const float sc = need ? frame_scale(F_prev, Fn) : 1.0f;
       const bool anyneed = __any_sync(0xFFFFFFFFu, need);
-      // PV(t-2) is complete: P buffer t&1 is free, and this warpgroup's
-      // row-sum column holds l_{t-2} alone (reset here for l_t)
-      uint32_t lraw = 0u;
-      if (t >= 2) {
-        if (!wwait(&bars.pvdone[(t - 2) & 3], ((t - 2) >> 2) & 1)) return false;
-        tc_fence_after();
-        lraw = tmem_ld1(trow + lcol);
-        tmem_wait_ld();
-        tmem_st1(trow + lcol, 0u);
-      }
+      // P slot t%3 was last read by PV(t-3), complete since the bookkeeping of
+      // tile t-2 (which waited for PV(t-3) and, by commit order, all before it)
       // bytes against the frame Fn: one 32-column store of the row's 128
       // bytes, 4 per column
       {
@@ -499,11 +505,11 @@ __global__ void __launch_bounds__(352, 1)
             w[q] &= keep;
           }
         }
-        tmem_st32(trow + TM_P + 32 * b, w);
+        tmem_st32(trow + TM_P + 32 * (t % 3), w);
       }
       if (anyneed) {
         // O holds PV(0..t-1) in frame F_prev: rescale it before PV(t)
-        if (!wwait(&bars.pvdone[(t - 1) & 3], ((t - 1) >> 2) & 1)) return false;
+        if (!wwait(&bars.pvdone[(t - 1) % NPD], ((t - 1) / NPD) & 1)) return false;
         tc_fence_after();
         uint32_t o[128];
 #pragma unroll
@@ -516,41 +522,63 @@ __global__ void __launch_bounds__(352, 1)
         for (int i = 0; i < 4; ++i)
           tmem_st32(trow + TM_O + 32 * i, *reinterpret_cast<const uint32_t(*)[32]>(&o[32 * i]));
       }
-      tmem_wait_st();  // the P bytes, the column reset and any O rescale are in TMEM
+      tmem_wait_st();  // the P bytes (and any O rescale) are in TMEM
       tc_fence_before();
       mbar_arrive(&bars.pfull[b]);
-      // row-sum bookkeeping, in tile order after tile t-1's
-      if (t > 0 && !wwait(&bars.tdone[(t - 1) & 1], ((t - 1) >> 1) & 1)) return false;
-      if (need)
-        for (int sl = 0; sl < 32; ++sl) sLb[sl * 128 + r] *= sc;
-      float lt = (t > 0 ? s_ltot[r] : 0.0f) * sc;
-      bool flushed = false;
+
+      // ---- row-sum bookkeeping of this warpgroup, off the PV path
+      if (g == 0 && t >= 34 && ((t - 34) & 31) == 0) {
+        // the other warpgroup flushed chunk (t-34)/32 at tile t-1: it has read
+        // this warpgroup's slots once lflush completes
+        if (!wwait(&bars.lflush, ((t - 34) >> 5) & 1)) return false;
+      }
+      // PV(t-1) complete, and with it every earlier PV: the P slot of tile t+2
+      // (last read by PV(t-1)) is free, and l_{t-2} can be read
+      if (t >= 1) {
+        if (!wwait(&bars.pvdone[(t - 1) % NPD], ((t - 1) / NPD) & 1)) return false;
+        tc_fence_after();
+      }
       if (t >= 2) {
-        // l_{t-2}: this warpgroup's previous tile, computed in frame F_own
-        const float lo = __uint_as_float(lraw) * frame_scale(F_own, Fn);
+        // l_{t-2} (own previous tile, frame F_own): what PV(t-2) added to its column
+        const float v = __uint_as_float(tmem_ld1(trow + lcol_of(t - 2)));
+        tmem_wait_ld();
+        float lraw;
+        if ((t - 2) & 2) {
+          lraw = __fsub_rn(v, lprev1);
+          lprev1 = v;
+        } else {
+          lraw = __fsub_rn(v, lprev0);
+          lprev0 = v;
+        }
+        const float scw = frame_scale(F_own, Fn);
+        if (F_own != Fn) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) sLb[(2 * i + g) * 128 + r] *= scw;
+        }
+        const float lo = lraw * scw;
+        lt_own = lt_own * scw + lo;
         const int slot = (t - 2) & 31;
         sLb[slot * 128 + r] = lo;
-        lt += lo;
         if (slot == 31) {
-          flush(32);
-          flushed = true;
+          // chunk (t-33)/32 is complete: the other warpgroup's slots are in the
+          // frame of tile t-1 once its bookkeeping of that tile is done (bk)
+          if (!wwait(&bars.bk, ((t - 33) >> 5) & 1)) return false;
+          flush(32, sc);
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(&bars.lflush);  // the restore follows PV(t)
         }
       }
-      s_ltot[r] = lt;
+      if (g == 0 && t >= 32 && (t & 31) == 0) mbar_arrive(&bars.bk);
       F_own = Fn;
       F_hand = F_prev;
-      if (flushed) {  // the restore of this chunk follows PV(t)
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&bars.lflush);
-      }
-      mbar_arrive(&bars.tdone[b]);
       return true;
     };
 
-    // this warpgroup's row-sum column starts at zero: the first odd PV
-    // accumulates onto it (the first even PV overwrites)
-    tmem_st1(trow + lcol, 0u);
+    // this warpgroup's row-sum columns start at zero: odd tiles accumulate
+    // onto theirs (the first even tile overwrites)
+    tmem_st1(trow + lcol_of(g), 0u);
+    tmem_st1(trow + lcol_of(g + 2), 0u);
     tmem_wait_st();
     const bool ragged = tail < 128;
     for (int t = g; t < T - 1 && ok; t += 2) ok = tile(t, std::false_type{});
@@ -558,31 +586,41 @@ __global__ void __launch_bounds__(352, 1)
       ok = ragged ? tile(T - 1, std::true_type{}) : tile(T - 1, std::false_type{});
 
     // ---------------------------------------------------------- end of the KV loop
-    // The warpgroup of the last tile adds l_{T-2} and l_{T-1} to the row sum
-    // and flushes the remaining one or two restore chunks; then it runs the
-    // repair; then both warpgroups write half of the output columns each.
+    // The warpgroup of the last tile (fin_wg) takes the other's row-sum state,
+    // adds l_{T-2} and l_{T-1}, and flushes the remaining one or two restore
+    // chunks; then it runs the repair; then both warpgroups write half of the
+    // output columns each.
     const bool fin_wg = ((T - 1) & 1) == g;
-    if (ok && fin_wg) ok = wwait(&bars.main, 0);
+    if (!fin_wg) {
+      s_lto[r] = lt_own;  // frame F_{T-2}, the frame the last tile was handed
+      s_lprev[0][r] = lprev0;
+      s_lprev[1][r] = lprev1;
+      mbar_arrive(&bars.wgdone);
+    }
+    if (ok && fin_wg) ok = wwait(&bars.main, 0) && wwait(&bars.wgdone, 0);
     const float F_fin = F_own;  // frame of the last tile (meaningful in fin_wg)
     if (ok && fin_wg) {
       tc_fence_after();
-      float lt = s_ltot[r];
+      const float sc_o = frame_scale(F_hand, F_fin);  // other warpgroup's frame -> F_fin
+      float lt = lt_own + s_lto[r] * sc_o;
       int e = 0;
       for (int u = (T >= 2 ? T - 2 : 0); u <= T - 1; ++u) {
-        // l_u is in the row-sum column of parity u%2, computed in frame F_{T-1} (own last tile) or
-        // F_{T-2} (the frame handed over to the last tile)
-        const float lu_raw = __uint_as_float(tmem_ld1(trow + ((u & 1) ? TM_LO : TM_LE)));
+        // l_u: u = T-1 in frame F_fin, u = T-2 in frame F_hand (its slot keeps
+        // the other warpgroup's frame convention)
+        const float v = __uint_as_float(tmem_ld1(trow + lcol_of(u)));
         tmem_wait_ld();
-        const float lo = lu_raw * frame_scale(u == T - 1 ? F_own : F_hand, F_fin);
+        const int cix = (u >> 1) & 1;
+        const float prev = u == T - 1 ? (cix ? lprev1 : lprev0) : s_lprev[cix][r];
+        const float lu_raw = __fsub_rn(v, prev);
         const int slot = u & 31;
-        sLb[slot * 128 + r] = lo;
-        lt += lo;
+        sLb[slot * 128 + r] = lu_raw;
+        lt += u == T - 1 ? lu_raw : lu_raw * sc_o;
         if (slot == 31 || u == T - 1) {
           if (e > 0) {  // the restore of the previous flush must have read sAr
             ok = wwait(&bars.rdone, (e - 1) & 1);
             if (!ok) break;
           }
-          flush(slot + 1);
+          flush(slot + 1, sc_o);
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(&bars.epi);

@@ -31,7 +31,7 @@ Shape make_shape(int B, int H, int N, const vc_params &p, int R) {
   const int target = std::max(1, (4 * 148 + s.BH - 1) / s.BH);  // k-means blocks per (b,h)
   s.km_cpb = std::max(1, (s.Nb + target - 1) / target);
   s.km_nblk = (s.Nb + s.km_cpb - 1) / s.km_cpb;
-  s.kb_nchunk = std::max(1, std::min(s.Nb, (2 * 148 + s.BH - 1) / s.BH));
+  s.kb_nchunk = std::max(1, std::min(s.Nb, (4 * 148 + s.BH - 1) / s.BH));
   s.flags = p.flags;
   return s;
 }
@@ -49,6 +49,7 @@ WsLayout make_layout(const Shape &s) {
   L.status = take(256);
   L.km_counter = take(BH * 4);
   L.vq_counter = take(BH * 4);
+  L.kb_counter = take(BH * 4);
   L.perm = take(BH * N * 4);
   L.labels = take(BH * N * 4);
   L.cent = take(BH * k * D * 4);
@@ -213,7 +214,7 @@ vc_status last_error() { return cudaGetLastError() == cudaSuccess ? VC_OK : VC_E
 
 // Clear the completion counters and the status word at the start of a call.
 vc_status clear_small(const Ws &w, cudaStream_t s) {
-  // status, km_counter and vq_counter are the first three regions of the layout
+  // status and the per-(b,h) counters are the regions of the layout before perm
   if (cudaMemsetAsync(w.base, 0, w.L.perm, s) != cudaSuccess) return VC_ERR_CUDA;
   return VC_OK;
 }
@@ -245,11 +246,12 @@ void launch_quant_qk(const Shape &sh, const Ws &w, const uint16_t *Q, const uint
   double *part = w.at<double>(w.L.kbar_part);
   float *kbar = w.at<float>(w.L.kbar);
   if (ks) {
-    k_kbar_partial<<<dim3(sh.kb_nchunk, sh.BH), 128, 0, s>>>(K, sh.N, sh.kb_nchunk, part);
+    k_kbar<<<dim3(sh.kb_nchunk, sh.BH), 256, 0, s>>>(K, sh.N, sh.kb_nchunk, 1, part, w.at<unsigned>(w.L.kb_counter),
+                                                     kbar);
     count_launch();
+  } else {
+    cudaMemsetAsync(kbar, 0, static_cast<size_t>(sh.BH) * D * sizeof(float), s);  // no K smoothing: mean 0
   }
-  k_kbar_final<<<sh.BH, 128, 0, s>>>(part, sh.N, ks ? sh.kb_nchunk : 0, ks, kbar);
-  count_launch();
   k_qk_quant<<<dim3(sh.Nb, sh.BH, 2), 256, 0, s>>>(Q, K, perm, kbar, sh.N, sh.Npad, q8, sq, k8, sk);
   count_launch();
 }
@@ -258,11 +260,11 @@ void launch_quant_v(const Shape &sh, const Ws &w, const uint16_t *V, const int32
                     float *vscale, uint16_t *vmean, int32_t *rep_idx, uint16_t *rep_delta, cudaStream_t s) {
   const int demean = (sh.flags & VC_VSMOOTH) ? 1 : 0;
   int *vexpo = w.at<int>(w.L.vexpo);
-  k_quantv_pass1<<<dim3(sh.Nb, sh.BH), 128, 0, s>>>(V, perm, sh.N, sh.Nb, demean, vmean,
+  k_quantv_pass1<<<dim3(sh.Nb, sh.BH), 256, QUANTV1_SMEM, s>>>(V, perm, sh.N, sh.Nb, demean, vmean,
                                                      w.at<float>(w.L.amax_part), vscale, vexpo,
                                                      w.at<unsigned>(w.L.vq_counter));
   count_launch();
-  k_quantv_pass2<<<dim3(sh.Nb, sh.BH), 128, QUANTV2_SMEM, s>>>(V, perm, sh.N, sh.Nb, sh.Npad, sh.nch32, vmean, vscale, vexpo,
+  k_quantv_pass2<<<dim3(sh.Nb, sh.BH), 256, QUANTV2_SMEM, s>>>(V, perm, sh.N, sh.Nb, sh.Npad, sh.nch32, vmean, vscale, vexpo,
                                                      v8t, w.at<float>(w.L.err), w.at<uint16_t>(w.L.mut2));
   count_launch();
   if (sh.R > 0) {

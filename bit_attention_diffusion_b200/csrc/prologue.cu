@@ -325,152 +325,224 @@ __global__ void __launch_bounds__(1024) k_perm_sort(const int32_t *__restrict__ 
   }
 }
 
-// ============================================================== Q/K smoothing + quantization
-// Partial fp64 channel sums of K over a row range (one block per (chunk, b,h)).
-__global__ void __launch_bounds__(128) k_kbar_partial(const uint16_t *__restrict__ K, int N, int nchunk,
-                                                      double *__restrict__ part) {
-  const int bh = blockIdx.y, ch = blockIdx.x, c = threadIdx.x;
-  const int rows = (N + nchunk - 1) / nchunk;
-  const int r0 = ch * rows, r1 = min(N, r0 + rows);
-  const uint16_t *Kh = K + static_cast<size_t>(bh) * N * D;
-  double s = 0.0;
-  for (int r = r0; r < r1; ++r) s += static_cast<double>(bf16_to_f32(Kh[static_cast<size_t>(r) * D + c]));
-  part[(static_cast<size_t>(bh) * nchunk + ch) * D + c] = s;
+// ============================================================== streaming helpers
+// The HBM-bound kernels below move a 128-row tile with 256 threads: thread
+// (g, c) = (tid / 16, tid % 16) owns the 16-byte chunk c (channels 8c..8c+7)
+// of rows g, g+16, ..., g+112, so every thread has eight independent 16-byte
+// loads in flight and a warp covers two full rows per load.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
+               "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void bf16x8(const uint4 &w, float *x) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(ws[i] << 16);
+    x[2 * i + 1] = __uint_as_float(ws[i] & 0xFFFF0000u);
+  }
 }
 
-__global__ void __launch_bounds__(128) k_kbar_final(const double *__restrict__ part, int N, int nchunk,
-                                                    int ksmooth, float *__restrict__ kbar) {
-  const int bh = blockIdx.x, c = threadIdx.x;
-  double s = 0.0;
-  for (int ch = 0; ch < nchunk; ++ch) s += part[(static_cast<size_t>(bh) * nchunk + ch) * D + c];
-  kbar[static_cast<size_t>(bh) * D + c] = ksmooth ? static_cast<float>(s / static_cast<double>(N)) : 0.0f;
+// ============================================================== Q/K smoothing + quantization
+// Channel sums of K in fp64 over a row range (one block per (chunk, b,h));
+// the last block of a (b,h) adds the chunk sums in chunk order and writes the
+// channel mean (0 without K smoothing).
+__global__ void __launch_bounds__(256) k_kbar(const uint16_t *__restrict__ K, int N, int nchunk, int ksmooth,
+                                              double *__restrict__ part, unsigned *__restrict__ counter,
+                                              float *__restrict__ kbar) {
+  __shared__ double red[16][128];
+  __shared__ int s_last;
+  const int bh = blockIdx.y, ch = blockIdx.x, tid = threadIdx.x;
+  const int g = tid >> 4, c = tid & 15;
+  const int rows = (N + nchunk - 1) / nchunk;
+  const int r0 = ch * rows, r1 = min(N, r0 + rows);
+  const uint16_t *Kh = K + static_cast<size_t>(bh) * N * D + 8 * c;
+  double a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int r = r0 + g; r < r1; r += 64) {
+    uint4 w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      w[u] = (r + 16 * u < r1) ? __ldg(reinterpret_cast<const uint4 *>(Kh + static_cast<size_t>(r + 16 * u) * D))
+                               : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float x[8];
+      bf16x8(w[u], x);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] += static_cast<double>(x[j]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[g][8 * c + j] = a[j];
+  __syncthreads();
+  if (tid < 128) {
+    double sum = 0.0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sum += red[i][tid];
+    part[(static_cast<size_t>(bh) * nchunk + ch) * D + tid] = sum;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&counter[bh], 1u) == static_cast<unsigned>(nchunk - 1));
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (tid < 128) {
+    double sum = 0.0;
+    for (int i = 0; i < nchunk; ++i) sum += __ldcg(part + (static_cast<size_t>(bh) * nchunk + i) * D + tid);
+    kbar[static_cast<size_t>(bh) * D + tid] = ksmooth ? static_cast<float>(sum / static_cast<double>(N)) : 0.0f;
+  }
+  if (tid == 0) counter[bh] = 0u;
 }
 
 // Block quantization: z = 0 -> Q rows [128t, 128t+128) in original order;
 // z = 1 -> K rows perm[128t + r] minus the channel mean. scale = amax/448,
-// codes = E4M3(x * (448/amax)). 8 warps x 16 rows, 4 channels per lane.
+// codes = E4M3(x * (448/amax)); rows past N get code 0.
 __global__ void __launch_bounds__(256) k_qk_quant(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                                                   const int32_t *__restrict__ perm, const float *__restrict__ kbar,
                                                   int N, int Npad, uint8_t *__restrict__ q8, float *__restrict__ sq,
                                                   uint8_t *__restrict__ k8, float *__restrict__ sk) {
   __shared__ float wmax[8];
   const int t = blockIdx.x, bh = blockIdx.y, z = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, g = tid >> 4, c = tid & 15;
   const int cnt = min(TILE, N - t * TILE);
-  const uint16_t *src = (z == 0 ? Q : K) + static_cast<size_t>(bh) * N * D;
-  float kb[4] = {0.f, 0.f, 0.f, 0.f};
-  if (z == 1) {
-    const float4 k4 = *reinterpret_cast<const float4 *>(kbar + static_cast<size_t>(bh) * D + 4 * lane);
-    kb[0] = k4.x; kb[1] = k4.y; kb[2] = k4.z; kb[3] = k4.w;
+  const uint16_t *src = (z == 0 ? Q : K) + static_cast<size_t>(bh) * N * D + 8 * c;
+  int row[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int rr = g + 16 * i, pos = t * TILE + rr;
+    row[i] = rr < cnt ? ((z == 1 && perm != nullptr) ? __ldg(perm + static_cast<size_t>(bh) * N + pos) : pos) : -1;
   }
-  float x[16][4];
+  uint4 w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    w[i] = row[i] >= 0 ? __ldg(reinterpret_cast<const uint4 *>(src + static_cast<size_t>(row[i]) * D))
+                       : make_uint4(0u, 0u, 0u, 0u);
+  float kb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (z == 1) {
+    const float4 k0 = *reinterpret_cast<const float4 *>(kbar + static_cast<size_t>(bh) * D + 8 * c);
+    const float4 k1 = *reinterpret_cast<const float4 *>(kbar + static_cast<size_t>(bh) * D + 8 * c + 4);
+    kb[0] = k0.x; kb[1] = k0.y; kb[2] = k0.z; kb[3] = k0.w;
+    kb[4] = k1.x; kb[5] = k1.y; kb[6] = k1.z; kb[7] = k1.w;
+  }
   float amax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int r = warp * 16 + i;
-    if (r < cnt) {
-      const int p = t * TILE + r;
-      const int row = (z == 1 && perm != nullptr) ? perm[static_cast<size_t>(bh) * N + p] : p;
-      const uint2 w = *reinterpret_cast<const uint2 *>(src + static_cast<size_t>(row) * D + 4 * lane);
-      const float v[4] = {__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u),
-                          __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u)};
+  for (int i = 0; i < 8; ++i) {
+    if (row[i] < 0) continue;  // rows past N do not enter the block's amax
+    float x[8];
+    bf16x8(w[i], x);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        x[i][e] = (z == 1) ? __fsub_rn(v[e], kb[e]) : v[e];
-        amax = fmaxf(amax, fabsf(x[i][e]));
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) x[i][e] = 0.0f;
-    }
+    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(z == 1 ? __fsub_rn(x[j], kb[j]) : x[j]));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-  if (lane == 0) wmax[warp] = amax;
+  if ((tid & 31) == 0) wmax[tid >> 5] = amax;
   __syncthreads();
   amax = wmax[0];
 #pragma unroll
-  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, wmax[w]);
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, wmax[i]);
   const float scale = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 448.0f);
   const float mult = amax == 0.0f ? 0.0f : __fdiv_rn(448.0f, amax);
-  uint8_t *dst = (z == 0 ? q8 : k8) + (static_cast<size_t>(bh) * Npad + static_cast<size_t>(t) * TILE) * D;
+  uint8_t *dst = (z == 0 ? q8 : k8) + (static_cast<size_t>(bh) * Npad + static_cast<size_t>(t) * TILE) * D + 8 * c;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int r = warp * 16 + i;
-    uint32_t packed = 0;
-    if (r < cnt) {
-      const uint32_t lo = e4m3x2(__fmul_rn(x[i][0], mult), __fmul_rn(x[i][1], mult));
-      const uint32_t hi = e4m3x2(__fmul_rn(x[i][2], mult), __fmul_rn(x[i][3], mult));
-      packed = lo | (hi << 16);
+  for (int i = 0; i < 8; ++i) {
+    float x[8];
+    bf16x8(w[i], x);
+    uint32_t lo = 0, hi = 0;
+    if (row[i] >= 0) {
+      float y[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(z == 1 ? __fsub_rn(x[j], kb[j]) : x[j], mult);
+      lo = static_cast<uint32_t>(e4m3x2(y[0], y[1])) | (static_cast<uint32_t>(e4m3x2(y[2], y[3])) << 16);
+      hi = static_cast<uint32_t>(e4m3x2(y[4], y[5])) | (static_cast<uint32_t>(e4m3x2(y[6], y[7])) << 16);
     }
-    *reinterpret_cast<uint32_t *>(dst + static_cast<size_t>(r) * D + 4 * lane) = packed;
+    *reinterpret_cast<uint2 *>(dst + static_cast<size_t>(g + 16 * i) * D) = make_uint2(lo, hi);
   }
   if (tid == 0) (z == 0 ? sq : sk)[static_cast<size_t>(bh) * (Npad / TILE) + t] = scale;
 }
 
 // ============================================================== V demean + quantization
-constexpr int VQ_ROW_WORDS = 66;
+// The block's 128 rows (gathered through perm) are copied to shared memory
+// with cp.async, row stride 272 bytes: 16-byte reads of one row per thread
+// then hit 8 different bank groups per quarter warp.
+constexpr int VQ_ROW_BYTES = 272;
 
-// Gather the block's rows (through perm) into shared memory, one warp per row.
-__device__ __forceinline__ void gather_rows(uint32_t *sv, const uint16_t *Vh, const int32_t *permh, int p0, int cnt) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nw = blockDim.x >> 5;
-  for (int r = warp; r < TILE; r += nw) {
-    uint2 w = make_uint2(0u, 0u);
-    if (r < cnt) {
-      const int row = permh ? permh[p0 + r] : p0 + r;
-      w = *reinterpret_cast<const uint2 *>(Vh + static_cast<size_t>(row) * D + 4 * lane);
+__device__ __forceinline__ void gather_tile(uint8_t *sv, const uint16_t *Vh, const int32_t *permh, int p0, int cnt) {
+  const int g = threadIdx.x >> 4, c = threadIdx.x & 15;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int rr = g + 16 * i;
+    uint8_t *d = sv + rr * VQ_ROW_BYTES + 16 * c;
+    if (rr < cnt) {
+      const int row = permh ? __ldg(permh + p0 + rr) : p0 + rr;
+      cp_async16(d, Vh + static_cast<size_t>(row) * D + 8 * c);
+    } else {
+      *reinterpret_cast<uint4 *>(d) = make_uint4(0u, 0u, 0u, 0u);
     }
-    sv[r * VQ_ROW_WORDS + 2 * lane] = w.x;
-    sv[r * VQ_ROW_WORDS + 2 * lane + 1] = w.y;
   }
+  cp_async_wait_all();
 }
-__device__ __forceinline__ float sv_get(const uint32_t *sv, int r, int c) {
-  const uint32_t w = sv[r * VQ_ROW_WORDS + (c >> 1)];
-  return (c & 1) ? __uint_as_float(w & 0xFFFF0000u) : __uint_as_float(w << 16);
+__device__ __forceinline__ float sv_at(const uint8_t *sv, int r, int c) {
+  const uint16_t b = *reinterpret_cast<const uint16_t *>(sv + r * VQ_ROW_BYTES + 2 * c);
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
 
-// Pass 1: block means and per-block residual amax; the last block of a (b,h)
-// turns the channel amax into the power-of-two scale.
-__global__ void __launch_bounds__(128) k_quantv_pass1(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
+// Pass 1: block means (fp64 sums over the block's tokens) and per-block
+// residual amax; the last block of a (b,h) turns the channel amax into the
+// power-of-two scale. Thread (h, c): channel c over rows [64h, 64h+64).
+__global__ void __launch_bounds__(256) k_quantv_pass1(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
                                                       int N, int Nb, int demean, uint16_t *__restrict__ vmean,
                                                       float *__restrict__ amax_part, float *__restrict__ vscale,
                                                       int *__restrict__ vexpo, unsigned *__restrict__ counter) {
-  __shared__ uint32_t sv[TILE * VQ_ROW_WORDS];
+  extern __shared__ __align__(16) uint8_t dsm[];
+  uint8_t *sv = dsm;  // 128 rows x 272 bytes
+  __shared__ double ssum[2][128];
+  __shared__ float smax[2][128];
   __shared__ int s_last;
-  const int t = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
+  const int t = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
   const int p0 = t * TILE, cnt = min(TILE, N - p0);
-  gather_rows(sv, V + static_cast<size_t>(bh) * N * D, perm ? perm + static_cast<size_t>(bh) * N : nullptr, p0, cnt);
+  gather_tile(sv, V + static_cast<size_t>(bh) * N * D, perm ? perm + static_cast<size_t>(bh) * N : nullptr, p0, cnt);
   __syncthreads();
+  const int c = tid & 127, h = tid >> 7;
+  const int ra = 64 * h, rb = min(cnt, ra + 64);
   uint16_t mu = 0;
   if (demean) {
     double s = 0.0;
-    for (int r = 0; r < cnt; ++r) s += static_cast<double>(sv_get(sv, r, c));
-    mu = f32_to_bf16_rn(static_cast<float>(s / static_cast<double>(cnt)));
+    for (int r = ra; r < rb; ++r) s += static_cast<double>(sv_at(sv, r, c));
+    ssum[h][c] = s;
+    __syncthreads();
+    mu = f32_to_bf16_rn(static_cast<float>((ssum[0][c] + ssum[1][c]) / static_cast<double>(cnt)));
   }
   const float muf = bf16_to_f32(mu);
   float amax = 0.0f;
-  for (int r = 0; r < cnt; ++r) amax = fmaxf(amax, fabsf(__fsub_rn(sv_get(sv, r, c), muf)));
-  vmean[(static_cast<size_t>(bh) * Nb + t) * D + c] = mu;
-  amax_part[(static_cast<size_t>(bh) * Nb + t) * D + c] = amax;
+  for (int r = ra; r < rb; ++r) amax = fmaxf(amax, fabsf(__fsub_rn(sv_at(sv, r, c), muf)));
+  smax[h][c] = amax;
+  __syncthreads();
+  if (h == 0) {
+    vmean[(static_cast<size_t>(bh) * Nb + t) * D + c] = mu;
+    amax_part[(static_cast<size_t>(bh) * Nb + t) * D + c] = fmaxf(smax[0][c], smax[1][c]);
+  }
   __threadfence();
   __syncthreads();
-  if (c == 0) s_last = (atomicAdd(&counter[bh], 1u) == static_cast<unsigned>(Nb - 1));
+  if (tid == 0) s_last = (atomicAdd(&counter[bh], 1u) == static_cast<unsigned>(Nb - 1));
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  if (tid >= 128) return;
   float a = 0.0f;
 #pragma unroll 32
   for (int b = 0; b < Nb; ++b) a = fmaxf(a, __ldcg(amax_part + (static_cast<size_t>(bh) * Nb + b) * D + c));
   int e = 0;
-  float s = 1.0f;
+  float sc = 1.0f;
   if (a > 0.0f) {
     int E;
     const float f = frexpf(a, &E);  // a = f * 2^E, f in [0.5, 1); 448 = 0.875 * 2^9
     e = (f > 0.875f) ? E - 8 : E - 9;
-    s = ldexpf(1.0f, e);
+    sc = ldexpf(1.0f, e);
   }
-  vscale[static_cast<size_t>(bh) * D + c] = s;
+  vscale[static_cast<size_t>(bh) * D + c] = sc;
   vexpo[static_cast<size_t>(bh) * D + c] = e;
   if (c == 0) counter[bh] = 0u;
 }
@@ -478,21 +550,22 @@ __global__ void __launch_bounds__(128) k_quantv_pass1(const uint16_t *__restrict
 // Pass 2: residual codes (written channel-major), per-token error, and the
 // bf16 block means pre-divided by the channel scale for the in-kernel restore
 // (mut2[bh][chunk][c][0..63]: slots 0..31 and 32..63 both hold tile
-// chunk*32 + slot; unused slots of the last chunk are zero).
-__global__ void __launch_bounds__(128) k_quantv_pass2(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
+// chunk*32 + slot; unused slots of the last chunk are zero). Thread r < 128
+// owns token r: its error is fmaf-accumulated in channel order.
+__global__ void __launch_bounds__(256) k_quantv_pass2(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
                                                       int N, int Nb, int Npad, int nch32,
                                                       const uint16_t *__restrict__ vmean,
                                                       const float *__restrict__ vscale, const int *__restrict__ vexpo,
                                                       uint8_t *__restrict__ v8t, float *__restrict__ err,
                                                       uint16_t *__restrict__ mut2) {
   extern __shared__ __align__(16) uint8_t dsm[];
-  uint32_t *sv = reinterpret_cast<uint32_t *>(dsm);          // TILE x VQ_ROW_WORDS words
-  uint8_t *codeT = dsm + TILE * VQ_ROW_WORDS * 4;              // D rows x 144 bytes
-  __shared__ float smu[D], smult[D], sscale[D];
+  uint8_t *sv = dsm;                            // 128 rows x 272 bytes
+  uint8_t *codeT = dsm + TILE * VQ_ROW_BYTES;   // 128 channels x 144 bytes
+  __shared__ __align__(16) float smu[D], smult[D], sscale[D];
   const int t = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
   const int p0 = t * TILE, cnt = min(TILE, N - p0);
-  gather_rows(sv, V + static_cast<size_t>(bh) * N * D, perm ? perm + static_cast<size_t>(bh) * N : nullptr, p0, cnt);
-  {
+  gather_tile(sv, V + static_cast<size_t>(bh) * N * D, perm ? perm + static_cast<size_t>(bh) * N : nullptr, p0, cnt);
+  if (tid < 128) {
     const int c = tid;
     const uint16_t mu = vmean[(static_cast<size_t>(bh) * Nb + t) * D + c];
     smu[c] = bf16_to_f32(mu);
@@ -512,33 +585,42 @@ __global__ void __launch_bounds__(128) k_quantv_pass2(const uint16_t *__restrict
       }
   }
   __syncthreads();
-  {
+  if (tid < 128) {
     const int r = tid;
     float acc = 0.0f;
-    for (int c = 0; c < D; c += 2) {
-      uint16_t codes = 0;
-      if (r < cnt) {
-        const float r0 = __fsub_rn(sv_get(sv, r, c), smu[c]);
-        const float r1 = __fsub_rn(sv_get(sv, r, c + 1), smu[c + 1]);
-        codes = e4m3x2(__fmul_rn(r0, smult[c]), __fmul_rn(r1, smult[c + 1]));
-        const float2 dq = e4m3x2_value(codes);
-        const float e0 = __fsub_rn(r0, __fmul_rn(dq.x, sscale[c]));
-        const float e1 = __fsub_rn(r1, __fmul_rn(dq.y, sscale[c + 1]));
-        acc = __fmaf_rn(e0, e0, acc);
-        acc = __fmaf_rn(e1, e1, acc);
+    const uint8_t *row = sv + r * VQ_ROW_BYTES;
+#pragma unroll 2
+    for (int c0 = 0; c0 < D; c0 += 8) {
+      float x[8];
+      bf16x8(*reinterpret_cast<const uint4 *>(row + 2 * c0), x);
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) {
+        const int c = c0 + j;
+        uint16_t codes = 0;
+        if (r < cnt) {
+          const float r0 = __fsub_rn(x[j], smu[c]);
+          const float r1 = __fsub_rn(x[j + 1], smu[c + 1]);
+          codes = e4m3x2(__fmul_rn(r0, smult[c]), __fmul_rn(r1, smult[c + 1]));
+          const float2 dq = e4m3x2_value(codes);
+          const float e0 = __fsub_rn(r0, __fmul_rn(dq.x, sscale[c]));
+          const float e1 = __fsub_rn(r1, __fmul_rn(dq.y, sscale[c + 1]));
+          acc = __fmaf_rn(e0, e0, acc);
+          acc = __fmaf_rn(e1, e1, acc);
+        }
+        codeT[c * 144 + r] = static_cast<uint8_t>(codes & 0xFF);
+        codeT[(c + 1) * 144 + r] = static_cast<uint8_t>(codes >> 8);
       }
-      codeT[c * 144 + r] = static_cast<uint8_t>(codes & 0xFF);
-      codeT[(c + 1) * 144 + r] = static_cast<uint8_t>(codes >> 8);
     }
     if (r < cnt) err[static_cast<size_t>(bh) * N + p0 + r] = acc;
   }
   __syncthreads();
   {
-    const int c = tid;
-    uint8_t *dst = v8t + (static_cast<size_t>(bh) * D + c) * Npad + p0;
+    const int c = tid >> 1, half = tid & 1;
+    uint8_t *dst = v8t + (static_cast<size_t>(bh) * D + c) * Npad + p0 + 64 * half;
+    const uint8_t *srcT = codeT + c * 144 + 64 * half;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      *reinterpret_cast<uint4 *>(dst + 16 * i) = *reinterpret_cast<const uint4 *>(codeT + c * 144 + 16 * i);
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<uint4 *>(dst + 16 * i) = *reinterpret_cast<const uint4 *>(srcT + 16 * i);
   }
 }
 

@@ -10,8 +10,8 @@ __global__ void k_kmeans_pass(const uint16_t *V, int N, int k, int cpb, int nblk
 __global__ void k_kmeans_pass8(const uint16_t *V, int N, int k, int cpb, int nblk, float *cent, int32_t *labels,
                                double *psum, int *pcnt, unsigned *counter, int accumulate);
 __global__ void k_perm_sort(const int32_t *labels, int N, int k, int32_t *perm);
-__global__ void k_kbar_partial(const uint16_t *K, int N, int nchunk, double *part);
-__global__ void k_kbar_final(const double *part, int N, int nchunk, int ksmooth, float *kbar);
+__global__ void k_kbar(const uint16_t *K, int N, int nchunk, int ksmooth, double *part, unsigned *counter,
+                       float *kbar);
 __global__ void k_qk_quant(const uint16_t *Q, const uint16_t *K, const int32_t *perm, const float *kbar, int N,
                            int Npad, uint8_t *q8, float *sq, uint8_t *k8, float *sk);
 __global__ void k_quantv_pass1(const uint16_t *V, const int32_t *perm, int N, int Nb, int demean, uint16_t *vmean,
@@ -25,7 +25,8 @@ __global__ void k_repair_delta(const uint16_t *V, const int32_t *perm, int N, in
                                uint16_t *rep_delta, uint16_t *deltat);
 __global__ void k_identity_perm(int32_t *perm, int N, long long total);
 
-constexpr int QUANTV2_SMEM = 128 * 66 * 4 + 128 * 144;  // rows + transposed codes
+constexpr int QUANTV1_SMEM = 128 * 272;              // gathered rows
+constexpr int QUANTV2_SMEM = 128 * 272 + 128 * 144;  // rows + transposed codes
 constexpr int KMEANS_SMEM_FIXED = 128 * 66 * 4;  // chunk rows; + k*128*(4+8) for centroids and sums
 
 }  // namespace vc

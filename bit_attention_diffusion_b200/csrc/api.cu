@@ -28,7 +28,7 @@ Shape make_shape(int B, int H, int N, const vc_params &p, int R) {
   s.R = R;
   s.Rpad = R > 0 ? ((R + 127) / 128) * 128 : 0;
   s.nch32 = (s.Nb + CHUNK32 - 1) / CHUNK32;
-  const int target = std::max(1, (4 * 148 + s.BH - 1) / s.BH);  // k-means blocks per (b,h)
+  const int target = std::max(1, (3 * 148) / s.BH);  // k-means blocks per (b,h): three resident per SM
   s.km_cpb = std::max(1, (s.Nb + target - 1) / target);
   s.km_nblk = (s.Nb + s.km_cpb - 1) / s.km_cpb;
   s.kb_nchunk = std::max(1, std::min(s.Nb, (4 * 148 + s.BH - 1) / s.BH));
@@ -147,6 +147,8 @@ vc_status check_device() {
           cudaFuncSetAttribute(k_kmeans_pass, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                KMEANS_SMEM_FIXED + 64 * D * 12) != cudaSuccess ||
           cudaFuncSetAttribute(k_quantv_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, QUANTV2_SMEM) !=
+              cudaSuccess ||
+          cudaFuncSetAttribute(k_kmeans_pass8, cudaFuncAttributeMaxDynamicSharedMemorySize, KMEANS8_SMEM) !=
               cudaSuccess) {
         ok_cache[dev] = 0;
         return VC_ERR_CUDA;
@@ -227,7 +229,7 @@ void launch_cluster(const Shape &sh, const Ws &w, const uint16_t *V, int32_t *pe
   const dim3 grid(sh.km_nblk, sh.BH);
   for (int it = 0; it <= sh.iters; ++it) {
     if (sh.k <= 8)
-      k_kmeans_pass8<<<grid, 128, 0, s>>>(V, sh.N, sh.k, sh.km_cpb, sh.km_nblk, cent, labels,
+      k_kmeans_pass8<<<grid, 256, KMEANS8_SMEM, s>>>(V, sh.N, sh.k, sh.km_cpb, sh.km_nblk, cent, labels,
                                           w.at<double>(w.L.km_psum), w.at<int>(w.L.km_pcnt),
                                           w.at<unsigned>(w.L.km_counter), it < sh.iters ? 1 : 0);
     else

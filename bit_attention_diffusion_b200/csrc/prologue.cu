@@ -143,11 +143,15 @@ __global__ void __launch_bounds__(128) k_kmeans_pass(const uint16_t *__restrict_
 // Fast path of the Lloyd pass for k <= 8, same arithmetic per (token,
 // cluster) as k_kmeans_pass: d = fp32(v - c) and acc = fma(d, d, acc) in
 // channel order, two clusters per packed f32x2 instruction (each lane rounds
-// exactly like the scalar instruction). Centroids sit channel-major in shared
-// memory ([c][8]) so one 16-byte load brings four clusters of a channel; the
-// fp64 sums run in registers of the channel's thread behind a label switch
-// that is uniform across the warp (all lanes read the same token).
-constexpr int KM8_ROW_WORDS = 68;  // 272-byte rows: 16-byte aligned, spread over banks
+// exactly like the scalar instruction). 256 threads; the block's 128-token
+// chunks are double-buffered in shared memory with cp.async (272-byte rows).
+// Labels: two threads per token (clusters 0-3 and 4-7), centroids
+// channel-major in shared memory ([c][8]); the halves combine with ties to the
+// lower cluster. Sums: the chunk's tokens are sorted by label (stable, by
+// ballots), then thread (channel pair, quarter) adds its two channels of the
+// tokens of each label in fp64 registers; exact, so the order is free.
+constexpr int KM8_ROW_BYTES = 272;
+static_assert(KMEANS8_SMEM == 2 * TILE * KM8_ROW_BYTES, "chunk buffers");
 
 __device__ __forceinline__ void sub_fma2(float x, float c0, float c1, float &a0, float &a1) {
   asm("{\n\t.reg .b64 xx, cc, dd, aa;\n\t"
@@ -159,116 +163,175 @@ __device__ __forceinline__ void sub_fma2(float x, float c0, float c1, float &a0,
       : "f"(x), "f"(c0), "f"(c1));
 }
 
-__global__ void __launch_bounds__(128) k_kmeans_pass8(const uint16_t *__restrict__ V, int N, int k, int cpb,
+__device__ __forceinline__ void km8_load_chunk(uint8_t *buf, const uint16_t *Vh, int n0, int cnt) {
+  const int g = threadIdx.x >> 4, c = threadIdx.x & 15;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int rr = g + 16 * i;
+    if (rr < cnt)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(
+                       __cvta_generic_to_shared(buf + rr * KM8_ROW_BYTES + 16 * c))),
+                   "l"(Vh + static_cast<size_t>(n0 + rr) * D + 8 * c)
+                   : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(256) k_kmeans_pass8(const uint16_t *__restrict__ V, int N, int k, int cpb,
                                                       int nblk, float *__restrict__ cent,
                                                       int32_t *__restrict__ labels, double *__restrict__ psum,
                                                       int *__restrict__ pcnt, unsigned *__restrict__ counter,
                                                       int accumulate) {
-  __shared__ __align__(16) uint32_t sv[TILE * KM8_ROW_WORDS];
-  __shared__ __align__(16) float scent[D * 8];  // [c][j], j >= k padded with +inf-distance values
+  extern __shared__ __align__(16) uint8_t dsm[];
+  __shared__ __align__(16) float scent[D * 8];  // [c][j]; j >= k unused
   __shared__ int slab[TILE];
-  __shared__ int scnt[8];
+  __shared__ int slist[TILE];
+  __shared__ int sstart[9];
   __shared__ int s_last;
   const int bh = blockIdx.y, blk = blockIdx.x, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const uint16_t *Vh = V + static_cast<size_t>(bh) * N * D;
   float *cent_h = cent + static_cast<size_t>(bh) * k * D;
-  for (int i = tid; i < D * 8; i += TILE) {
+  for (int i = tid; i < D * 8; i += 256) {
     const int c = i >> 3, j = i & 7;
     scent[i] = j < k ? cent_h[j * D + c] : 0.0f;
   }
-  if (tid < 8) scnt[tid] = 0;
-  double acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0, acc4 = 0, acc5 = 0, acc6 = 0, acc7 = 0;
   const int n_begin = blk * cpb * TILE;
   const int n_end = min(N, n_begin + cpb * TILE);
-  for (int n0 = n_begin; n0 < n_end; n0 += TILE) {
-    const int cnt = min(TILE, n_end - n0);
-    __syncthreads();
-    // coalesced chunk load: 16 lanes per 256-byte row, two rows per warp per step
-    for (int r = warp * 2 + (lane >> 4); r < cnt; r += 8) {
-      const uint4 w = *reinterpret_cast<const uint4 *>(Vh + static_cast<size_t>(n0 + r) * D + 8 * (lane & 15));
-      *reinterpret_cast<uint4 *>(&sv[r * KM8_ROW_WORDS + 4 * (lane & 15)]) = w;
+  const int nchunk = (n_end - n_begin + TILE - 1) / TILE;
+  if (nchunk > 0) km8_load_chunk(dsm, Vh, n_begin, min(TILE, n_end - n_begin));
+  double acc[8][2];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = 0.0;
+  int cntj[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // tokens per label (thread 0)
+  const int tok = warp * 16 + (lane & 15), half = lane >> 4;
+  const int cp = tid & 63, qtr = tid >> 6;
+  for (int i = 0; i < nchunk; ++i) {
+    const int n0 = n_begin + i * TILE, cnt = min(TILE, n_end - n0);
+    uint8_t *buf = dsm + (i & 1) * TILE * KM8_ROW_BYTES;
+    if (i + 1 < nchunk) {
+      km8_load_chunk(dsm + ((i + 1) & 1) * TILE * KM8_ROW_BYTES, Vh, n0 + TILE, min(TILE, n_end - n0 - TILE));
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
     __syncthreads();
-    if (tid < cnt) {
-      float a[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) a[j] = 0.0f;
-      const uint32_t *row = sv + tid * KM8_ROW_WORDS;
+    // ---- labels: this thread's four clusters 4*half .. 4*half+3 for token tok
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    if (tok < cnt) {
+      const uint8_t *row = buf + tok * KM8_ROW_BYTES;
 #pragma unroll 2
-      for (int g = 0; g < 16; ++g) {  // 8 channels per 16-byte load
-        const uint4 w = *reinterpret_cast<const uint4 *>(row + 4 * g);
+      for (int g8 = 0; g8 < 16; ++g8) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(row + 16 * g8);
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int c = 8 * g + 2 * h + e;
+            const int c = 8 * g8 + 2 * h + e;
             const float x = e ? __uint_as_float(ws[h] & 0xFFFF0000u) : __uint_as_float(ws[h] << 16);
-            const float4 cA = *reinterpret_cast<const float4 *>(&scent[c * 8]);
-            const float4 cB = *reinterpret_cast<const float4 *>(&scent[c * 8 + 4]);
-            sub_fma2(x, cA.x, cA.y, a[0], a[1]);
-            sub_fma2(x, cA.z, cA.w, a[2], a[3]);
-            sub_fma2(x, cB.x, cB.y, a[4], a[5]);
-            sub_fma2(x, cB.z, cB.w, a[6], a[7]);
+            const float4 cc = *reinterpret_cast<const float4 *>(&scent[c * 8 + 4 * half]);
+            sub_fma2(x, cc.x, cc.y, a0, a1);
+            sub_fma2(x, cc.z, cc.w, a2, a3);
           }
         }
       }
-      int best = 0;
-      float bestd = a[0];
+    }
+    const float av[4] = {a0, a1, a2, a3};
+    int best = -1;
+    float bestd = 0.0f;
 #pragma unroll
-      for (int j = 1; j < 8; ++j)
-        if (j < k && a[j] < bestd) {
-          bestd = a[j];
-          best = j;
-        }
-      slab[tid] = best;
-      labels[static_cast<size_t>(bh) * N + n0 + tid] = best;
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = 4 * half + jj;
+      if (j < k && (best < 0 || av[jj] < bestd)) {
+        bestd = av[jj];
+        best = j;
+      }
+    }
+    const float od = __shfl_xor_sync(0xFFFFFFFFu, bestd, 16);
+    const int oj = __shfl_xor_sync(0xFFFFFFFFu, best, 16);
+    // lower half first; the upper half wins only with a strictly smaller distance
+    const float dlo = half ? od : bestd, dhi = half ? bestd : od;
+    const int jlo = half ? oj : best, jhi = half ? best : oj;
+    const int lab = (jhi >= 0 && dhi < dlo) ? jhi : jlo;
+    if (half == 0 && tok < cnt) {
+      slab[tok] = lab;
+      labels[static_cast<size_t>(bh) * N + n0 + tok] = lab;
     }
     if (accumulate) {
       __syncthreads();
-      const int c = tid;
-      for (int r = 0; r < cnt; ++r) {
-        const uint32_t pr = sv[r * KM8_ROW_WORDS + (c >> 1)];
-        const double x = static_cast<double>((c & 1) ? __uint_as_float(pr & 0xFFFF0000u) : __uint_as_float(pr << 16));
-        switch (slab[r]) {  // uniform across the warp
-          case 0: acc0 += x; break;
-          case 1: acc1 += x; break;
-          case 2: acc2 += x; break;
-          case 3: acc3 += x; break;
-          case 4: acc4 += x; break;
-          case 5: acc5 += x; break;
-          case 6: acc6 += x; break;
-          default: acc7 += x; break;
+      // ---- stable sort of the chunk's tokens by label (warp 0)
+      if (warp == 0) {
+        int lm[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) lm[m] = (32 * m + lane < cnt) ? slab[32 * m + lane] : -1;
+        const unsigned lt = (1u << lane) - 1u;
+        int base = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j >= k) break;
+          unsigned bm[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) bm[m] = __ballot_sync(0xFFFFFFFFu, lm[m] == j);
+          if (lane == 0) sstart[j] = base;
+          int pre = base;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            if (lm[m] == j) slist[pre + __popc(bm[m] & lt)] = 32 * m + lane;
+            pre += __popc(bm[m]);
+          }
+          if (lane == 0) cntj[j] += pre - base;
+          base = pre;
+        }
+        if (lane == 0) sstart[k] = base;
+      }
+      __syncthreads();
+      // ---- fp64 sums: thread (channel pair cp, quarter qtr)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < k) {
+          const int e1 = sstart[j + 1];
+          for (int ii = sstart[j] + qtr; ii < e1; ii += 4) {
+            const uint32_t pr = *reinterpret_cast<const uint32_t *>(buf + slist[ii] * KM8_ROW_BYTES + 4 * cp);
+            acc[j][0] += static_cast<double>(__uint_as_float(pr << 16));
+            acc[j][1] += static_cast<double>(__uint_as_float(pr & 0xFFFF0000u));
+          }
         }
       }
-      if (tid < 8) {
-        int n = 0;
-        for (int r = 0; r < cnt; ++r) n += (slab[r] == tid);
-        scnt[tid] += n;
-      }
     }
+    __syncthreads();  // the buffer is refilled by the load issued in the next iteration
   }
   if (!accumulate) return;
+  // reduce the four quarters in shared memory (the chunk buffers are free now)
+  double *red = reinterpret_cast<double *>(dsm);  // [4][8][128]
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    red[(qtr * 8 + j) * D + 2 * cp] = acc[j][0];
+    red[(qtr * 8 + j) * D + 2 * cp + 1] = acc[j][1];
+  }
+  __syncthreads();
   double *ps = psum + (static_cast<size_t>(bh) * nblk + blk) * k * D;
   int *pc = pcnt + (static_cast<size_t>(bh) * nblk + blk) * k;
-  const double accs[8] = {acc0, acc1, acc2, acc3, acc4, acc5, acc6, acc7};
+  for (int i = tid; i < k * D; i += 256) {
+    const int j = i / D, c = i % D;
+    ps[i] = red[(0 * 8 + j) * D + c] + red[(1 * 8 + j) * D + c] + red[(2 * 8 + j) * D + c] + red[(3 * 8 + j) * D + c];
+  }
+  if (tid == 0) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < k) ps[j * D + tid] = accs[j];
-  __syncthreads();
-  if (tid < k) pc[tid] = scnt[tid];
+    for (int j = 0; j < 8; ++j)
+      if (j < k) pc[j] = cntj[j];
+  }
   __threadfence();
   __syncthreads();
   if (tid == 0) s_last = (atomicAdd(&counter[bh], 1u) == static_cast<unsigned>(nblk - 1));
   __syncthreads();
-  if (!s_last) return;
+  if (!s_last || tid >= 128) return;
   __threadfence();
   for (int j = 0; j < k; ++j) {
     double sum = 0.0;
     long long n = 0;
 #pragma unroll 16
-    for (int b = 0; b < nblk; ++b) {  // loads batched by the unroll, sums kept in block order
+    for (int b = 0; b < nblk; ++b) {  // loads batched by the unroll
       sum += __ldcg(psum + ((static_cast<size_t>(bh) * nblk + b) * k + j) * D + tid);
       n += __ldcg(pcnt + (static_cast<size_t>(bh) * nblk + b) * k + j);
     }

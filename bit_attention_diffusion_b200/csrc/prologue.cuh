@@ -27,6 +27,7 @@ __global__ void k_identity_perm(int32_t *perm, int N, long long total);
 
 constexpr int QUANTV1_SMEM = 128 * 272;              // gathered rows
 constexpr int QUANTV2_SMEM = 128 * 272 + 128 * 144;  // rows + transposed codes
+constexpr int KMEANS8_SMEM = 2 * 128 * 272;  // double-buffered chunk rows
 constexpr int KMEANS_SMEM_FIXED = 128 * 66 * 4;  // chunk rows; + k*128*(4+8) for centroids and sums
 
 }  // namespace vc

@@ -127,6 +127,13 @@ __device__ __forceinline__ float frame_scale(float F_from, float F_to) {
 
 __device__ __forceinline__ void softmax_bar256() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 __device__ __forceinline__ void softmax_bar128(int g) { asm volatile("bar.sync %0, 128;" ::"r"(2 + g) : "memory"); }
+// One arrive per warp on the barriers the softmax warpgroups signal (their
+// expected count is 4 warps): the warp synchronizes first, which orders every
+// lane's prior writes before lane 0's release.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
 
 // Restore chunks. Chunk X (KV tiles 32X .. 32X+31) is flushed by the tail of
 // tile 32X+33, which reads l_{32X+31}; the chunks whose flush tile would lie
@@ -173,14 +180,14 @@ __global__ void __launch_bounds__(352, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.mufull[i], 1); mbar_init(&bars.muempty[i], 1);
-      mbar_init(&bars.sfull[i], 1); mbar_init(&bars.sfree[i], 128); mbar_init(&bars.pfull[i], 128);
-      mbar_init(&bars.mxr[i], 128);
+      mbar_init(&bars.sfull[i], 1); mbar_init(&bars.sfree[i], 4); mbar_init(&bars.pfull[i], 4);
+      mbar_init(&bars.mxr[i], 4);
     }
     for (int i = 0; i < NPD; ++i) mbar_init(&bars.pvdone[i], 1);
-    mbar_init(&bars.bk, 128); mbar_init(&bars.lflush, 128); mbar_init(&bars.wgdone, 128);
+    mbar_init(&bars.bk, 4); mbar_init(&bars.lflush, 4); mbar_init(&bars.wgdone, 4);
     mbar_init(&bars.main, 2);  // one commit from each issuing warp
-    mbar_init(&bars.epi, 128); mbar_init(&bars.rdone, 1);
-    mbar_init(&bars.repk, 128); mbar_init(&bars.reps, 1); mbar_init(&bars.repp, 128);
+    mbar_init(&bars.epi, 4); mbar_init(&bars.rdone, 1);
+    mbar_init(&bars.repk, 4); mbar_init(&bars.reps, 1); mbar_init(&bars.repp, 4);
     mbar_init(&bars.repdone, 1); mbar_init(&bars.dt, 1); mbar_init(&bars.fin, 1);
     fence_mbar_init();
   }
@@ -216,7 +223,6 @@ __global__ void __launch_bounds__(352, 1)
     }
     return true;
   };
-
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // Lane 0 streams Q and the K tiles (then the repair deltas), lane 1 the V
@@ -448,7 +454,7 @@ __global__ void __launch_bounds__(352, 1)
         tmem_ld32(trow + TM_S0 + b * 128 + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * i]));
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&bars.sfree[b]);  // the issuer may now compute S(t+2) into this buffer
+      warp_arrive(&bars.sfree[b]);  // the issuer may now compute S(t+2) into this buffer
       float s[128];
 #pragma unroll
       for (int j = 0; j < 128; ++j) s[j] = __uint_as_float(sr[j]);
@@ -481,7 +487,7 @@ __global__ void __launch_bounds__(352, 1)
       const float Fn = fmaxf(F_prev, 8.0f * ceilf(__fmul_rn(mx, alpha) * 0.125f));
       if (t == 0) F_prev = Fn;
       s_F[r] = Fn;  // for tile t+1 (after the last tile it holds the final frame)
-      if (t + 1 < T) mbar_arrive(&bars.mxr[b]);
+      if (t + 1 < T) warp_arrive(&bars.mxr[b]);
       const bool need = Fn != F_prev;
       const float sc = need ? frame_scale(F_prev, Fn) : 1.0f;
       const bool anyneed = __any_sync(0xFFFFFFFFu, need);
@@ -524,7 +530,7 @@ __global__ void __launch_bounds__(352, 1)
       }
       tmem_wait_st();  // the P bytes (and any O rescale) are in TMEM
       tc_fence_before();
-      mbar_arrive(&bars.pfull[b]);
+      warp_arrive(&bars.pfull[b]);
 
       // ---- row-sum bookkeeping of this warpgroup, off the PV path
       if (g == 0 && t >= 34 && ((t - 34) & 31) == 0) {
@@ -566,10 +572,10 @@ __global__ void __launch_bounds__(352, 1)
           flush(32, sc);
           fence_proxy_async_smem();
           tc_fence_before();
-          mbar_arrive(&bars.lflush);  // the restore follows PV(t)
+          warp_arrive(&bars.lflush);  // the restore follows PV(t)
         }
       }
-      if (g == 0 && t >= 32 && (t & 31) == 0) mbar_arrive(&bars.bk);
+      if (g == 0 && t >= 32 && (t & 31) == 0) warp_arrive(&bars.bk);
       F_own = Fn;
       F_hand = F_prev;
       return true;
@@ -595,7 +601,7 @@ __global__ void __launch_bounds__(352, 1)
       s_lto[r] = lt_own;  // frame F_{T-2}, the frame the last tile was handed
       s_lprev[0][r] = lprev0;
       s_lprev[1][r] = lprev1;
-      mbar_arrive(&bars.wgdone);
+      warp_arrive(&bars.wgdone);
     }
     if (ok && fin_wg) ok = wwait(&bars.main, 0) && wwait(&bars.wgdone, 0);
     const float F_fin = F_own;  // frame of the last tile (meaningful in fin_wg)
@@ -623,7 +629,7 @@ __global__ void __launch_bounds__(352, 1)
           flush(slot + 1, sc_o);
           fence_proxy_async_smem();
           tc_fence_before();
-          mbar_arrive(&bars.epi);
+          warp_arrive(&bars.epi);
           ++e;
         }
       }
@@ -656,7 +662,7 @@ __global__ void __launch_bounds__(352, 1)
       s_alphaR[r] = al * TWO_M24;
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars.repk);
+      warp_arrive(&bars.repk);
       softmax_bar128(g);  // s_alphaR visible to every row of this warpgroup
       ok = wwait(&bars.reps, rc & 1);
       if (!ok) continue;  // one barrier per iteration on every path
@@ -689,7 +695,7 @@ __global__ void __launch_bounds__(352, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars.repp);
+      warp_arrive(&bars.repp);
     }
     // ---------------------------------------------------------- epilogue (each warpgroup 64 columns)
     if (ok) ok = wwait(&bars.fin, 0);

@@ -112,6 +112,23 @@ class ClockSampler:
                 "power_w_max": max(power), "reasons": sorted(reasons)}
 
 
+def max_over_ranks(val: float, world: int, device: str = "cuda") -> float:
+    """Largest value over all ranks of the default process group (identity at world 1)."""
+    if world == 1:
+        return val
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([val], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes its own copy of the workload
+    (independent heads, no exchange), timed by the slowest rank."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def _dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -227,12 +244,6 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(val: float) -> float:
-        if world == 1:
-            return val
-        t = torch.tensor([val], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # ---- main timed region: K full steps (clustering inside the call)
     for _ in range(args.warmup):
@@ -254,10 +265,10 @@ def run_ours(args):
     barrier()
     ph_mean = vcattn.vc_attn_profile_read()  # mean over the timed steps (<= 64), read after the loop
     vcattn.vc_attn_profile(False)
-    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world)
     ms_step = ms_total / args.steps
     flops = wl.flops
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = job_tflops(world, flops, ms_step)
     if len(ph_mean) != 4:
         ph_mean = [0.0, 0.0, 0.0, 0.0]
     attn_ms = float(ph_mean[3])
@@ -282,7 +293,7 @@ def run_ours(args):
         step(perm)
     e1.record(stream)
     e1.synchronize()
-    ms_cached = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    ms_cached = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
 
     # ---- BF16 comparator kernel
     for _ in range(args.warmup):
@@ -293,7 +304,7 @@ def run_ours(args):
         vcattn.fwd_ref_bf16(q, k, v, out=out)
     e1.record(stream)
     e1.synchronize()
-    ms_ref = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    ms_ref = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
 
     # ---- end to end through the C ABI with host buffers
     hq, hk, hv = (torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True) for _ in range(3))
@@ -316,7 +327,7 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     e1.synchronize()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
     bytes_in = 3 * q.numel() * 2
     bytes_out = out.numel() * 2
 

@@ -85,7 +85,7 @@ constexpr uint32_t IDESC_BF = idesc_make(1, 1, 128, 128, false, false);  // bf16
 
 struct Bars {
   uint64_t q, kfull[KS], kempty[KS], vfull[VS], vempty[VS], mufull[2], muempty[2];
-  uint64_t sfull[2], sfree[2], pfull[2], mxr[2], pvdone[NPD], bk, lflush, wgdone, main, epi, rdone, repk, reps,
+  uint64_t sfull[2], sfree[2], pfull[4], mxr[2], pvdone[NPD], bk, lflush, wgdone, main, epi, rdone, repk, reps,
       repp, repdone, dt, fin;
 };
 
@@ -180,10 +180,14 @@ __global__ void __launch_bounds__(352, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.mufull[i], 1); mbar_init(&bars.muempty[i], 1);
-      mbar_init(&bars.sfull[i], 1); mbar_init(&bars.sfree[i], 4); mbar_init(&bars.pfull[i], 4);
+      mbar_init(&bars.sfull[i], 1); mbar_init(&bars.sfree[i], 4);
       mbar_init(&bars.mxr[i], 4);
     }
     for (int i = 0; i < NPD; ++i) mbar_init(&bars.pvdone[i], 1);
+    // pfull is indexed t % 4: before a warpgroup arrives for tile t+4, its
+    // bookkeeping of tile t+2 has waited for PV(t+1), so the issuer has already
+    // consumed pfull(t); a barrier never runs two phases ahead of its waiter
+    for (int i = 0; i < 4; ++i) mbar_init(&bars.pfull[i], 4);
     mbar_init(&bars.bk, 4); mbar_init(&bars.lflush, 4); mbar_init(&bars.wgdone, 4);
     mbar_init(&bars.main, 2);  // one commit from each issuing warp
     mbar_init(&bars.epi, 4); mbar_init(&bars.rdone, 1);
@@ -322,7 +326,7 @@ __global__ void __launch_bounds__(352, 1)
         const int s = t % VS;
         ok = mwait(&bars.vfull[s], (t / VS) & 1);
         if (!ok) break;
-        ok = mwait(&bars.pfull[t & 1], (t >> 1) & 1);
+        ok = mwait(&bars.pfull[t & 3], (t >> 2) & 1);
         if (!ok) break;
         tc_fence_after();
         if (elect_one()) {
@@ -530,7 +534,7 @@ __global__ void __launch_bounds__(352, 1)
       }
       tmem_wait_st();  // the P bytes (and any O rescale) are in TMEM
       tc_fence_before();
-      warp_arrive(&bars.pfull[b]);
+      warp_arrive(&bars.pfull[t & 3]);
 
       // ---- row-sum bookkeeping of this warpgroup, off the PV path
       if (g == 0 && t >= 34 && ((t - 34) & 31) == 0) {

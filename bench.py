@@ -112,6 +112,9 @@ class ClockSampler:
                 "power_w_max": max(power), "reasons": sorted(reasons)}
 
 
+E2E_HEADS_PER_RUN = 2  # heads per run of the end-to-end call (copies overlap compute)
+
+
 def max_over_ranks(val: float, world: int, device: str = "cuda") -> float:
     """Largest value over all ranks of the default process group (identity at world 1)."""
     if world == 1:
@@ -313,12 +316,19 @@ def run_ours(args):
         hbuf.copy_(torch.from_numpy(np.ascontiguousarray(x[n]).view(np.int16)).view(torch.bfloat16))
     hout = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
 
+    # vc_attn_fwd_host: runs of E2E_HEADS_PER_RUN heads, host->device copies of a
+    # run overlapped with the computation of the previous one and the copy-out
+    # of the one before (q, k, v, out serve as the device staging buffers)
+    runs = max(1, (B * H) // E2E_HEADS_PER_RUN)
+    gh = -(-(B * H) // runs)
+    ws_run, ws_run_bytes = vcattn.workspace(1, gh, N, p)
+
     def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
+        st = vcattn.vc_attn_fwd_host(hq.data_ptr(), hk.data_ptr(), hv.data_ptr(), B, H, N, d, p, hout.data_ptr(),
+                                     q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), runs,
+                                     ws_run.data_ptr(), ws_run_bytes, sptr)
+        if st != 0:
+            raise vcattn.VcError(st, "vc_attn_fwd_host")
 
     for _ in range(args.warmup):
         e2e_step()

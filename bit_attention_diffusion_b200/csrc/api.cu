@@ -478,6 +478,75 @@ int vc_attn_profile_read(float *ms, int max_n) {
   return 4;
 }
 
+// End-to-end forward from host buffers: runs of consecutive heads, copy-in on
+// one stream, compute on the caller's stream, copy-out on another; each stream
+// waits for the event of the previous stage of the same run. An event can be
+// re-recorded after a wait has been issued on it (the wait binds to the record
+// current at the time of the wait), so one event per direction suffices.
+vc_status vc_attn_fwd_host(const void *hQ, const void *hK, const void *hV, int B, int H, int N, int d,
+                           const vc_params *p, void *hO, void *dQ, void *dK, void *dV, void *dO, int groups,
+                           void *ws, size_t ws_bytes, void *stream) {
+  vc_status st = check_shape(B, H, N, d);
+  if (st != VC_OK) return st;
+  if ((st = check_params(p)) != VC_OK) return st;
+  if (!hQ || !hK || !hV || !hO || !dQ || !dK || !dV || !dO || groups < 1 || !aligned(dQ, 16) || !aligned(dK, 16) ||
+      !aligned(dV, 16) || !aligned(dO, 16) || !ws || !aligned(ws, 256))
+    return VC_ERR_INVALID_ARG;
+  const long long BH = static_cast<long long>(B) * H;
+  const int G = static_cast<int>(std::min<long long>(groups, BH));
+  const int gh = static_cast<int>((BH + G - 1) / G);
+  // the workspace must hold one run of gh heads; vc_attn_fwd checks the rest
+  if (vc_attn_workspace_bytes(1, gh, N, d, p) > ws_bytes) return VC_ERR_WORKSPACE;
+  st = check_device();
+  if (st != VC_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_in = nullptr, ev_out = nullptr, ev_done = nullptr;
+  auto release = [&]() {
+    if (ev_start) cudaEventDestroy(ev_start);
+    if (ev_in) cudaEventDestroy(ev_in);
+    if (ev_out) cudaEventDestroy(ev_out);
+    if (ev_done) cudaEventDestroy(ev_done);
+    if (s_in) cudaStreamDestroy(s_in);  // released once its work completes
+    if (s_out) cudaStreamDestroy(s_out);
+  };
+  if (cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ev_out, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming) != cudaSuccess) {
+    release();
+    return VC_ERR_CUDA;
+  }
+  bool ok = cudaEventRecord(ev_start, s) == cudaSuccess && cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess;
+  const size_t head_bytes = static_cast<size_t>(N) * d * sizeof(uint16_t);
+  for (int g = 0; g < G && ok && st == VC_OK; ++g) {
+    const long long h0 = static_cast<long long>(g) * gh;
+    if (h0 >= BH) break;
+    const int hn = static_cast<int>(std::min<long long>(gh, BH - h0));
+    const size_t off = static_cast<size_t>(h0) * head_bytes, bytes = static_cast<size_t>(hn) * head_bytes;
+    auto at = [&](const void *base) { return static_cast<const char *>(base) + off; };
+    auto atw = [&](void *base) { return static_cast<char *>(base) + off; };
+    ok = cudaMemcpyAsync(atw(dQ), at(hQ), bytes, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+         cudaMemcpyAsync(atw(dK), at(hK), bytes, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+         cudaMemcpyAsync(atw(dV), at(hV), bytes, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+         cudaEventRecord(ev_in, s_in) == cudaSuccess && cudaStreamWaitEvent(s, ev_in, 0) == cudaSuccess;
+    if (!ok) break;
+    st = vc_attn_fwd(at(dQ), at(dK), at(dV), 1, hn, N, d, nullptr, p, atw(dO), ws, ws_bytes, stream);
+    if (st != VC_OK) break;
+    ok = cudaEventRecord(ev_out, s) == cudaSuccess && cudaStreamWaitEvent(s_out, ev_out, 0) == cudaSuccess &&
+         cudaMemcpyAsync(atw(hO), at(dO), bytes, cudaMemcpyDeviceToHost, s_out) == cudaSuccess;
+  }
+  // the caller's stream resumes after the last copy-out (also on an error path,
+  // so that nothing of this call is left running unordered)
+  const bool tail_ok = cudaEventRecord(ev_done, s_out) == cudaSuccess && cudaStreamWaitEvent(s, ev_done, 0) == cudaSuccess;
+  release();
+  if (st != VC_OK) return st;
+  return (ok && tail_ok) ? VC_OK : VC_ERR_CUDA;
+}
+
 vc_status vc_attn_fwd_ref_bf16(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
                                float softmax_scale, void *O, void *stream) {
   vc_status st = check_shape(B, H, N, d);

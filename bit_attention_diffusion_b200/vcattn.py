@@ -30,7 +30,7 @@ EXPORTED = [
     "vc_attn_cluster", "vc_attn_quant_qk", "vc_attn_quant_v", "vc_attn_fwd", "vc_attn_fwd_ref_bf16",
     "vc_attn_expcast", "vc_attn_e4m3_encode", "vc_attn_device_status", "vc_attn_wait_selftest",
     "vc_attn_launch_count", "vc_attn_profile", "vc_attn_profile_read",
-    "vc_attn_cluster_noalloc", "vc_attn_cluster_noalloc_max_bytes",
+    "vc_attn_cluster_noalloc", "vc_attn_cluster_noalloc_max_bytes", "vc_attn_fwd_host",
 ]
 
 
@@ -72,6 +72,7 @@ def lib():
             L.vc_attn_quant_qk.argtypes = [P, P, P, I, I, I, I, PP, P, P, P, P, P, Z, P]
             L.vc_attn_quant_v.argtypes = [P, P, I, I, I, I, PP, P, P, P, P, P, P, Z, P]
             L.vc_attn_fwd.argtypes = [P, P, P, I, I, I, I, P, PP, P, P, Z, P]
+            L.vc_attn_fwd_host.argtypes = [P, P, P, I, I, I, I, PP, P, P, P, P, P, I, P, Z, P]
             L.vc_attn_fwd_ref_bf16.argtypes = [P, P, P, I, I, I, I, F, P, P]
             L.vc_attn_expcast.argtypes = [P, P, P, LL, P, P]
             L.vc_attn_e4m3_encode.argtypes = [P, LL, P, P]
@@ -139,6 +140,11 @@ def vc_attn_quant_v(V, perm, B, H, N, d, p, v8, v_scale, v_mean, rep_idx, rep_de
 
 def vc_attn_fwd(Q, K, V, B, H, N, d, perm, p, O, ws, ws_bytes, stream) -> int:
     return lib().vc_attn_fwd(Q, K, V, B, H, N, d, perm, ctypes.byref(p), O, ws, ws_bytes, stream)
+
+
+def vc_attn_fwd_host(hQ, hK, hV, B, H, N, d, p, hO, dQ, dK, dV, dO, groups, ws, ws_bytes, stream) -> int:
+    return lib().vc_attn_fwd_host(hQ, hK, hV, B, H, N, d, ctypes.byref(p), hO, dQ, dK, dV, dO, groups, ws, ws_bytes,
+                                  stream)
 
 
 def vc_attn_fwd_ref_bf16(Q, K, V, B, H, N, d, softmax_scale, O, stream) -> int:
@@ -227,6 +233,28 @@ def fwd(q, k, v, perm=None, p: VcParams | None = None, out=None, ws=None, stream
     _check(vc_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, _ptr(perm), p, out.data_ptr(),
                        ws.data_ptr(), nbytes, _stream(stream)), "vc_attn_fwd")
     return out
+
+
+def fwd_host(hq, hk, hv, groups: int, p: VcParams | None = None, hout=None, dev=None, ws=None, stream=None):
+    """O = VC-Attention FP8 forward from host (CPU, ideally pinned) bf16 [B,H,N,128]
+    tensors; the device staging tensors `dev` = (dQ, dK, dV, dO) and the
+    workspace for one run of ceil(B*H/groups) heads are allocated if not given."""
+    torch = _torch()
+    p = p or params()
+    B, H, N, d = _shape(hq)
+    if hout is None:
+        hout = torch.empty_like(hq, pin_memory=True)
+    if dev is None:
+        dev = tuple(torch.empty(hq.shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    gh = -(-(B * H) // min(groups, B * H))
+    if ws is None:
+        ws, nbytes = workspace(1, gh, N, p)
+    else:
+        nbytes = ws.numel()
+    _check(vc_attn_fwd_host(hq.data_ptr(), hk.data_ptr(), hv.data_ptr(), B, H, N, d, p, hout.data_ptr(),
+                            *(t.data_ptr() for t in dev), groups, ws.data_ptr(), nbytes, _stream(stream)),
+           "vc_attn_fwd_host")
+    return hout
 
 
 def cluster(v, p: VcParams | None = None, ws=None, stream=None):

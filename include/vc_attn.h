@@ -179,6 +179,40 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
                       const int32_t *perm, const vc_params *p, void *O, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * vc_attn_fwd from host memory: the same forward pass (clustering inside the
+ * call), with Q, K, V read from host buffers and O written to a host buffer.
+ * The (b,h) heads are split into `groups` runs of consecutive heads. Every step
+ * of the method is per head, so the result is bit-identical to vc_attn_fwd.
+ *
+ * Per run, the call:
+ *   1. copies the run's Q, K and V slices host -> device;
+ *   2. runs the forward on that run;
+ *   3. copies the run's O slice back device -> host.
+ * The copies go on two streams the call creates and releases, so the copy-in of
+ * one run and the copy-out of another overlap the computation of a third.
+ *
+ * Host buffers: hQ, hK, hV, hO, [B][H][N][d] bf16. They should be page-locked
+ * (cudaHostAlloc or cudaHostRegister); pageable memory works but does not
+ * overlap.
+ * Device buffers: dQ, dK, dV, dO, each B*H*N*d bf16, owned by the caller and
+ * used as staging.
+ * Workspace: ws is a workspace for ONE run, i.e.
+ *   vc_attn_workspace_bytes(1, ceil(B*H / groups), N, d, p).
+ * groups: 1 .. B*H; it is clamped to B*H.
+ *
+ * Ordering: the call is asynchronous. Its work is ordered after earlier work on
+ * `stream`, and later work on `stream` is ordered after its last copy.
+ * Errors: as vc_attn_fwd, plus VC_ERR_INVALID_ARG for a null host or device
+ * pointer or groups < 1.
+ *
+ * The pages give no host interface (the kernel is proprietary); this call is the
+ * end-to-end form of vc_attn_fwd that the measurement uses.
+ */
+vc_status vc_attn_fwd_host(const void *hQ, const void *hK, const void *hV, int B, int H, int N, int d,
+                           const vc_params *p, void *hO, void *dQ, void *dK, void *dV, void *dO, int groups,
+                           void *ws, size_t ws_bytes, void *stream);
+
+/*
  * In-library comparator: exact-softmax attention in BF16 on the tcgen05
  * tensor cores (bf16 operands, fp32 accumulation, fp32 exp2 softmax).
  * softmax_scale 0 => 1/sqrt(d). O bf16 [B,H,N,d].

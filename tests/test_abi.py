@@ -104,3 +104,30 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     with pytest.raises(RuntimeError, match="missing"):
         mod.lib()
     importlib.reload(vcattn)
+
+
+@pytest.mark.parametrize("case,status", [
+    (dict(d=96), vcattn.VC_ERR_UNSUPPORTED),
+    (dict(groups=0), vcattn.VC_ERR_INVALID_ARG),
+    (dict(null_host=True), vcattn.VC_ERR_INVALID_ARG),
+    (dict(dev_off=8), vcattn.VC_ERR_INVALID_ARG),                # device staging not 16-byte aligned
+    (dict(ws_bytes=1024), vcattn.VC_ERR_WORKSPACE),             # smaller than one run of heads
+])
+def test_fwd_host_rejects_bad_arguments_on_host(L, case, status):
+    p = vcattn.params()
+    d = case.get("d", 128)
+    host = 0 if case.get("null_host") else FAKE
+    dev = FAKE + case.get("dev_off", 0)
+    st = vcattn.vc_attn_fwd_host(host, FAKE, FAKE, 1, 4, 256, d, p, FAKE, dev, FAKE, FAKE, FAKE,
+                                 case.get("groups", 2), FAKE, case.get("ws_bytes", 1 << 40), None)
+    assert st == status
+
+
+def test_fwd_host_workspace_is_sized_for_one_run_of_heads(L):
+    """The workspace needed is the one for a run of ceil(B*H/groups) heads (here
+    B*H = 6 in 2 runs of 3): one byte less is rejected before any device work."""
+    p = vcattn.params()
+    need = vcattn.vc_attn_workspace_bytes(1, 3, 256, 128, p)   # B*H = 6, groups = 2 -> runs of 3 heads
+    st = vcattn.vc_attn_fwd_host(FAKE, FAKE, FAKE, 2, 3, 256, 128, p, FAKE, FAKE, FAKE, FAKE, FAKE, 2, FAKE,
+                                 need - 1, None)
+    assert st == vcattn.VC_ERR_WORKSPACE

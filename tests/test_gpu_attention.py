@@ -199,3 +199,18 @@ def test_fwd_restore_chunk_boundaries(torch, N):
     out = _run_gpu(torch, x, vcattn.params())
     rel, worst = _compare(x, out, [(0, 0), (0, 1)], lambda n: _sampled_rows(n, 48), oracle.FLAGS_DEFAULT)
     assert rel <= TOL and worst <= 2 * TOL, (rel, worst)
+
+
+@pytest.mark.parametrize("groups", [1, 2, 7])
+def test_fwd_host_equals_device_call(torch, groups):
+    """vc_attn_fwd_host (host buffers, runs of heads, copies overlapped with
+    compute) gives bit-identical output to vc_attn_fwd on device buffers;
+    groups = 2 leaves a shorter last run (7 heads in runs of 4 and 3)."""
+    B, H, N = 1, 7, 700
+    x = synth.make_inputs(synth.custom(B, H, N, seed=800 + groups))
+    q, k, v = (to_dev_bf16(x[n]) for n in "qkv")
+    ref = vcattn.fwd(q, k, v, p=vcattn.params())
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hout = vcattn.fwd_host(hq, hk, hv, groups, p=vcattn.params())
+    torch.cuda.synchronize()
+    assert torch.equal(hout, ref.cpu())

@@ -270,7 +270,10 @@ void launch_quant_v(const Shape &sh, const Ws &w, const uint16_t *V, const int32
                                                      v8t, w.at<float>(w.L.err), w.at<uint16_t>(w.L.mut2));
   count_launch();
   if (sh.R > 0) {
-    k_repair_select<<<sh.BH, 1024, 0, s>>>(w.at<float>(w.L.err), sh.N, sh.R, rep_idx);
+    if (sh.N <= 512 * 64)
+      k_repair_select_reg<<<sh.BH, 512, 0, s>>>(w.at<float>(w.L.err), sh.N, sh.R, rep_idx);
+    else
+      k_repair_select<<<sh.BH, 1024, 0, s>>>(w.at<float>(w.L.err), sh.N, sh.R, rep_idx);
     count_launch();
     k_repair_delta<<<dim3((sh.Rpad + 7) / 8, sh.BH), 256, 0, s>>>(V, perm, sh.N, sh.Nb, sh.R, sh.Rpad, rep_idx,
                                                                   vmean, vscale, vexpo, rep_delta,

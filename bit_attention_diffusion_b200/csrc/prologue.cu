@@ -774,6 +774,103 @@ __global__ void __launch_bounds__(1024) k_repair_select(const float *__restrict_
   }
 }
 
+// Same selection for N <= 32768, with no serial step: the keys stay in
+// registers (key i of thread t is position 512 i + t); each radix pass picks
+// its digit with a block scan of the 256-bin histogram; the ordered compaction
+// counts (chunk, warp) hits for all chunks at once, scans those counts once and
+// writes every taken position in a second sweep.
+constexpr int RS_T = 512, RS_KPT = 64, RS_W = RS_T / 32;
+
+// Inclusive scan of one value per thread over the first `nthreads` threads
+// (a multiple of 32, <= RS_T), through warp shuffles and one shared array.
+__device__ __forceinline__ unsigned rs_block_scan(unsigned v, unsigned *wsum, int nthreads) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (tid < nthreads && lane == 31) wsum[warp] = x;
+  __syncthreads();
+  unsigned add = 0u;
+  for (int w = 0; w < warp && tid < nthreads; ++w) add += wsum[w];
+  __syncthreads();
+  return x + add;
+}
+
+__global__ void __launch_bounds__(RS_T) k_repair_select_reg(const float *__restrict__ err, int N, int R,
+                                                            int32_t *__restrict__ rep_idx) {
+  __shared__ unsigned hist[256];
+  __shared__ unsigned wsum[RS_W];
+  __shared__ unsigned s_digit, s_run;
+  __shared__ unsigned cgt[RS_KPT * RS_W], ceq[RS_KPT * RS_W];
+  const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const unsigned *keyg = reinterpret_cast<const unsigned *>(err + static_cast<size_t>(bh) * N);
+  int32_t *out = rep_idx + static_cast<size_t>(bh) * R;
+  unsigned key[RS_KPT];
+#pragma unroll
+  for (int i = 0; i < RS_KPT; ++i) {
+    const int n = RS_T * i + tid;
+    key[i] = n < N ? __ldg(keyg + n) : 0u;
+  }
+  unsigned prefix = 0u, mask = 0u, need = static_cast<unsigned>(R);
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    if (tid < 256) hist[tid] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < RS_KPT; ++i)
+      if (RS_T * i + tid < N && (key[i] & mask) == prefix) atomicAdd(&hist[(key[i] >> shift) & 0xFFu], 1u);
+    __syncthreads();
+    // thread j holds digit 255 - j: the inclusive scan over j counts the keys
+    // whose digit is >= 255 - j; the digit where that count first reaches
+    // `need` is the one of the R-th largest key (counts here sum to >= need)
+    const unsigned c = tid < 256 ? hist[255 - tid] : 0u;
+    const unsigned incl = rs_block_scan(c, wsum, 256);
+    if (tid < 256 && incl >= need && incl - c < need) {
+      s_digit = 255u - static_cast<unsigned>(tid);
+      s_run = incl - c;
+    }
+    __syncthreads();
+    need -= s_run;
+    prefix |= s_digit << shift;
+    mask |= 0xFFu << shift;
+  }
+  const unsigned T = prefix;  // the R-th largest key; `need` keys equal to T are taken
+  // ---- ordered compaction (ascending position; ties to the lowest positions)
+#pragma unroll
+  for (int i = 0; i < RS_KPT; ++i) {
+    const int n = RS_T * i + tid;
+    const unsigned bg = __ballot_sync(0xFFFFFFFFu, n < N && key[i] > T);
+    const unsigned be = __ballot_sync(0xFFFFFFFFu, n < N && key[i] == T);
+    if (lane == 0) {
+      cgt[i * RS_W + warp] = __popc(bg);
+      ceq[i * RS_W + warp] = __popc(be);
+    }
+  }
+  __syncthreads();
+  {  // exclusive scan of the (chunk, warp) counts, two entries per thread
+    const unsigned g0 = cgt[2 * tid], g1 = cgt[2 * tid + 1], e0 = ceq[2 * tid], e1 = ceq[2 * tid + 1];
+    const unsigned ig = rs_block_scan(g0 + g1, wsum, RS_T);
+    const unsigned ie = rs_block_scan(e0 + e1, wsum, RS_T);
+    cgt[2 * tid] = ig - g0 - g1;
+    cgt[2 * tid + 1] = ig - g1;
+    ceq[2 * tid] = ie - e0 - e1;
+    ceq[2 * tid + 1] = ie - e1;
+  }
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int i = 0; i < RS_KPT; ++i) {
+    const int n = RS_T * i + tid;
+    const bool gt = n < N && key[i] > T, eq = n < N && key[i] == T;
+    const unsigned bg = __ballot_sync(0xFFFFFFFFu, gt), be = __ballot_sync(0xFFFFFFFFu, eq);
+    const unsigned rank_eq = ceq[i * RS_W + warp] + __popc(be & lt);  // equal keys before this one
+    const unsigned pos = cgt[i * RS_W + warp] + __popc(bg & lt) + min(rank_eq, need);
+    if (gt || (eq && rank_eq < need)) out[pos] = n;
+  }
+}
+
 // delta = bf16(r - value(code)*scale) for every repaired token; also the
 // channel-major copy divided by the channel scale (deltat[bh][c][r], zero for
 // r in [R, Rpad)) that the attention kernel's repair MMA reads.

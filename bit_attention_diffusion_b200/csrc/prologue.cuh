@@ -20,6 +20,7 @@ __global__ void k_quantv_pass2(const uint16_t *V, const int32_t *perm, int N, in
                                const uint16_t *vmean, const float *vscale, const int *vexpo, uint8_t *v8t, float *err,
                                uint16_t *mut2);
 __global__ void k_repair_select(const float *err, int N, int R, int32_t *rep_idx);
+__global__ void k_repair_select_reg(const float *err, int N, int R, int32_t *rep_idx);
 __global__ void k_repair_delta(const uint16_t *V, const int32_t *perm, int N, int Nb, int R, int Rpad,
                                const int32_t *rep_idx, const uint16_t *vmean, const float *vscale, const int *vexpo,
                                uint16_t *rep_delta, uint16_t *deltat);

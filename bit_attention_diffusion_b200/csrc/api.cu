@@ -164,7 +164,7 @@ vc_status check_params(const vc_params *p) {
   if (!(p->rho >= 0.0f && p->rho < 1.0f)) return VC_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.0f) || !std::isfinite(p->softmax_scale)) return VC_ERR_INVALID_ARG;
   if (p->expcast_bias < 8 || p->expcast_bias > 126) return VC_ERR_INVALID_ARG;
-  if (p->flags & ~(VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH)) return VC_ERR_INVALID_ARG;
+  if (p->flags & ~(VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH | VC_WARMSTART)) return VC_ERR_INVALID_ARG;
   return VC_OK;
 }
 
@@ -223,8 +223,10 @@ vc_status clear_small(const Ws &w, cudaStream_t s) {
 
 void launch_cluster(const Shape &sh, const Ws &w, const uint16_t *V, int32_t *perm, float *cent, cudaStream_t s) {
   int32_t *labels = w.at<int32_t>(w.L.labels);
-  k_kmeans_init<<<sh.BH, 128, 0, s>>>(V, sh.N, sh.k, cent);
-  count_launch();
+  if (!(sh.flags & VC_WARMSTART)) {  // warm start: cent already holds the previous step's centroids
+    k_kmeans_init<<<sh.BH, 128, 0, s>>>(V, sh.N, sh.k, cent);
+    count_launch();
+  }
   const size_t smem = KMEANS_SMEM_FIXED + static_cast<size_t>(sh.k) * D * 12;
   const dim3 grid(sh.km_nblk, sh.BH);
   for (int it = 0; it <= sh.iters; ++it) {
@@ -333,7 +335,8 @@ vc_status vc_attn_cluster(const void *V, int B, int H, int N, int d, const vc_pa
   Ws w;
   vc_status st = prep(B, H, N, d, p, ws, ws_bytes, &sh, &w);
   if (st != VC_OK) return st;
-  if (!V || !perm || !aligned(V, 16) || !aligned(perm, 16) || (centroids && !aligned(centroids, 16)))
+  if (!V || !perm || !aligned(V, 16) || !aligned(perm, 16) || (centroids && !aligned(centroids, 16)) ||
+      ((sh.flags & VC_WARMSTART) && !centroids))
     return VC_ERR_INVALID_ARG;
   if ((st = check_device()) != VC_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -396,7 +399,9 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
   prof_mark(0, s);
   const int32_t *pm = perm;
   if (!pm && (sh.flags & VC_VSMOOTH)) {
-    launch_cluster(sh, w, Vh, w.at<int32_t>(w.L.perm), w.at<float>(w.L.cent), s);
+    Shape cold = sh;  // vc_attn_fwd has no centroid input: always the default start
+    cold.flags &= ~VC_WARMSTART;
+    launch_cluster(cold, w, Vh, w.at<int32_t>(w.L.perm), w.at<float>(w.L.cent), s);
     pm = w.at<int32_t>(w.L.perm);
   }
   prof_mark(1, s);

@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libvcattn.so")
 
 VC_OK, VC_ERR_INVALID_ARG, VC_ERR_UNSUPPORTED, VC_ERR_WORKSPACE, VC_ERR_CUDA, VC_ERR_TIMEOUT = range(6)
-VC_VSMOOTH, VC_REPAIR, VC_KSMOOTH = 1, 2, 8
+VC_VSMOOTH, VC_REPAIR, VC_KSMOOTH, VC_WARMSTART = 1, 2, 8, 16
 FLAGS_DEFAULT = VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH
 D = 128
 
@@ -257,8 +257,10 @@ def fwd_host(hq, hk, hv, groups: int, p: VcParams | None = None, hout=None, dev=
     return hout
 
 
-def cluster(v, p: VcParams | None = None, ws=None, stream=None):
-    """V-Smooth Group: returns (perm int32 [B,H,N], centroids fp32 [B,H,k,128])."""
+def cluster(v, p: VcParams | None = None, ws=None, stream=None, init=None):
+    """V-Smooth Group: returns (perm int32 [B,H,N], centroids fp32 [B,H,k,128]).
+    `init` (fp32 [B,H,k,128] on the device): warm start from these centroids
+    (VC_WARMSTART), e.g. the previous denoising step's."""
     torch = _torch()
     p = p or params()
     B, H, N, d = _shape(v)
@@ -267,10 +269,36 @@ def cluster(v, p: VcParams | None = None, ws=None, stream=None):
     else:
         nbytes = ws.numel()
     perm = torch.empty((B, H, N), dtype=torch.int32, device=v.device)
-    cent = torch.empty((B, H, p.k, D), dtype=torch.float32, device=v.device)
+    if init is None:
+        cent = torch.empty((B, H, p.k, D), dtype=torch.float32, device=v.device)
+    else:
+        cent = init.to(dtype=torch.float32).contiguous().clone()
+        p = VcParams(p.k, p.iters, p.rho, p.softmax_scale, p.expcast_bias, p.flags | VC_WARMSTART)
     _check(vc_attn_cluster(v.data_ptr(), B, H, N, d, p, perm.data_ptr(), cent.data_ptr(), ws.data_ptr(), nbytes,
                            _stream(stream)), "vc_attn_cluster")
     return perm, cent
+
+
+class VSmoothSchedule:
+    """Cross-step V-Smooth over a denoising run: the value grouping is
+    recomputed (warm-started from the previous step's centroids) only in the
+    first `cluster_fraction` of the steps; later steps reuse the last
+    permutation. `perm(v, step)` returns the permutation to pass to fwd()."""
+
+    def __init__(self, total_steps: int, cluster_fraction: float = 0.25, p: VcParams | None = None):
+        self.total = int(total_steps)
+        self.last_cluster_step = max(0, int(self.total * cluster_fraction + 0.5) - 1)
+        self.p = p or params()
+        self._perm = None
+        self._cent = None
+
+    def clusters_at(self, step: int) -> bool:
+        return step <= self.last_cluster_step or self._perm is None
+
+    def perm(self, v, step: int, ws=None, stream=None):
+        if self.clusters_at(step):
+            self._perm, self._cent = cluster(v, self.p, ws=ws, stream=stream, init=self._cent)
+        return self._perm
 
 
 def quant_qk(q, k, perm=None, p: VcParams | None = None, ws=None, stream=None):

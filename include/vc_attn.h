@@ -52,6 +52,10 @@ typedef enum {
 #define VC_VSMOOTH 1u /* V-Smooth: k-means grouping + block demean/restore */
 #define VC_REPAIR 2u  /* rho-repair of the worst-quantized value tokens */
 #define VC_KSMOOTH 8u /* subtract the per-(b,h) channel mean of K */
+/* vc_attn_cluster / vc_attn_cluster_noalloc only: start the Lloyd iterations
+ * from the centroids passed in (the previous denoising step's) instead of the
+ * tokens V[floor(j*N/k)]. Ignored by vc_attn_fwd, which clusters from scratch. */
+#define VC_WARMSTART 16u
 
 typedef struct {
   int k;             /* k-means clusters, 1..64 (default 8) */
@@ -59,7 +63,7 @@ typedef struct {
   float rho;         /* repair budget, [0, 1) (default 0.005); R = ceil(rho*N) */
   float softmax_scale; /* 0 => 1/sqrt(d) */
   int expcast_bias;  /* C: the running row maximum maps to byte C, 8..126 (default 120) */
-  unsigned flags;    /* VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH (default all) */
+  unsigned flags;    /* VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH (default), optionally VC_WARMSTART */
 } vc_params;
 
 /* Fill the defaults listed above. */
@@ -83,8 +87,11 @@ int vc_attn_repair_count(int N, const vc_params *p);
  *   V        bf16 [B,H,N,d]                       in
  *   perm     int32 [B,H,N] out: perm[p] = original index of the token at
  *            permuted position p (K and V are both read through it)
- *   centroids fp32 [B,H,k,d] out (final centroids), or NULL
- * Init c_j = V[floor(j*N/k)]; distances are fp32, accumulated by fma in
+ *   centroids fp32 [B,H,k,d] out (final centroids), or NULL; in and out
+ *            with VC_WARMSTART (then required: the starting centroids)
+ * Init c_j = V[floor(j*N/k)] (or the given centroids with VC_WARMSTART, the
+ * cross-step form of the pages' online grouping, which they run only in the
+ * first quarter of the denoising steps); distances are fp32, accumulated by fma in
  * channel order; ties go to the lowest cluster; centroid = fp32(fp64 sum /
  * count); an empty cluster keeps its centroid; `iters` rounds, then a final
  * assignment. Bit-identical to the CPU oracle.

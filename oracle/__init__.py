@@ -71,7 +71,7 @@ def lib():
             L.orc_kappa.argtypes = [f32]
             L.orc_repair_count.restype = i32
             L.orc_repair_count.argtypes = [f32, i32]
-            L.orc_kmeans_head.argtypes = [P, i32, i32, i32, i32, P, P]
+            L.orc_kmeans_head.argtypes = [P, i32, i32, i32, i32, P, P, i32]
             L.orc_stable_sort_labels.argtypes = [P, i32, i32, P]
             L.orc_quant_qk_head.argtypes = [P, P, P, i32, i32, i32, P, P, P, P, P]
             L.orc_quant_v_head.argtypes = [P, P, i32, i32, i32, i32, P, P, P, P, P, P]
@@ -144,13 +144,15 @@ def set_threads(n: int) -> int:
 
 
 # ---------------------------------------------------------------- steps, one (b,h)
-def kmeans_head(v_bits: np.ndarray, k: int = 8, iters: int = 3):
-    """V-Smooth Group: Lloyd k-means of one head's value tokens -> (centroids, labels)."""
+def kmeans_head(v_bits: np.ndarray, k: int = 8, iters: int = 3, init: np.ndarray | None = None):
+    """V-Smooth Group: Lloyd k-means of one head's value tokens -> (centroids, labels).
+    `init` (fp32 [k, d]): start from these centroids (warm start from the
+    previous step) instead of the tokens floor(j N / k)."""
     v = np.ascontiguousarray(v_bits, dtype=np.uint16)
     N, d = v.shape
-    cent = np.empty((k, d), np.float32)
+    cent = np.empty((k, d), np.float32) if init is None else np.array(init, dtype=np.float32, copy=True, order="C")
     labels = np.empty(N, np.int32)
-    lib().orc_kmeans_head(_p(v), N, d, k, iters, _p(cent), _p(labels))
+    lib().orc_kmeans_head(_p(v), N, d, k, iters, _p(cent), _p(labels), 0 if init is None else 1)
     return cent, labels
 
 

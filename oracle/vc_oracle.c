@@ -176,11 +176,15 @@ static void kmeans_assign(const uint16_t *V, int N, int d, int k, const float *c
     }
 }
 
-void orc_kmeans_head(const uint16_t *V, int N, int d, int k, int iters, float *cent, int32_t *labels)
+/* warm != 0: the iterations start from the centroids already in `cent` (the
+ * previous denoising step's, [VCA] "V-Smooth", Group: the grouping is online
+ * and runs only in the first quarter of the steps) instead of the tokens
+ * floor(j N / k). */
+void orc_kmeans_head(const uint16_t *V, int N, int d, int k, int iters, float *cent, int32_t *labels, int warm)
 {
     double *sum = (double *)calloc((size_t)k * d, sizeof(double));
     long long *cnt = (long long *)calloc((size_t)k, sizeof(long long));
-    for (int j = 0; j < k; ++j) {
+    for (int j = 0; j < k && !warm; ++j) {
         int src = (int)(((long long)j * N) / k);
         for (int c = 0; c < d; ++c)
             cent[(size_t)j * d + c] = orc_bf16_value(V[(size_t)src * d + c]);

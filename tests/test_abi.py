@@ -131,3 +131,10 @@ def test_fwd_host_workspace_is_sized_for_one_run_of_heads(L):
     st = vcattn.vc_attn_fwd_host(FAKE, FAKE, FAKE, 2, 3, 256, 128, p, FAKE, FAKE, FAKE, FAKE, FAKE, 2, FAKE,
                                  need - 1, None)
     assert st == vcattn.VC_ERR_WORKSPACE
+
+
+def test_vsmooth_schedule_clusters_in_the_first_quarter(L):
+    sched = vcattn.VSmoothSchedule(20, cluster_fraction=0.25)
+    assert sched.last_cluster_step == 4
+    sched._perm = object()   # as after a first clustering
+    assert [sched.clusters_at(s) for s in range(7)] == [True] * 5 + [False] * 2

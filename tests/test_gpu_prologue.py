@@ -96,3 +96,22 @@ def test_quant_v_ties_in_repair_take_lowest_positions(torch):
     r = vcattn.quant_v(to_dev_bf16(v), None, p)
     R = vcattn.vc_attn_repair_count(N, p)
     assert r["rep_idx"].cpu().numpy()[0, 0].tolist() == list(range(R))
+
+
+@pytest.mark.parametrize("B,H,N", [(1, 2, 1024), (2, 1, 300)])
+def test_cluster_warm_start_bit_exact(torch, B, H, N):
+    """VC_WARMSTART: starting from given centroids matches the oracle started
+    from the same centroids; and warm start from the 2-iteration centroids plus
+    3 more iterations equals the cold 5-iteration result."""
+    x = _inputs(B, H, N, seed=3)
+    v = to_dev_bf16(x["v"])
+    _, c2 = vcattn.cluster(v, vcattn.params(iters=2))
+    perm_w, cent_w = vcattn.cluster(v, vcattn.params(iters=3), init=c2)
+    perm_5, cent_5 = vcattn.cluster(v, vcattn.params(iters=5))
+    assert torch.equal(perm_w, perm_5) and torch.equal(cent_w, cent_5)
+    c2h, pw, cw = c2.cpu().numpy(), perm_w.cpu().numpy(), cent_w.cpu().numpy()
+    for b in range(B):
+        for h in range(H):
+            c_o, lab_o = oracle.kmeans_head(x["v"][b, h], 8, 3, init=c2h[b, h])
+            assert np.array_equal(pw[b, h], oracle.stable_sort_labels(lab_o, 8)), (b, h)
+            assert np.array_equal(cw[b, h].view(np.uint32), c_o.view(np.uint32)), (b, h)

@@ -196,3 +196,23 @@ def test_quant_v_constant_channel_gets_unit_scale(orc):
     assert r["vscale"][7] == 1.0
     assert np.all(r["v8"][:, 7] == 0)
     assert np.all(orc.bf16_value(r["vmean"][:, 7]) == 3.0)
+
+
+def test_kmeans_warm_start_chains_lloyd_iterations(orc):
+    """Warm start (cross-step V-Smooth): starting from the centroids a cold run
+    reached after i iterations and running m more gives exactly the cold run
+    with i + m iterations (Lloyd is a deterministic map on the centroids); and
+    starting from a fixed point changes nothing."""
+    rng = np.random.default_rng(5)
+    N, d, k = 600, 128, 5
+    v = synth.f32_to_bf16_bits(rng.standard_normal((N, d)).astype(np.float32) + 3.0 * (rng.integers(0, k, N)[:, None]
+                                                                                      == np.arange(d)[None, :] % k))
+    c2, _ = orc.kmeans_head(v, k, 2)
+    c5, l5 = orc.kmeans_head(v, k, 5)
+    cw, lw = orc.kmeans_head(v, k, 3, init=c2)
+    assert np.array_equal(cw.view(np.uint32), c5.view(np.uint32))
+    assert np.array_equal(lw, l5)
+    # run to a fixed point, then a warm start with one more iteration is the identity
+    cf, lf = orc.kmeans_head(v, k, 30)
+    cg, lg = orc.kmeans_head(v, k, 1, init=cf)
+    assert np.array_equal(cg.view(np.uint32), cf.view(np.uint32)) and np.array_equal(lg, lf)

@@ -1,4 +1,4 @@
-"""CPU oracle for VC-Attention FP8 - test infrastructure, not part of the product.
+"""CPU oracle for VC-Attention (FP8 path and NVFP4-residual variant) - test infrastructure, not part of the product.
 
 Only tests/, ``__graft_entry__.smoke()`` and bench.py's CPU-baseline leg may
 import this package. The CUDA library never loads it and shares no code with
@@ -36,6 +36,7 @@ DEFAULT_SCALE = float(np.float32(1.0 / np.sqrt(128.0)))
 FLAG_VSMOOTH = 1
 FLAG_REPAIR = 2
 FLAG_KSMOOTH = 8
+FLAG_VFMT_NVFP4 = 32
 FLAGS_DEFAULT = FLAG_VSMOOTH | FLAG_REPAIR | FLAG_KSMOOTH
 
 
@@ -84,6 +85,15 @@ def lib():
             L.orc_e4m3_value_n.argtypes = [P, i64, P]
             L.orc_bf16_round_n.argtypes = [P, i64, P]
             L.orc_expcast_n.argtypes = [P, P, P, i64, P]
+            L.orc_e2m1_value.restype = ctypes.c_double
+            L.orc_e2m1_value.argtypes = [ctypes.c_uint8]
+            L.orc_e2m1_encode.restype = ctypes.c_uint8
+            L.orc_e2m1_encode.argtypes = [f32]
+            L.orc_e2m1_encode_n.argtypes = [P, i64, P]
+            L.orc_nvfp4_p_block.argtypes = [P, i32, P, P]
+            L.orc_quant_v4_head.argtypes = [P, P, i32, i32, i32, i32, P, P, P, P, P, P, P]
+            L.orc_attn_vc4_rows.argtypes = [P, P, P, P, P, P, P, P, P, P, i32, i32, i32, f32,
+                                            P, i32, P, P, P]
             _lib = L
     return _lib
 
@@ -232,6 +242,73 @@ def attn_exactv_rows(qk: dict, v_bits, perm, N: int, rows, softmax_scale: float 
     return out
 
 
+# ---------------------------------------------------------------- NVFP4 variant
+def e2m1_value(codes) -> np.ndarray:
+    c = np.asarray(codes, dtype=np.uint8)
+    L = lib()
+    table = np.array([L.orc_e2m1_value(i) for i in range(16)], np.float64)
+    return table[c & 15]
+
+
+def e2m1_encode(x) -> np.ndarray:
+    a = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(a.shape, np.uint8)
+    lib().orc_e2m1_encode_n(_p(a), a.size, _p(out))
+    return out
+
+
+def nvfp4_p_block(x):
+    """NVFP4 codes of the probabilities 2^x of one block of <= 16 keys: (codes, scale code)."""
+    a = np.ascontiguousarray(x, dtype=np.float32)
+    assert 0 < a.size <= 16
+    codes = np.empty(a.size, np.uint8)
+    sfc = np.empty(1, np.uint8)
+    lib().orc_nvfp4_p_block(_p(a), a.size, _p(codes), _p(sfc))
+    return codes, int(sfc[0])
+
+
+def quant_v4_head(v_bits, perm, demean: bool = True, R: int = 0):
+    """NVFP4 residual of one head: codes [N, d] (low nibble), block scale codes
+    [ceil(N/16), d], per-channel global scales g [d], block means, token errors,
+    the repair list and its deltas."""
+    v = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    pm = np.ascontiguousarray(perm, dtype=np.int32)
+    N, d = v.shape
+    Nb = (N + TILE - 1) // TILE
+    codes = np.empty((N, d), np.uint8)
+    sfc = np.empty(((N + 15) // 16, d), np.uint8)
+    vscale = np.empty(d, np.float32)
+    vmean = np.empty((Nb, d), np.uint16)
+    err = np.empty(N, np.float32)
+    rep_idx = np.empty(max(R, 1), np.int32)
+    rep_delta = np.empty((max(R, 1), d), np.uint16)
+    lib().orc_quant_v4_head(_p(v), _p(pm), N, d, int(bool(demean)), int(R), _p(codes), _p(sfc), _p(vscale),
+                            _p(vmean), _p(err), _p(rep_idx), _p(rep_delta))
+    return dict(codes=codes, sfc=sfc, vscale=vscale, vmean=vmean, err=err,
+                rep_idx=rep_idx[:R].copy(), rep_delta=rep_delta[:R].copy())
+
+
+def attn_vc4_rows(qk: dict, vq: dict, N: int, rows, softmax_scale: float = DEFAULT_SCALE):
+    """The 4-bit variant's attention for the given query rows of one head.
+
+    Returns (out float64 [len(rows), d], row sums l (2688 x the dequantized
+    probabilities), final frames F)."""
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    d = qk["q8"].shape[1]
+    out = np.empty((rows.size, d), np.float64)
+    out_l = np.empty(rows.size, np.float64)
+    out_F = np.empty(rows.size, np.float32)
+    R = int(vq["rep_idx"].size)
+    ri = vq["rep_idx"] if R else np.zeros(1, np.int32)
+    rd = vq["rep_delta"] if R else np.zeros((1, d), np.uint16)
+    lib().orc_attn_vc4_rows(_p(qk["q8"]), _p(qk["sq"]), _p(qk["k8"]), _p(qk["sk"]),
+                            _p(vq["codes"]), _p(vq["sfc"]), _p(vq["vscale"]), _p(vq["vmean"]),
+                            _p(np.ascontiguousarray(ri)), _p(np.ascontiguousarray(rd)), R,
+                            int(N), d, float(kappa(softmax_scale)), _p(rows), rows.size,
+                            _p(out), _p(out_l), _p(out_F))
+    return out, out_l, out_F
+
+
 # ---------------------------------------------------------------- whole path
 def head_prologue(q_bits, k_bits, v_bits, flags: int = FLAGS_DEFAULT, k: int = 8, iters: int = 3,
                   rho: float = 0.005, perm=None):
@@ -247,7 +324,8 @@ def head_prologue(q_bits, k_bits, v_bits, flags: int = FLAGS_DEFAULT, k: int = 8
     perm = np.ascontiguousarray(perm, dtype=np.int32)
     R = repair_count(rho, N) if (flags & FLAG_REPAIR) else 0
     qk = quant_qk_head(q_bits, k_bits, perm, ksmooth=bool(flags & FLAG_KSMOOTH))
-    vq = quant_v_head(v_bits, perm, demean=bool(flags & FLAG_VSMOOTH), R=R)
+    quant_v = quant_v4_head if (flags & FLAG_VFMT_NVFP4) else quant_v_head
+    vq = quant_v(v_bits, perm, demean=bool(flags & FLAG_VSMOOTH), R=R)
     return dict(perm=perm, cent=cent, labels=labels, qk=qk, vq=vq, R=R)
 
 
@@ -259,7 +337,10 @@ def vc_attention_head(q_bits, k_bits, v_bits, rows=None, flags: int = FLAGS_DEFA
     pro = head_prologue(q_bits, k_bits, v_bits, flags, k, iters, rho, perm)
     if rows is None:
         rows = np.arange(N, dtype=np.int32)
-    out, l, F = attn_vc_rows(pro["qk"], pro["vq"], N, rows, softmax_scale, C)
+    if flags & FLAG_VFMT_NVFP4:
+        out, l, F = attn_vc4_rows(pro["qk"], pro["vq"], N, rows, softmax_scale)
+    else:
+        out, l, F = attn_vc_rows(pro["qk"], pro["vq"], N, rows, softmax_scale, C)
     pro.update(out=out, l=l, F=F, rows=np.asarray(rows, np.int32))
     return pro
 

@@ -1,5 +1,6 @@
 /*
- * vc_oracle.c - plain, slow CPU oracle for VC-Attention FP8.
+ * vc_oracle.c - plain, slow CPU oracle for VC-Attention (the FP8 path and the
+ * NVFP4-residual variant).
  *
  * TEST INFRASTRUCTURE ONLY. Nothing in the library's product path may link,
  * load or call this file; only tests, the smoke check and the bench's CPU
@@ -563,6 +564,289 @@ void orc_attn_exactv_rows(const uint8_t *q8, const float *sq, const uint8_t *k8,
     }
     free(kd);
     free(vx);
+}
+
+/* ------------------------------------------------------------------ */
+/* NVFP4-residual variant ([VCA] "V-Smooth…", item Demean: the residual  */
+/* is quantized per channel in E4M3 for the 8-bit kernel or in NVFP4 for */
+/* the 4-bit one; "ExpCast-FP8…": ExpCast is 8-bit only, so the 4-bit   */
+/* kernel takes the probabilities from an exp2 softmax)                 */
+/* ------------------------------------------------------------------ */
+/* OCP FP4 E2M1: 1 sign, 2 exponent bits (bias 1), 1 mantissa bit, no
+ * infinities or NaN. Exponent field 0 is subnormal (m * 0.5); otherwise the
+ * value is (1 + m/2) * 2^(e-1). The eight magnitudes are 0, 0.5, 1, 1.5, 2,
+ * 3, 4, 6. The code sits in the low 4 bits. */
+double orc_e2m1_value(uint8_t code)
+{
+    int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -v : v;
+}
+
+/* binary32 -> E2M1, round to nearest, ties to even, saturating to +/-6.
+ * The grid spacing is 0.5 below 2 (the subnormal 0.5 and the binade [1, 2)),
+ * 1 in [2, 4) and 2 in [4, 8); a rounded value past 6 saturates. An even
+ * grid index is an even mantissa bit in every binade, so ties to an even
+ * index are ties to even. The sign is kept (a negative value that rounds to
+ * zero gives code 8, negative zero). */
+uint8_t orc_e2m1_encode(float x)
+{
+    uint8_t sign = signbit(x) ? 8 : 0;
+    double a = fabs((double)x), q, val;
+    if (isnan(x))
+        return 7; /* NaN converts to +6 */
+    q = (a < 2.0) ? 0.5 : (a < 4.0) ? 1.0 : 2.0;
+    val = nearbyint(a / q) * q; /* a/q is exact; ties to even */
+    if (val > 6.0)
+        val = 6.0;
+    for (int c = 0; c < 8; ++c)
+        if (orc_e2m1_value((uint8_t)c) == val)
+            return (uint8_t)(sign | c);
+    return (uint8_t)(sign | 7); /* unreachable: val is on the grid */
+}
+
+/* NVFP4 global/ block scale of the probabilities [R]: p <= 1 in the frame of
+ * its tile, so the global decode scale is 1/2688 (2688 = 6 * 448, the E2M1
+ * maximum times the E4M3 maximum) and a block of 16 keys with maximum a gets
+ * the E4M3 scale sf = E4M3(fp32(a * 448)). The element code of p is
+ * E2M1(fp32(p * fp32(2688 / sf))), with every code 0 when sf is 0. The value
+ * the tensor core multiplies is value(code) * sf = 2688 * (dequantized p).
+ *   x_j = fmaf(acc_j, alpha/8, -F/8)      (the exponent, one rounding)
+ *   p_j = binary32(2^x_j)
+ * n <= 16 valid keys; codes[] gets n codes, *sfc the scale code. */
+void orc_nvfp4_p_block(const float *x, int n, uint8_t *codes, uint8_t *sfc)
+{
+    float p[16], a = 0.0f, sfv, rcp;
+    for (int j = 0; j < n; ++j) {
+        p[j] = (float)exp2((double)x[j]);
+        if (p[j] > a)
+            a = p[j];
+    }
+    *sfc = orc_e4m3_encode(a * 448.0f);
+    sfv = (float)orc_e4m3_value(*sfc);
+    rcp = (sfv == 0.0f) ? 0.0f : 2688.0f / sfv;
+    for (int j = 0; j < n; ++j)
+        codes[j] = orc_e2m1_encode(p[j] * rcp);
+}
+
+/* V residual in NVFP4 [R]. Demean and residual as in orc_quant_v_head; then
+ *   g_c   = 2^e_c, the least power of two with amax_c(r) <= 2688 * 2^e_c
+ *           (1 when every residual of the channel is zero), the per-channel
+ *           fp32 global scale
+ *   block = 16 consecutive permuted positions of one channel (the K-major
+ *           scale block of the PV product); positions >= N count as zero
+ *   sf    = E4M3(fp32(fp32(b * 2^-e_c) / 6)), b = max |r| over the block
+ *   code  = E2M1(fp32(r * 2^-e_c) / sf)     (every code 0 when sf is 0)
+ *   deq   = value(code) * sf * g_c          (exact in binary32)
+ *   err   = fp32(r - deq); e_p, the repair list and delta as in the 8-bit path.
+ * Outputs: codes[N][d] (one per byte, low 4 bits), sfc[ceil(N/16)][d],
+ * vscale[d] = g_c, vmean[Nb][d], errsum[N], rep_idx[R], rep_delta[R][d]. */
+void orc_quant_v4_head(const uint16_t *V, const int32_t *perm, int N, int d, int demean, int R,
+                       uint8_t *codes, uint8_t *sfc, float *vscale, uint16_t *vmean, float *errsum,
+                       int32_t *rep_idx, uint16_t *rep_delta)
+{
+    int Nb = (N + TILE - 1) / TILE, N16 = (N + 15) / 16;
+    float *res = (float *)malloc((size_t)N * d * sizeof(float));
+    float *amax = (float *)calloc((size_t)d, sizeof(float));
+    int *expo = (int *)calloc((size_t)d, sizeof(int));
+    for (int t = 0; t < Nb; ++t) {
+        int p0 = t * TILE, cntb = (N - p0 < TILE) ? N - p0 : TILE;
+        for (int c = 0; c < d; ++c) {
+            double s = 0.0;
+            uint16_t mu = 0;
+            float muf;
+            for (int i = 0; i < cntb; ++i)
+                s += (double)orc_bf16_value(V[(size_t)perm[p0 + i] * d + c]);
+            if (demean)
+                mu = orc_bf16_round((float)(s / (double)cntb));
+            vmean[(size_t)t * d + c] = mu;
+            muf = orc_bf16_value(mu);
+            for (int i = 0; i < cntb; ++i) {
+                float r = orc_bf16_value(V[(size_t)perm[p0 + i] * d + c]) - muf;
+                res[(size_t)(p0 + i) * d + c] = r;
+                if (fabsf(r) > amax[c])
+                    amax[c] = fabsf(r);
+            }
+        }
+    }
+    for (int c = 0; c < d; ++c) {
+        int E;
+        float f;
+        if (amax[c] == 0.0f) {
+            expo[c] = 0;
+        } else {
+            f = frexpf(amax[c], &E); /* amax = f 2^E; 2688 = 0.65625 * 2^12 */
+            expo[c] = (f > 0.65625f) ? E - 11 : E - 12;
+        }
+        vscale[c] = ldexpf(1.0f, expo[c]);
+    }
+    for (int jb = 0; jb < N16; ++jb) {
+        int p0 = 16 * jb, n = (N - p0 < 16) ? N - p0 : 16;
+        for (int c = 0; c < d; ++c) {
+            float b = 0.0f, sfv;
+            uint8_t sc;
+            for (int i = 0; i < n; ++i) {
+                float a = fabsf(res[(size_t)(p0 + i) * d + c]);
+                if (a > b)
+                    b = a;
+            }
+            sc = orc_e4m3_encode(ldexpf(b, -expo[c]) / 6.0f);
+            sfc[(size_t)jb * d + c] = sc;
+            sfv = (float)orc_e4m3_value(sc);
+            for (int i = 0; i < n; ++i) {
+                float r = res[(size_t)(p0 + i) * d + c];
+                uint8_t code = (sfv == 0.0f) ? 0 : orc_e2m1_encode(ldexpf(r, -expo[c]) / sfv);
+                codes[(size_t)(p0 + i) * d + c] = code;
+            }
+        }
+    }
+    for (int p = 0; p < N; ++p) {
+        float acc = 0.0f;
+        for (int c = 0; c < d; ++c) {
+            float r = res[(size_t)p * d + c];
+            float sfv = (float)orc_e4m3_value(sfc[(size_t)(p / 16) * d + c]);
+            float deq = (float)(orc_e2m1_value(codes[(size_t)p * d + c]) * (double)sfv * (double)vscale[c]);
+            float err = r - deq;
+            res[(size_t)p * d + c] = err;
+            acc = fmaf(err, err, acc);
+        }
+        errsum[p] = acc;
+    }
+    if (R > 0) {
+        char *taken = (char *)calloc((size_t)N, 1);
+        for (int r = 0; r < R; ++r) {
+            int best = -1;
+            for (int p = 0; p < N; ++p)
+                if (!taken[p] && (best < 0 || errsum[p] > errsum[best]))
+                    best = p;
+            taken[best] = 1;
+        }
+        int w = 0;
+        for (int p = 0; p < N; ++p)
+            if (taken[p])
+                rep_idx[w++] = p;
+        for (int r = 0; r < R; ++r)
+            for (int c = 0; c < d; ++c)
+                rep_delta[(size_t)r * d + c] = orc_bf16_round(res[(size_t)rep_idx[r] * d + c]);
+        free(taken);
+    }
+    free(res);
+    free(amax);
+    free(expo);
+}
+
+/* The 4-bit attention forward of one (b,h) for selected query rows. The
+ * scores, the running max and the frames are those of orc_attn_vc_rows; the
+ * probabilities are 2^((u - F)/8) quantized per 16 keys by orc_nvfp4_p_block,
+ * and the values are the NVFP4 residuals:
+ *   x_ij   = fmaf(acc_ij, alpha_t/8, -F/8),  p_ij = binary32(2^x_ij)
+ *   P_ij   = value(code_ij) * sf_i,kb          (2688 x the dequantized p)
+ *   l_t    = sum_j P_ij
+ *   num   += sum_j P_ij * value(vcode_j) * vsf_j * g + l_t * mu_t
+ * after the last tile, repair adds P'_ij * delta_j for each listed token j,
+ * with P'_ij = bf16(fp32(2^x'_ij * 2688)) and x'_ij the exponent against the
+ * final frame [R]; then O_i = num / l. Inputs: vcodes[N][d], vsfc[ceil(N/16)][d]
+ * and vscale[d] = g_c as orc_quant_v4_head writes them. */
+void orc_attn_vc4_rows(const uint8_t *q8, const float *sq, const uint8_t *k8, const float *sk,
+                       const uint8_t *vcodes, const uint8_t *vsfc, const float *vscale, const uint16_t *vmean,
+                       const int32_t *rep_idx, const uint16_t *rep_delta, int R,
+                       int N, int d, float kappa, const int32_t *rows, int nrows,
+                       double *out, double *out_l, float *out_F)
+{
+    int Nb = (N + TILE - 1) / TILE;
+    double *kd = (double *)malloc((size_t)N * d * sizeof(double));
+    double *vd = (double *)malloc((size_t)N * d * sizeof(double));
+    double *mud = (double *)malloc((size_t)Nb * d * sizeof(double));
+    for (int j = 0; j < N; ++j)
+        for (int c = 0; c < d; ++c) {
+            kd[(size_t)j * d + c] = orc_e4m3_value(k8[(size_t)j * d + c]);
+            vd[(size_t)j * d + c] = orc_e2m1_value(vcodes[(size_t)j * d + c]) *
+                                    orc_e4m3_value(vsfc[(size_t)(j / 16) * d + c]) * (double)vscale[c];
+        }
+    for (int t = 0; t < Nb; ++t)
+        for (int c = 0; c < d; ++c)
+            mud[(size_t)t * d + c] = (double)orc_bf16_value(vmean[(size_t)t * d + c]);
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int ir = 0; ir < nrows; ++ir) {
+        int i = rows[ir];
+        double qd[TILE * 2];
+        double *num = (double *)calloc((size_t)d, sizeof(double));
+        float *acc = (float *)malloc((size_t)TILE * sizeof(float));
+        double l = 0.0;
+        float m = -INFINITY, F = -INFINITY;
+        float sqi = sq[i / TILE];
+        for (int c = 0; c < d; ++c)
+            qd[c] = orc_e4m3_value(q8[(size_t)i * d + c]);
+        for (int t = 0; t < Nb; ++t) {
+            int j0 = t * TILE, j1 = (j0 + TILE < N) ? j0 + TILE : N;
+            float alpha = (sqi * sk[t]) * kappa;
+            float Fnew;
+            double lt = 0.0;
+            for (int j = j0; j < j1; ++j) {
+                double s = 0.0;
+                for (int c = 0; c < d; ++c)
+                    s += qd[c] * kd[(size_t)j * d + c];
+                acc[j - j0] = (float)s;
+                float u = acc[j - j0] * alpha;
+                if (u > m)
+                    m = u;
+            }
+            Fnew = 8.0f * ceilf(m * 0.125f);
+            if (t > 0 && Fnew != F) {
+                double sc = ldexp(1.0, (int)((F - Fnew) / 8.0f));
+                for (int c = 0; c < d; ++c)
+                    num[c] *= sc;
+                l *= sc;
+            }
+            F = Fnew;
+            for (int b0 = j0; b0 < j1; b0 += 16) {
+                int n = (j1 - b0 < 16) ? j1 - b0 : 16;
+                float x[16];
+                uint8_t codes[16], sfc;
+                double sfv;
+                for (int e = 0; e < n; ++e)
+                    x[e] = fmaf(acc[b0 + e - j0], alpha * 0.125f, -F * 0.125f);
+                orc_nvfp4_p_block(x, n, codes, &sfc);
+                sfv = orc_e4m3_value(sfc);
+                for (int e = 0; e < n; ++e) {
+                    double P = orc_e2m1_value(codes[e]) * sfv;
+                    lt += P;
+                    for (int c = 0; c < d; ++c)
+                        num[c] += P * vd[(size_t)(b0 + e) * d + c];
+                }
+            }
+            for (int c = 0; c < d; ++c)
+                num[c] += lt * mud[(size_t)t * d + c];
+            l += lt;
+        }
+        for (int r = 0; r < R; ++r) {
+            int j = rep_idx[r], t = j / TILE;
+            float alpha = (sqi * sk[t]) * kappa;
+            double s = 0.0;
+            for (int c = 0; c < d; ++c)
+                s += qd[c] * kd[(size_t)j * d + c];
+            float x = fmaf((float)s, alpha * 0.125f, -F * 0.125f);
+            float P = orc_bf16_value(orc_bf16_round((float)exp2((double)x) * 2688.0f));
+            for (int c = 0; c < d; ++c)
+                num[c] += (double)P * (double)orc_bf16_value(rep_delta[(size_t)r * d + c]);
+        }
+        for (int c = 0; c < d; ++c)
+            out[(size_t)ir * d + c] = num[c] / l;
+        out_l[ir] = l;
+        out_F[ir] = F;
+        free(num);
+        free(acc);
+    }
+    free(kd);
+    free(vd);
+    free(mud);
+}
+
+void orc_e2m1_encode_n(const float *x, long long n, uint8_t *out)
+{
+    for (long long i = 0; i < n; ++i)
+        out[i] = orc_e2m1_encode(x[i]);
 }
 
 /* Thread control for the bench's CPU baseline (OpenMP over query rows). */

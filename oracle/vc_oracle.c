@@ -636,7 +636,9 @@ void orc_nvfp4_p_block(const float *x, int n, uint8_t *codes, uint8_t *sfc)
  *   block = 16 consecutive permuted positions of one channel (the K-major
  *           scale block of the PV product); positions >= N count as zero
  *   sf    = E4M3(fp32(fp32(b * 2^-e_c) / 6)), b = max |r| over the block
- *   code  = E2M1(fp32(r * 2^-e_c) / sf)     (every code 0 when sf is 0)
+ *   code  = E2M1(fp32(fp32(r * 2^-e_c) * fp32(1 / sf)))
+ *           (the reciprocal of the block scale rounded once, the multiplier
+ *           form of the probability codes too; every code 0 when sf is 0)
  *   deq   = value(code) * sf * g_c          (exact in binary32)
  *   err   = fp32(r - deq); e_p, the repair list and delta as in the 8-bit path.
  * Outputs: codes[N][d] (one per byte, low 4 bits), sfc[ceil(N/16)][d],
@@ -683,7 +685,7 @@ void orc_quant_v4_head(const uint16_t *V, const int32_t *perm, int N, int d, int
     for (int jb = 0; jb < N16; ++jb) {
         int p0 = 16 * jb, n = (N - p0 < 16) ? N - p0 : 16;
         for (int c = 0; c < d; ++c) {
-            float b = 0.0f, sfv;
+            float b = 0.0f, sfv, rcpv;
             uint8_t sc;
             for (int i = 0; i < n; ++i) {
                 float a = fabsf(res[(size_t)(p0 + i) * d + c]);
@@ -693,9 +695,10 @@ void orc_quant_v4_head(const uint16_t *V, const int32_t *perm, int N, int d, int
             sc = orc_e4m3_encode(ldexpf(b, -expo[c]) / 6.0f);
             sfc[(size_t)jb * d + c] = sc;
             sfv = (float)orc_e4m3_value(sc);
+            rcpv = (sfv == 0.0f) ? 0.0f : 1.0f / sfv;
             for (int i = 0; i < n; ++i) {
                 float r = res[(size_t)(p0 + i) * d + c];
-                uint8_t code = (sfv == 0.0f) ? 0 : orc_e2m1_encode(ldexpf(r, -expo[c]) / sfv);
+                uint8_t code = (sfv == 0.0f) ? 0 : orc_e2m1_encode(ldexpf(r, -expo[c]) * rcpv);
                 codes[(size_t)(p0 + i) * d + c] = code;
             }
         }

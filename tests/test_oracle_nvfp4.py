@@ -165,6 +165,30 @@ def test_quant_v4_commutes_with_power_of_two_scaling(orc):
     assert np.array_equal(orc.bf16_value(b["rep_delta"]), orc.bf16_value(a["rep_delta"]) * 4)
 
 
+def test_quant_v4_matches_library_roundings(orc):
+    """Block scales and codes from library conversions (ml_dtypes E4M3 and
+    E2M1, round to nearest even) applied to the same binary32 steps: the
+    scaled block maximum over 6, and the scaled residual times the rounded
+    reciprocal of the block scale."""
+    v, perm = _v_case(42, N=200)
+    vq = orc.quant_v4_head(v, perm, demean=True, R=0)
+    N = v.shape[0]
+    vf = synth.bf16_bits_to_f32(v)[perm]
+    mu = orc.bf16_value(vq["vmean"])[np.arange(N) // 128].astype(np.float32)
+    x = ((vf - mu).astype(np.float32) / vq["vscale"]).astype(np.float32)   # exact: g is a power of two
+    for jb in range((N + 15) // 16):
+        xb = x[16 * jb:16 * jb + 16]
+        b = np.abs(xb).max(0).astype(np.float32)
+        sf = (b / np.float32(6.0)).astype(np.float32).astype(E4M3_LIB)
+        assert np.array_equal(sf.view(np.uint8), vq["sfc"][jb])
+        sfv = sf.astype(np.float32)
+        with np.errstate(divide="ignore"):
+            rcp = np.where(sfv == 0, np.float32(0), (np.float32(1.0) / sfv).astype(np.float32)).astype(np.float32)
+        want = (xb * rcp).astype(np.float32).astype(E2M1_LIB).view(np.uint8)
+        want = np.where(sfv == 0, 0, want)
+        assert np.array_equal(vq["codes"][16 * jb:16 * jb + 16], want), jb
+
+
 # ---------------------------------------------------------------- lossless case
 def _lossless_case(seed, N=300, d=128):
     """Scores on multiples of 8 byte units (kappa = 1), so every probability

@@ -170,7 +170,7 @@ def test_quant_v4_matches_library_roundings(orc):
     E2M1, round to nearest even) applied to the same binary32 steps: the
     scaled block maximum over 6, and the scaled residual times the rounded
     reciprocal of the block scale."""
-    v, perm = _v_case(42, N=200)
+    v, perm = _v_case(42, N=260)
     vq = orc.quant_v4_head(v, perm, demean=True, R=0)
     N = v.shape[0]
     vf = synth.bf16_bits_to_f32(v)[perm]

@@ -6,6 +6,7 @@
 #include <mutex>
 
 #include "attn_bf16.cuh"
+#include "attn_fp4.cuh"
 #include "attn_fp8.cuh"
 #include "common.cuh"
 #include "prologue.cuh"
@@ -148,6 +149,10 @@ vc_status check_device() {
                                KMEANS_SMEM_FIXED + 64 * D * 12) != cudaSuccess ||
           cudaFuncSetAttribute(k_quantv_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, QUANTV2_SMEM) !=
               cudaSuccess ||
+          cudaFuncSetAttribute(k_quantv4_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, QUANTV2_SMEM) !=
+              cudaSuccess ||
+          cudaFuncSetAttribute(k_vc_attn_fwd4, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(attn_fp4_smem_bytes())) != cudaSuccess ||
           cudaFuncSetAttribute(k_kmeans_pass8, cudaFuncAttributeMaxDynamicSharedMemorySize, KMEANS8_SMEM) !=
               cudaSuccess) {
         ok_cache[dev] = 0;
@@ -164,7 +169,7 @@ vc_status check_params(const vc_params *p) {
   if (!(p->rho >= 0.0f && p->rho < 1.0f)) return VC_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.0f) || !std::isfinite(p->softmax_scale)) return VC_ERR_INVALID_ARG;
   if (p->expcast_bias < 8 || p->expcast_bias > 126) return VC_ERR_INVALID_ARG;
-  if (p->flags & ~(VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH | VC_WARMSTART)) return VC_ERR_INVALID_ARG;
+  if (p->flags & ~(VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH | VC_WARMSTART | VC_VFMT_NVFP4)) return VC_ERR_INVALID_ARG;
   return VC_OK;
 }
 
@@ -263,13 +268,20 @@ void launch_quant_qk(const Shape &sh, const Ws &w, const uint16_t *Q, const uint
 void launch_quant_v(const Shape &sh, const Ws &w, const uint16_t *V, const int32_t *perm, uint8_t *v8t,
                     float *vscale, uint16_t *vmean, int32_t *rep_idx, uint16_t *rep_delta, cudaStream_t s) {
   const int demean = (sh.flags & VC_VSMOOTH) ? 1 : 0;
+  const int fp4 = (sh.flags & VC_VFMT_NVFP4) ? 1 : 0;
   int *vexpo = w.at<int>(w.L.vexpo);
-  k_quantv_pass1<<<dim3(sh.Nb, sh.BH), 256, QUANTV1_SMEM, s>>>(V, perm, sh.N, sh.Nb, demean, vmean,
+  k_quantv_pass1<<<dim3(sh.Nb, sh.BH), 256, QUANTV1_SMEM, s>>>(V, perm, sh.N, sh.Nb, demean, fp4, vmean,
                                                      w.at<float>(w.L.amax_part), vscale, vexpo,
                                                      w.at<unsigned>(w.L.vq_counter));
   count_launch();
-  k_quantv_pass2<<<dim3(sh.Nb, sh.BH), 256, QUANTV2_SMEM, s>>>(V, perm, sh.N, sh.Nb, sh.Npad, sh.nch32, vmean, vscale, vexpo,
-                                                     v8t, w.at<float>(w.L.err), w.at<uint16_t>(w.L.mut2));
+  if (fp4)
+    k_quantv4_pass2<<<dim3(sh.Nb, sh.BH), 256, QUANTV2_SMEM, s>>>(V, perm, sh.N, sh.Nb, sh.nch32, vmean, vscale,
+                                                                  vexpo, v8t, w.at<float>(w.L.err),
+                                                                  w.at<uint16_t>(w.L.mut2));
+  else
+    k_quantv_pass2<<<dim3(sh.Nb, sh.BH), 256, QUANTV2_SMEM, s>>>(V, perm, sh.N, sh.Nb, sh.Npad, sh.nch32, vmean,
+                                                                 vscale, vexpo, v8t, w.at<float>(w.L.err),
+                                                                 w.at<uint16_t>(w.L.mut2));
   count_launch();
   if (sh.R > 0) {
     if (sh.N <= 512 * 64)
@@ -277,9 +289,14 @@ void launch_quant_v(const Shape &sh, const Ws &w, const uint16_t *V, const int32
     else
       k_repair_select<<<sh.BH, 1024, 0, s>>>(w.at<float>(w.L.err), sh.N, sh.R, rep_idx);
     count_launch();
-    k_repair_delta<<<dim3((sh.Rpad + 7) / 8, sh.BH), 256, 0, s>>>(V, perm, sh.N, sh.Nb, sh.R, sh.Rpad, rep_idx,
-                                                                  vmean, vscale, vexpo, rep_delta,
-                                                                  w.at<uint16_t>(w.L.deltat));
+    if (fp4)
+      k_repair_delta4<<<dim3((sh.Rpad + 7) / 8, sh.BH), 256, 0, s>>>(V, perm, sh.N, sh.Nb, sh.R, sh.Rpad, rep_idx,
+                                                                     vmean, vscale, vexpo, v8t, rep_delta,
+                                                                     w.at<uint16_t>(w.L.deltat));
+    else
+      k_repair_delta<<<dim3((sh.Rpad + 7) / 8, sh.BH), 256, 0, s>>>(V, perm, sh.N, sh.Nb, sh.R, sh.Rpad, rep_idx,
+                                                                    vmean, vscale, vexpo, rep_delta,
+                                                                    w.at<uint16_t>(w.L.deltat));
     count_launch();
   }
 }
@@ -413,11 +430,13 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
   launch_quant_v(sh, w, Vh, pm, v8t, vscale, w.at<uint16_t>(w.L.vmean), rep_idx, w.at<uint16_t>(w.L.rep_delta), s);
   prof_mark(3, s);
 
+  const bool fp4 = (sh.flags & VC_VFMT_NVFP4) != 0;
   CUtensorMap tq, tk, tv, tmu, tdt;
   const uint64_t rows = static_cast<uint64_t>(sh.BH) * sh.Npad;
   bool ok = map2d(&tq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, rows, 128, 128) &&
             map2d(&tk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, rows, 128, 128) &&
-            map2d(&tv, v8t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, sh.Npad, static_cast<uint64_t>(sh.BH) * 128, 128, 128) &&
+            (fp4 || map2d(&tv, v8t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, sh.Npad, static_cast<uint64_t>(sh.BH) * 128,
+                          128, 128)) &&
             map2d(&tmu, w.at<uint16_t>(w.L.mut2), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64,
                   static_cast<uint64_t>(sh.BH) * sh.nch32 * 128, 64, 128);
   if (ok) {
@@ -428,6 +447,29 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
       tdt = tmu;  // unused when R == 0
   }
   if (!ok) return VC_ERR_CUDA;
+  if (fp4) {
+    AttnFp4Params ap{};
+    ap.N = sh.N;
+    ap.Nb = sh.Nb;
+    ap.Npad = sh.Npad;
+    ap.nch32 = sh.nch32;
+    ap.R = sh.R;
+    ap.Rpad = sh.Rpad;
+    ap.kappa = kappa_of(scale_or_default(p->softmax_scale));
+    ap.sq = sq;
+    ap.sk = sk;
+    ap.vscale = vscale;
+    ap.v4img = v8t;
+    ap.rep_idx = rep_idx;
+    ap.k8 = k8;
+    ap.O = static_cast<uint16_t *>(O);
+    ap.status = w.at<uint32_t>(w.L.status);
+    k_vc_attn_fwd4<<<dim3(sh.Nb, sh.BH), 352, attn_fp4_smem_bytes(), s>>>(tq, tk, tmu, tdt, ap);
+    count_launch();
+    prof_mark(4, s);
+    if (g_prof.on) ++g_prof.calls;
+    return last_error();
+  }
   AttnFp8Params ap{};
   ap.N = sh.N;
   ap.Nb = sh.Nb;

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -60,6 +61,31 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 __device__ __forceinline__ float2 e4m3x2_value(uint16_t codes) {
   __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes), __NV_E4M3);
   return __half22float2(*reinterpret_cast<__half2 *>(&h));
+}
+// Two floats -> two E2M1 (FP4) codes, round to nearest even, saturating to
+// +/-6; lo in the low nibble.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp4x2(make_float2(lo, hi), __NV_E2M1, cudaRoundNearest));
+}
+// Exact value of two E2M1 codes (low nibble, high nibble).
+__device__ __forceinline__ float2 e2m1x2_value(uint32_t codes) {
+  __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(codes & 0xFFu), __NV_E2M1);
+  return __half22float2(*reinterpret_cast<__half2 *>(&h));
+}
+
+// NVFP4 tile image of the values (one per 128-token tile of a head): the
+// E4M3 block scales, 1024 bytes, byte 512*(jb/4) + 16*(c%32) + 4*(c/32) +
+// jb%4 for channel c and 16-token block jb; then the E2M1 codes, 8192 bytes,
+// channel rows of 64 bytes (token 2i in the low nibble of byte i) stored with
+// the 64-byte swizzle: 8-row groups of 512 bytes, 16-byte chunk index XOR
+// ((row / 2) mod 4).
+constexpr int V4_SF_BYTES = 1024;
+constexpr int V4_TILE_BYTES = V4_SF_BYTES + 128 * 64;
+__host__ __device__ constexpr uint32_t sw64_off(int r, int ch) {
+  return static_cast<uint32_t>((r >> 3) * 512 + (r & 7) * 64 + ((ch ^ ((r >> 1) & 3)) << 4));
+}
+__host__ __device__ constexpr uint32_t v4_sf_off(int c, int jb) {
+  return static_cast<uint32_t>(512 * (jb >> 2) + 16 * (c & 31) + 4 * (c >> 5) + (jb & 3));
 }
 
 }  // namespace vc

@@ -554,9 +554,10 @@ __device__ __forceinline__ float sv_at(const uint8_t *sv, int r, int c) {
 
 // Pass 1: block means (fp64 sums over the block's tokens) and per-block
 // residual amax; the last block of a (b,h) turns the channel amax into the
-// power-of-two scale. Thread (h, c): channel c over rows [64h, 64h+64).
+// power-of-two scale (the least with amax <= 448 * scale for E4M3 residuals,
+// amax <= 2688 * scale, the NVFP4 global scale, for 4-bit ones). Thread (h, c): channel c over rows [64h, 64h+64).
 __global__ void __launch_bounds__(256) k_quantv_pass1(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
-                                                      int N, int Nb, int demean, uint16_t *__restrict__ vmean,
+                                                      int N, int Nb, int demean, int fp4, uint16_t *__restrict__ vmean,
                                                       float *__restrict__ amax_part, float *__restrict__ vscale,
                                                       int *__restrict__ vexpo, unsigned *__restrict__ counter) {
   extern __shared__ __align__(16) uint8_t dsm[];
@@ -601,8 +602,11 @@ __global__ void __launch_bounds__(256) k_quantv_pass1(const uint16_t *__restrict
   float sc = 1.0f;
   if (a > 0.0f) {
     int E;
-    const float f = frexpf(a, &E);  // a = f * 2^E, f in [0.5, 1); 448 = 0.875 * 2^9
-    e = (f > 0.875f) ? E - 8 : E - 9;
+    const float f = frexpf(a, &E);  // a = f * 2^E, f in [0.5, 1)
+    if (fp4)
+      e = (f > 0.65625f) ? E - 11 : E - 12;  // NVFP4: a <= 2688 * 2^e, 2688 = 6 * 448 = 0.65625 * 2^12
+    else
+      e = (f > 0.875f) ? E - 8 : E - 9;      // E4M3: a <= 448 * 2^e, 448 = 0.875 * 2^9
     sc = ldexpf(1.0f, e);
   }
   vscale[static_cast<size_t>(bh) * D + c] = sc;
@@ -685,6 +689,121 @@ __global__ void __launch_bounds__(256) k_quantv_pass2(const uint16_t *__restrict
     for (int i = 0; i < 4; ++i)
       *reinterpret_cast<uint4 *>(dst + 16 * i) = *reinterpret_cast<const uint4 *>(srcT + 16 * i);
   }
+}
+
+// NVFP4 pass 2 (page "VC-Attention acelera atenção…", "V-Smooth: corrigindo
+// outliers de valor", item Demean, the 4-bit residual): per 16-token block and
+// channel the E4M3 scale sf = E4M3(fp32(b * 2^-e) / 6) of the block maximum
+// b = max |r|; codes E2M1(fp32(r * 2^-e) * fp32(1/sf)); the per-token error
+// of value(code) * sf * 2^e, fmaf-accumulated in channel order; the tile image
+// (scales, then the swizzled channel rows of codes) and the block means / g
+// for the restore, as in pass 2.
+__global__ void __launch_bounds__(256) k_quantv4_pass2(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
+                                                       int N, int Nb, int nch32, const uint16_t *__restrict__ vmean,
+                                                       const float *__restrict__ vscale, const int *__restrict__ vexpo,
+                                                       uint8_t *__restrict__ v4img, float *__restrict__ err,
+                                                       uint16_t *__restrict__ mut2) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  uint8_t *sv = dsm;                           // 128 rows x 272 bytes
+  uint8_t *codeT = dsm + TILE * VQ_ROW_BYTES;  // 128 channels x 144 bytes, one code per byte
+  __shared__ __align__(16) float smu[D], smult[D], sscale[D];
+  __shared__ float srcp[8][D], ssfv[8][D];
+  __shared__ __align__(16) uint8_t ssf[V4_SF_BYTES];
+  const int t = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int p0 = t * TILE, cnt = min(TILE, N - p0);
+  gather_tile(sv, V + static_cast<size_t>(bh) * N * D, perm ? perm + static_cast<size_t>(bh) * N : nullptr, p0, cnt);
+  if (tid < 128) {
+    const int c = tid;
+    const uint16_t mu = vmean[(static_cast<size_t>(bh) * Nb + t) * D + c];
+    smu[c] = bf16_to_f32(mu);
+    const int e = vexpo[static_cast<size_t>(bh) * D + c];
+    smult[c] = ldexpf(1.0f, -e);
+    sscale[c] = vscale[static_cast<size_t>(bh) * D + c];
+    const uint16_t ms = f32_to_bf16_rn(__fmul_rn(bf16_to_f32(mu), ldexpf(1.0f, -e)));
+    const int ch = t / CHUNK32, slot = t % CHUNK32;
+    uint16_t *m = mut2 + ((static_cast<size_t>(bh) * nch32 + ch) * D + c) * 64;
+    m[slot] = ms;
+    m[slot + 32] = ms;
+    if (t == Nb - 1)
+      for (int s2 = slot + 1; s2 < CHUNK32; ++s2) {
+        m[s2] = 0;
+        m[s2 + 32] = 0;
+      }
+  }
+  __syncthreads();
+  {
+    // block scales: thread (c, jb = tid/128 + 2i)
+    const int c = tid & 127;
+    for (int jb = tid >> 7; jb < 8; jb += 2) {
+      float b = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = 16 * jb + i;
+        if (r < cnt) b = fmaxf(b, fabsf(__fsub_rn(sv_at(sv, r, c), smu[c])));
+      }
+      const uint32_t sc = e4m3x2(__fdiv_rn(__fmul_rn(b, smult[c]), 6.0f), 0.0f) & 0xFFu;
+      const float sfv = e4m3x2_value(static_cast<uint16_t>(sc)).x;
+      ssfv[jb][c] = sfv;
+      srcp[jb][c] = sfv == 0.0f ? 0.0f : __frcp_rn(sfv);
+      ssf[v4_sf_off(c, jb)] = static_cast<uint8_t>(sc);
+    }
+  }
+  __syncthreads();
+  if (tid < 128) {
+    const int r = tid, jb = r >> 4;
+    float acc = 0.0f;
+    const uint8_t *row = sv + r * VQ_ROW_BYTES;
+#pragma unroll 2
+    for (int c0 = 0; c0 < D; c0 += 8) {
+      float x[8];
+      bf16x8(*reinterpret_cast<const uint4 *>(row + 2 * c0), x);
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) {
+        const int c = c0 + j;
+        uint32_t codes = 0;
+        if (r < cnt) {
+          const float r0 = __fsub_rn(x[j], smu[c]);
+          const float r1 = __fsub_rn(x[j + 1], smu[c + 1]);
+          codes = e2m1x2(__fmul_rn(__fmul_rn(r0, smult[c]), srcp[jb][c]),
+                         __fmul_rn(__fmul_rn(r1, smult[c + 1]), srcp[jb][c + 1]));
+          const float2 dq = e2m1x2_value(codes);
+          const float e0 = __fsub_rn(r0, __fmul_rn(__fmul_rn(dq.x, ssfv[jb][c]), sscale[c]));
+          const float e1 = __fsub_rn(r1, __fmul_rn(__fmul_rn(dq.y, ssfv[jb][c + 1]), sscale[c + 1]));
+          acc = __fmaf_rn(e0, e0, acc);
+          acc = __fmaf_rn(e1, e1, acc);
+        }
+        codeT[c * 144 + r] = static_cast<uint8_t>(codes & 15u);
+        codeT[(c + 1) * 144 + r] = static_cast<uint8_t>(codes >> 4);
+      }
+    }
+    if (r < cnt) err[static_cast<size_t>(bh) * N + p0 + r] = acc;
+  }
+  __syncthreads();
+  uint8_t *img = v4img + (static_cast<size_t>(bh) * Nb + t) * V4_TILE_BYTES;
+  {
+    // thread (c, h): the 16-byte chunks 2h and 2h+1 of channel row c (tokens 64h .. 64h+63)
+    const int c = tid >> 1, h = tid & 1;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int ch = 2 * h + k;
+      const uint8_t *src = codeT + c * 144 + 32 * ch;
+      uint32_t w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint2 b8 = *reinterpret_cast<const uint2 *>(src + 8 * q);
+        uint32_t v = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v |= ((b8.x >> (8 * e)) & 15u) << (4 * e);
+          v |= ((b8.y >> (8 * e)) & 15u) << (4 * e + 16);
+        }
+        w[q] = v;
+      }
+      *reinterpret_cast<uint4 *>(img + V4_SF_BYTES + sw64_off(c, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  if (tid < V4_SF_BYTES / 16)
+    *reinterpret_cast<uint4 *>(img + 16 * tid) = *reinterpret_cast<const uint4 *>(ssf + 16 * tid);
 }
 
 // ============================================================== repair selection
@@ -906,6 +1025,56 @@ __global__ void __launch_bounds__(256) k_repair_delta(const uint16_t *__restrict
     const float2 dq = e4m3x2_value(codes);
     dl[i] = f32_to_bf16_rn(__fsub_rn(res[i], __fmul_rn(dq.x, sc[i])));
     dl[i + 1] = f32_to_bf16_rn(__fsub_rn(res[i + 1], __fmul_rn(dq.y, sc[i + 1])));
+  }
+  uint2 o;
+  o.x = static_cast<uint32_t>(dl[0]) | (static_cast<uint32_t>(dl[1]) << 16);
+  o.y = static_cast<uint32_t>(dl[2]) | (static_cast<uint32_t>(dl[3]) << 16);
+  *reinterpret_cast<uint2 *>(rep_delta + (static_cast<size_t>(bh) * R + r) * D + 4 * lane) = o;
+  for (int i = 0; i < 4; ++i) {
+    const int c = 4 * lane + i;
+    deltat[(static_cast<size_t>(bh) * D + c) * Rpad + r] = f32_to_bf16_rn(__fmul_rn(bf16_to_f32(dl[i]), mult[i]));
+  }
+}
+
+// The repair deltas of the NVFP4 residual: the token's codes are recomputed
+// from its block's scale code in the tile image, exactly as pass 2 made them.
+__global__ void __launch_bounds__(256) k_repair_delta4(const uint16_t *__restrict__ V,
+                                                       const int32_t *__restrict__ perm, int N, int Nb, int R, int Rpad,
+                                                       const int32_t *__restrict__ rep_idx,
+                                                       const uint16_t *__restrict__ vmean,
+                                                       const float *__restrict__ vscale, const int *__restrict__ vexpo,
+                                                       const uint8_t *__restrict__ v4img,
+                                                       uint16_t *__restrict__ rep_delta, uint16_t *__restrict__ deltat) {
+  const int bh = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + warp;
+  if (r >= Rpad) return;
+  if (r >= R) {
+    for (int i = 0; i < 4; ++i) deltat[(static_cast<size_t>(bh) * D + 4 * lane + i) * Rpad + r] = 0;
+    return;
+  }
+  const int p = rep_idx[static_cast<size_t>(bh) * R + r];
+  const int row = perm ? perm[static_cast<size_t>(bh) * N + p] : p;
+  const int t = p / TILE, jb = (p % TILE) >> 4;
+  const uint8_t *sfimg = v4img + (static_cast<size_t>(bh) * Nb + t) * V4_TILE_BYTES;
+  const uint2 w = *reinterpret_cast<const uint2 *>(V + (static_cast<size_t>(bh) * N + row) * D + 4 * lane);
+  const float v[4] = {__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u), __uint_as_float(w.y << 16),
+                      __uint_as_float(w.y & 0xFFFF0000u)};
+  float res[4], mult[4], sc[4], sfv[4], rcp[4];
+  for (int i = 0; i < 4; ++i) {
+    const int c = 4 * lane + i;
+    res[i] = __fsub_rn(v[i], bf16_to_f32(vmean[(static_cast<size_t>(bh) * Nb + t) * D + c]));
+    mult[i] = ldexpf(1.0f, -vexpo[static_cast<size_t>(bh) * D + c]);
+    sc[i] = vscale[static_cast<size_t>(bh) * D + c];
+    sfv[i] = e4m3x2_value(static_cast<uint16_t>(sfimg[v4_sf_off(c, jb)])).x;
+    rcp[i] = sfv[i] == 0.0f ? 0.0f : __frcp_rn(sfv[i]);
+  }
+  uint16_t dl[4];
+  for (int i = 0; i < 4; i += 2) {
+    const uint32_t codes = e2m1x2(__fmul_rn(__fmul_rn(res[i], mult[i]), rcp[i]),
+                                  __fmul_rn(__fmul_rn(res[i + 1], mult[i + 1]), rcp[i + 1]));
+    const float2 dq = e2m1x2_value(codes);
+    dl[i] = f32_to_bf16_rn(__fsub_rn(res[i], __fmul_rn(__fmul_rn(dq.x, sfv[i]), sc[i])));
+    dl[i + 1] = f32_to_bf16_rn(__fsub_rn(res[i + 1], __fmul_rn(__fmul_rn(dq.y, sfv[i + 1]), sc[i + 1])));
   }
   uint2 o;
   o.x = static_cast<uint32_t>(dl[0]) | (static_cast<uint32_t>(dl[1]) << 16);

@@ -190,6 +190,59 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
                : "memory");
 }
 
+// ---------------------------------------------------------------- FP4 block-scaled MMA
+// Descriptor of a K-major tile stored with the 64-byte swizzle (64-byte rows,
+// 8-row groups of 512 bytes: layout type 4, stride 512).
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= 1ull << 16;  // leading-dimension offset (unused by the swizzled K-major layouts)
+  d |= static_cast<uint64_t>(512 >> 4) << 32;
+  d |= 1ull << 46;
+  d |= 4ull << 61;
+  return d;
+}
+// Descriptor of 32 rows x 16 bytes without swizzle (8-row core matrices 128
+// bytes apart): the source of a 32x128b scale-factor copy.
+__device__ __forceinline__ uint64_t sdesc_sf(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= 1ull << 46;
+  return d;
+}
+// Instruction descriptor of kind::mxf4nvf4 with 16-element E4M3 scales: A and
+// B E2M1 (format 1, bits [7,10) and [10,13)), K-major, scale format E4M3 (bit
+// 23 = 0), scale-factor byte ids 0, dense K = 64.
+__host__ __device__ constexpr uint32_t idesc_fp4_make(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(N) >> 3) << 17) | ((static_cast<uint32_t>(M) >> 4) << 24);
+}
+// D (+)= (A x SFA) (B x SFB)^T over K = 64; the scale factors are read from
+// TMEM (row m of an operand: lane m mod 32, column m / 32, byte = 16-element
+// block within the K step).
+__device__ __forceinline__ void mma_fp4_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+// Copy 32 rows x 16 bytes of shared memory into TMEM columns [taddr, taddr+4)
+// of lanes 0..31, replicated into the four 32-lane sub-partitions.
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from
+// global to shared memory, completing on an mbarrier transaction count.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // Offset of 16-byte chunk `ch` of row `r` in a K-major tile stored with the
 // 128-byte swizzle: 8-row groups of 1024 bytes, chunk index XOR (row mod 8).
 __device__ __forceinline__ uint32_t sw128_off(int r, int ch) {

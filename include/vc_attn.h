@@ -56,6 +56,14 @@ typedef enum {
  * from the centroids passed in (the previous denoising step's) instead of the
  * tokens V[floor(j*N/k)]. Ignored by vc_attn_fwd, which clusters from scratch. */
 #define VC_WARMSTART 16u
+/* The NVFP4-residual variant ([VCA] "V-Smooth…", item Demean: the residual in
+ * NVFP4 for the 4-bit kernel; "ExpCast-FP8…": ExpCast is 8-bit only). The V
+ * residual is stored as E2M1 codes with an E4M3 scale per 16 consecutive
+ * permuted tokens of a channel and a per-channel power-of-two global scale;
+ * the probabilities come from an exp2 softmax, quantized to NVFP4 per 16 keys;
+ * PV runs on the block-scaled FP4 tensor cores. QK^T stays FP8; the expcast
+ * bias is not used. vc_attn_quant_v and vc_attn_fwd honour it. */
+#define VC_VFMT_NVFP4 32u
 
 typedef struct {
   int k;             /* k-means clusters, 1..64 (default 8) */
@@ -63,7 +71,8 @@ typedef struct {
   float rho;         /* repair budget, [0, 1) (default 0.005); R = ceil(rho*N) */
   float softmax_scale; /* 0 => 1/sqrt(d) */
   int expcast_bias;  /* C: the running row maximum maps to byte C, 8..126 (default 120) */
-  unsigned flags;    /* VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH (default), optionally VC_WARMSTART */
+  unsigned flags;    /* VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH (default), optionally VC_WARMSTART,
+                        VC_VFMT_NVFP4 */
 } vc_params;
 
 /* Fill the defaults listed above. */
@@ -159,6 +168,20 @@ vc_status vc_attn_quant_qk(const void *Q, const void *K, const int32_t *perm, in
  * mean = bf16(fp32(fp64 sum / count)); r = v - mean; code = E4M3(r * 2^-e);
  * token error = sum_c (r - value(code)*scale)^2 (fp32, fma in channel order);
  * the R largest errors are repaired (ties to the lowest position).
+ * With VC_VFMT_NVFP4 the residual is NVFP4 instead:
+ *   v8          holds B*H*Nb tile images of 9216 bytes (the buffer size is
+ *               the same B*H*d*Npad bytes; the images fill the first 9/16):
+ *               bytes [0,1024) the E4M3 block scales, byte 512*(j/4) +
+ *               16*(c%32) + 4*(c/32) + j%4 for channel c and 16-token block
+ *               j of the tile; bytes [1024,9216) the E2M1 codes, channel row c
+ *               of 64 bytes (token 2i in the low nibble of byte i) with byte i
+ *               of row c at 1024 + 512*(c/8) + 64*(c%8) + 16*((i/16) XOR
+ *               ((c/2)%4)) + i%16 (the 64-byte swizzle of the tensor cores)
+ *   v_scale     per-channel global scale g = 2^e, the least with
+ *               max_p |r| <= 2688 * 2^e (2688 = 6 * 448)
+ *   sf = E4M3(fp32(b * 2^-e) / 6) for the block maximum b = max |r|;
+ *   code = E2M1(fp32(r * 2^-e) * fp32(1/sf)) (0 when sf is 0); token error
+ *   and repair as above with value(code) * sf * g.
  */
 vc_status vc_attn_quant_v(const void *V, const int32_t *perm, int B, int H, int N, int d, const vc_params *p,
                           uint8_t *v8, float *v_scale, void *v_mean, int32_t *rep_idx, void *rep_delta,
@@ -181,6 +204,11 @@ vc_status vc_attn_quant_v(const void *V, const int32_t *perm, int B, int H, int 
  * and the block mean is restored as l_t * mean_t ([VCA] "V-Smooth…", item
  * Restore) on the tensor cores in bf16; repair adds p * delta for the listed
  * tokens; O = scale_c * acc / l.
+ * With VC_VFMT_NVFP4 (the 4-bit variant): the same frames, then per 16 keys
+ * x = fma(acc, alpha/8, -F/8), p = 2^x, block scale sf = E4M3(448 * max p),
+ * codes E2M1(p * fl(2688/sf)); O += P V4 on the block-scaled FP4 tensor cores
+ * (kind::mxf4nvf4) with the row sums from the same product; repair uses
+ * bf16(2^x' * 2688) with x' against the final frame.
  */
 vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
                       const int32_t *perm, const vc_params *p, void *O, void *ws, size_t ws_bytes, void *stream);

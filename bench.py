@@ -11,6 +11,13 @@ attention kernel. Metric: TFLOPS = 4*B*H*N^2*d / t (the pages' attention FLOP
 count), also as % of the measured FP8 dense peak.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME] [--vfmt e4m3|nvfp4]
+
+The default line also carries "variants": the 720p video workload (B=1, H=40,
+N=75600) on the 8-bit path and on the NVFP4-residual variant (VC_VFMT_NVFP4),
+the latter with its roofline against the exp2 throughput of the special-
+function units (the variant has no ExpCast, so one 2^x per score bounds it).
+--vfmt nvfp4 [--workload NAME] times the variant as the main line instead.
 
 N > 1 runs under torchrun: every rank owns one independent copy of the
 workload (heads are independent problems; no data-path collective), the step
@@ -36,6 +43,9 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = "image2048_b1h24n16544"
 METRIC = "vc_attn_fwd TFLOPS (4N²dH/t) at N=16544,H=24,d=128; % of B200 FP8 peak"
+VARIANT_WORKLOAD = "video720p_b1h40n75600"  # the workload the NVFP4-residual variant is timed on
+SMS = 148
+EX2_PER_CLK_SM = 16  # special-function unit: 2^x results per clock per SM (CUDA throughput table, cc 10.0)
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -65,24 +75,34 @@ class ClockSampler:
         self._t = None
 
     def start(self):
+        """Spawn the sampler and wait for its first sample, so that sampling is
+        live when the timed region begins (right after this returns)."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
             return
         self._t = threading.Thread(target=self._read, daemon=True)
         self._t.start()
+        t0 = time.monotonic()
+        while not self.lines and time.monotonic() - t0 < 5.0 and self.proc.poll() is None:
+            time.sleep(0.005)
+        self.t_begin = time.monotonic()
 
     def _read(self):
         for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
+            self.lines.append((time.monotonic(), ln.strip()))
 
     def stop(self) -> dict:
+        """Samples that arrived during the timed region (start() return to this
+        call); if the region was shorter than the sampling interval, the three
+        samples nearest to it, marked as such."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
+        t_end = time.monotonic()
+        time.sleep(0.05)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -90,26 +110,33 @@ class ClockSampler:
             self.proc.kill()
         if self._t:
             self._t.join(timeout=2)
-        sm, smax, power, reasons = [], [], [], set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ts, ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-                power.append(float(parts[3]))
+                rows.append((ts, float(parts[1]), float(parts[2]), float(parts[3]),
+                             [nm for nm, val in zip(names, parts[5:9]) if val.lower() == "active"]))
             except ValueError:
                 continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        load = [s for s, p in zip(sm, power) if p > 200] or sm
-        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(smax), "samples": len(sm),
-                "power_w_max": max(power), "reasons": sorted(reasons)}
+        t_begin = getattr(self, "t_begin", rows[0][0])
+        inside = [r for r in rows if t_begin <= r[0] <= t_end]
+        window = "timed region"
+        if not inside:
+            mid = 0.5 * (t_begin + t_end)
+            inside = sorted(rows, key=lambda r: abs(r[0] - mid))[:3]
+            window = "nearest 3 samples (timed region shorter than the 20 ms interval)"
+        sm = [r[1] for r in inside]
+        power = [r[3] for r in inside]
+        load = [x for x, pw in zip(sm, power) if pw > 200] or sm
+        reasons = sorted(set(nm for r in inside for nm in r[4]))
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(r[2] for r in inside), "samples": len(inside),
+                "window": window, "region_ms": round(1e3 * (t_end - t_begin), 1),
+                "power_w_max": max(power), "reasons": reasons}
 
 
 E2E_HEADS_PER_RUN = 2  # heads per run of the end-to-end call (copies overlap compute)
@@ -145,7 +172,7 @@ def _to_dev(torch, bits):
 
 
 # ---------------------------------------------------------------- CPU oracle timing
-def cpu_oracle_sample(wl, x, rows_per_head: int = 96, heads=(0,)):
+def cpu_oracle_sample(wl, x, rows_per_head: int = 96, heads=(0,), nvfp4: bool = False):
     """Time the oracle on a bounded sample and extrapolate to the workload.
 
     For each sampled head: the full per-head prologue (k-means, quantization,
@@ -159,10 +186,14 @@ def cpu_oracle_sample(wl, x, rows_per_head: int = 96, heads=(0,)):
     for h in heads:
         q, k, v = x["q"][0, h], x["k"][0, h], x["v"][0, h]
         t0 = time.perf_counter()
-        pro = oracle.head_prologue(q, k, v)
+        flags = oracle.FLAGS_DEFAULT | (oracle.FLAG_VFMT_NVFP4 if nvfp4 else 0)
+        pro = oracle.head_prologue(q, k, v, flags=flags)
         t1 = time.perf_counter()
         rows = np.linspace(0, wl.N - 1, rows_per_head).astype(np.int32)
-        oracle.attn_vc_rows(pro["qk"], pro["vq"], wl.N, rows)
+        if nvfp4:
+            oracle.attn_vc4_rows(pro["qk"], pro["vq"], wl.N, rows)
+        else:
+            oracle.attn_vc_rows(pro["qk"], pro["vq"], wl.N, rows)
         t2 = time.perf_counter()
         t_pro += t1 - t0
         t_rows += t2 - t1
@@ -204,6 +235,68 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- GPU bench
+def exp2_roofline(B, H, N, attn_ms, sm_mhz):
+    """The NVFP4 variant has no ExpCast: every score goes through one 2^x on the
+    special-function unit, the kernel's bound (N^2 B H per launch)."""
+    if not attn_ms or not sm_mhz:
+        return None
+    achieved = B * H * float(N) * N / (attn_ms * 1e-3) / 1e9
+    peak = SMS * EX2_PER_CLK_SM * sm_mhz * 1e6 / 1e9
+    return {"kernel": "k_vc_attn_fwd4", "bound": "alu", "achieved": achieved, "peak": peak, "unit": "Gexp2/s",
+            "frac": achieved / peak, "traffic": None,
+            "peak_source": f"{SMS} SMs x {EX2_PER_CLK_SM} ex2/clk/SM x {sm_mhz:.0f} MHz (median SM clock under load)",
+            "algorithmic": "B*H*N^2 exp2 per launch"}
+
+
+def measure_video_variants(torch, vcattn, synth, stream, warmup, steps, world):
+    """The video workload on both paths: the 8-bit path and the NVFP4-residual
+    variant (vc_attn_fwd with clustering in the call, CUDA events on the stream)."""
+    wl, x = synth.make_by_name(VARIANT_WORKLOAD)
+    B, H, N = wl.B, wl.H, wl.N
+    q, k, v = (_to_dev(torch, x[n]) for n in "qkv")
+    del x
+    out = torch.empty_like(q)
+    res = {}
+    for tag, extra in (("fp8", 0), ("nvfp4", vcattn.VC_VFMT_NVFP4)):
+        p = vcattn.params(flags=vcattn.FLAGS_DEFAULT | extra)
+        ws, nb = vcattn.workspace(B, H, N, p)
+
+        def step():
+            st = vcattn.vc_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, 128, None, p,
+                                    out.data_ptr(), ws.data_ptr(), nb, stream.cuda_stream)
+            if st != 0:
+                raise vcattn.VcError(st, "vc_attn_fwd")
+
+        for _ in range(warmup):
+            step()
+        vcattn.vc_attn_profile(True)
+        torch.cuda.synchronize()
+        clocks = ClockSampler(torch.cuda.current_device())
+        clocks.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        e1.synchronize()
+        clk = clocks.stop()
+        ph = vcattn.vc_attn_profile_read()
+        vcattn.vc_attn_profile(False)
+        ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+        attn_ms = float(ph[3]) if len(ph) == 4 else None
+        r = {"workload": VARIANT_WORKLOAD, "vfmt": tag, "ms_per_step": ms,
+             "value": job_tflops(world, wl.flops, ms), "unit": "TFLOPS",
+             "attn_ms": attn_ms, "attn_tflops": wl.flops / (attn_ms * 1e-3) / 1e12 if attn_ms else None,
+             "clocks": clk}
+        if tag == "nvfp4":
+            r["roofline"] = exp2_roofline(B, H, N, attn_ms, clk.get("sm_mhz"))
+        res[tag] = r
+        del ws
+    del q, k, v, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -228,10 +321,11 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     sptr = stream.cuda_stream
 
-    wl, x = synth.make_by_name(WORKLOAD)
+    wl, x = synth.make_by_name(args.workload)
     B, H, N, d = wl.B, wl.H, wl.N, 128
     q, k, v = (_to_dev(torch, x[n]) for n in "qkv")
-    p = vcattn.params()
+    nvfp4 = args.vfmt == "nvfp4"
+    p = vcattn.params(flags=vcattn.FLAGS_DEFAULT | (vcattn.VC_VFMT_NVFP4 if nvfp4 else 0))
     ws, ws_bytes = vcattn.workspace(B, H, N, p)
     out = torch.empty_like(q)
 
@@ -359,20 +453,42 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        # four whole heads (every query row): about 10-15 s of oracle work
-        tf, cores, sample, _ = cpu_oracle_sample(wl, x, rows_per_head=wl.N, heads=(0, 1, 2, 3))
+        # four whole heads (every query row) on the image workload: about 10-15 s
+        # of oracle work; on larger workloads a bounded number of rows per head
+        rows = wl.N if wl.N <= 20000 else 2048
+        tf, cores, sample, _ = cpu_oracle_sample(wl, x, rows_per_head=rows, heads=(0, 1, 2, 3), nvfp4=nvfp4)
         cpu = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample}
+    variants = None
+    if args.workload == WORKLOAD and not nvfp4:
+        del x
+        variants = measure_video_variants(torch, vcattn, synth, stream, args.warmup, min(args.steps, 5), world)
 
     if rank == 0:
+        metric = METRIC if (args.workload == WORKLOAD and not nvfp4) else \
+            f"vc_attn_fwd TFLOPS (4N²dH/t) on {args.workload}, V residual {args.vfmt}"
+        if nvfp4:
+            roof = exp2_roofline(B, H, N, attn_ms, clk.get("sm_mhz"))
+        else:
+            roof = {"kernel": "k_vc_attn_fwd", "bound": "tensor", "achieved": attn_tflops,
+                    "peak": fp8_peak, "unit": "TFLOP/s",
+                    "frac": (attn_tflops / fp8_peak) if attn_tflops else None,
+                    "traffic": traffic,
+                    "peak_source": f"{peak_src}: 2 x {'sustained' if long_region else 'burst'} "
+                                   f"cuBLAS bf16 ({bf16_peak:.1f} TFLOP/s)",
+                    "algorithmic": "4*B*H*N^2*d FLOP per launch"}
         line = {
-            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "metric": metric, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate)", "data": "synthetic",
+            "vs_baseline": None,
+            "dtype": ("fp8_e4m3 QK, nvfp4 (e2m1 + e4m3 block-16 scales) PV, fp32 accumulate" if nvfp4
+                      else "fp8_e4m3 (fp32 accumulate)"),
+            "data": "synthetic",
             "pct_of_fp8_peak": 100.0 * (value / world) / fp8_peak,
-            "config": {"workload": WORKLOAD, "B": B, "H": H, "N": N, "d": d, "k": p.k, "iters": p.iters,
+            "config": {"workload": args.workload, "vfmt": args.vfmt, "B": B, "H": H, "N": N, "d": d, "k": p.k,
+                       "iters": p.iters,
                        "rho": round(p.rho, 6), "expcast_bias": p.expcast_bias,
                        "step": "vc_attn_fwd with clustering in the call",
-                       "l2": "inputs larger than L2 (Q, K, V bf16 = 305 MB > 126 MB)",
+                       "l2": f"inputs larger than L2 (Q, K, V bf16 = {3 * q.numel() * 2 / 1e6:.0f} MB > 126 MB)",
                        "parallelism": f"replicas x{world} (independent heads, no collective)"},
             "phases_ms": {"cluster": float(ph_mean[0]), "quant_qk": float(ph_mean[1]),
                           "quant_v_repair": float(ph_mean[2]), "attention": attn_ms},
@@ -382,19 +498,15 @@ def run_ours(args):
                               "cached_perm": (ms_cached - attn_ms) / attn_ms if attn_ms else None},
             "ref_bf16": {"value": world * flops / (ms_ref * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms_ref,
                          "pct_of_bf16_peak": 100.0 * (flops / (ms_ref * 1e-3) / 1e12) / bf16_peak},
-            "roofline": {"kernel": "k_vc_attn_fwd", "bound": "tensor", "achieved": attn_tflops,
-                         "peak": fp8_peak, "unit": "TFLOP/s",
-                         "frac": (attn_tflops / fp8_peak) if attn_tflops else None,
-                         "traffic": traffic,
-                         "peak_source": f"{peak_src}: 2 x {'sustained' if long_region else 'burst'} "
-                                        f"cuBLAS bf16 ({bf16_peak:.1f} TFLOP/s)",
-                         "algorithmic": "4*B*H*N^2*d FLOP per launch"},
+            "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms_e2e,
                     "h2d_bytes_per_step": bytes_in, "d2h_bytes_per_step": bytes_out},
             "gpu_launches": int(launches),
             "clocks": clk,
         }
+        if variants is not None:
+            line["variants"] = variants
         print(json.dumps(line))
     if world > 1:
         dist.barrier()
@@ -420,6 +532,9 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     ap.add_argument("--only-main", action="store_true",
                     help="warm-up + the timed main loop only (the small case profiler captures wrap)")
+    ap.add_argument("--workload", default=WORKLOAD, help="synthetic workload name (bit_attention_diffusion_b200.synth)")
+    ap.add_argument("--vfmt", default="e4m3", choices=["e4m3", "nvfp4"],
+                    help="V residual format: the 8-bit path (default) or the NVFP4-residual variant")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

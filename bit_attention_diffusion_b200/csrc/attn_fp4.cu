@@ -108,29 +108,60 @@ __device__ __forceinline__ float2 fma2(float a0, float a1, float b, float c) {
   return r;
 }
 
-// 16 scores of one key block -> 8 bytes of E2M1 codes (w0, w1: keys 0-7 and
-// 8-15, two per byte, the even key in the low nibble) and the E4M3 scale code.
-// bmax is the block's largest score (or -inf when no key is valid).
-__device__ __forceinline__ uint32_t p_block(const float *s, float bmax, float al8, float nF8, const float *rcp_tab,
-                                            uint32_t &w0, uint32_t &w1) {
-  const float a = ex2_approx(__fmaf_rn(bmax, al8, nF8));
-  const uint32_t sc = e4m3x2(__fmul_rn(a, 448.0f), 0.0f) & 0xFFu;
-  const float rcp = rcp_tab[sc];
-  uint32_t w[2];
+// Two lanes of a product at once (one packed f32x2 instruction).
+__device__ __forceinline__ float2 mul2(float a0, float a1, float b) {
+  float2 r;
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %4};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a0), "f"(a1), "f"(b));
+  return r;
+}
+
+// Eight values -> eight E2M1 codes (round to nearest even, saturating), value
+// 2i in the low nibble of byte i. cvt...e2m1x2 puts its first source in the
+// high nibble.
+__device__ __forceinline__ uint32_t e2m1x8(const float *q) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
+  return r;
+}
+
+// The E4M3 scale codes of the 8 key blocks of a row (bm: block maxima of the
+// scores, -inf for a block without valid keys): sf = E4M3(fl(2^x_max * 448)).
+__device__ __forceinline__ void p_scales(const float *bm, float al8, float nF8, uint32_t *sc) {
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t v = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 x = fma2(s[8 * h + 2 * e], s[8 * h + 2 * e + 1], al8, nF8);
-      const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
-      v |= e2m1x2(__fmul_rn(p0, rcp), __fmul_rn(p1, rcp)) << (8 * e);
-    }
-    w[h] = v;
+  for (int i = 0; i < 4; ++i) {
+    const float a0 = ex2_approx(__fmaf_rn(bm[2 * i], al8, nF8));
+    const float a1 = ex2_approx(__fmaf_rn(bm[2 * i + 1], al8, nF8));
+    const uint32_t c2 = e4m3x2(__fmul_rn(a0, 448.0f), __fmul_rn(a1, 448.0f));
+    sc[2 * i] = c2 & 0xFFu;
+    sc[2 * i + 1] = (c2 >> 8) & 0xFFu;
   }
-  w0 = w[0];
-  w1 = w[1];
-  return sc;
+}
+
+// 16 scores of one key block -> 8 bytes of E2M1 codes (w0: keys 0-7, w1: keys
+// 8-15): code = E2M1(fl(2^x) * rcp), x = fma(acc, alpha/8, -F/8).
+__device__ __forceinline__ void p_block(const float *s, float al8, float nF8, float rcp, uint32_t &w0,
+                                        uint32_t &w1) {
+  float q[16];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float2 x = fma2(s[2 * e], s[2 * e + 1], al8, nF8);
+    const float2 pq = mul2(ex2_approx(x.x), ex2_approx(x.y), rcp);
+    q[2 * e] = pq.x;
+    q[2 * e + 1] = pq.y;
+  }
+  w0 = e2m1x8(q);
+  w1 = e2m1x8(q + 8);
 }
 
 }  // namespace
@@ -507,16 +538,27 @@ __global__ void __launch_bounds__(352, 1)
       {
         const float al8 = __fmul_rn(alpha, 0.125f), nF8 = -Fn * 0.125f;
         uint8_t *slotp = sP + (t % NPSLOT) * SZ_PSLOT;
+        uint32_t sc[8];
+        p_scales(bm, al8, nF8, sc);
+        if constexpr (LAST) {
+#pragma unroll
+          for (int kb = 0; kb < 8; ++kb)
+            if (16 * kb >= tail) sc[kb] = 0u;  // no valid key: scale 0, codes 0
+        }
+        float rcp[8];
+#pragma unroll
+        for (int kb = 0; kb < 8; ++kb) rcp[kb] = s_rcp[sc[kb]];
         uint32_t scw[2] = {0u, 0u};
+#pragma unroll
+        for (int kb = 0; kb < 8; ++kb) scw[kb >> 2] |= sc[kb] << (8 * (kb & 3));
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {  // 32 keys = 2 blocks = one 16-byte chunk
           uint32_t w[4];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int kb = 2 * ch + h;
-            uint32_t scb = p_block(&s[16 * kb], bm[kb], al8, nF8, s_rcp, w[2 * h], w[2 * h + 1]);
+            p_block(&s[16 * kb], al8, nF8, rcp[kb], w[2 * h], w[2 * h + 1]);
             if constexpr (LAST) {
-              if (16 * kb >= tail) scb = 0u;
 #pragma unroll
               for (int q = 0; q < 2; ++q) {
                 uint32_t keep = 0u;
@@ -526,7 +568,6 @@ __global__ void __launch_bounds__(352, 1)
                 w[2 * h + q] &= keep;
               }
             }
-            scw[kb >> 2] |= scb << (8 * (kb & 3));
           }
           *reinterpret_cast<uint4 *>(slotp + V4_SF_BYTES + sw64_off(r, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
         }

@@ -517,7 +517,7 @@ def run_ours(args):
 def _kernel_hash() -> str:
     import hashlib
     h = hashlib.sha256()
-    for name in ("attn_fp8.cu", "attn_fp8.cuh", "expcast.cuh", "sm100.cuh"):
+    for name in ("attn_fp8.cu", "attn_fp8.cuh", "attn_common.cuh", "expcast.cuh", "sm100.cuh"):
         with open(os.path.join(ROOT, "bit_attention_diffusion_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -1,7 +1,6 @@
 // api.cu - the C ABI of libvcattn (declared in include/vc_attn.h): argument
 // validation, workspace layout, TMA tensor maps and kernel launches.
 #include <atomic>
-#include <cstdlib>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -154,8 +153,6 @@ vc_status check_device() {
               cudaSuccess ||
           cudaFuncSetAttribute(k_vc_attn_fwd4, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(attn_fp4_smem_bytes())) != cudaSuccess ||
-          cudaFuncSetAttribute(k_vc_attn_fwd_2q, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(attn_fp8_2q_smem_bytes())) != cudaSuccess ||
           cudaFuncSetAttribute(k_kmeans_pass8, cudaFuncAttributeMaxDynamicSharedMemorySize, KMEANS8_SMEM) !=
               cudaSuccess) {
         ok_cache[dev] = 0;
@@ -489,14 +486,7 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
   ap.k8 = k8;
   ap.O = static_cast<uint16_t *>(O);
   ap.status = w.at<uint32_t>(w.L.status);
-  static const bool one_q = [] {
-    const char *e = std::getenv("VCATTN_FP8_KERNEL");
-    return e && std::strcmp(e, "1q") == 0;
-  }();
-  if (one_q)
-    k_vc_attn_fwd<<<dim3(sh.Nb, sh.BH), 352, attn_fp8_smem_bytes(), s>>>(tq, tk, tv, tmu, tdt, ap);
-  else
-    k_vc_attn_fwd_2q<<<dim3((sh.Nb + 1) / 2, sh.BH), 352, attn_fp8_2q_smem_bytes(), s>>>(tq, tk, tv, tmu, tdt, ap);
+  k_vc_attn_fwd<<<dim3((sh.Nb + 1) / 2, sh.BH), 352, attn_fp8_smem_bytes(), s>>>(tq, tk, tv, tmu, tdt, ap);
   count_launch();
   prof_mark(4, s);
   if (g_prof.on) ++g_prof.calls;

@@ -10,8 +10,9 @@
 // génération d'images sur Blackwell", "Le compromis entre vitesse et
 // fidélité": repair of the worst tokens.
 //
-// The decomposition is the FP8 kernel's (k_vc_attn_fwd): one CTA per
-// (128-query tile, b*h), 11 warps:
+// One CTA per (128-query tile, b*h), 11 warps; the two softmax warpgroups
+// take the KV tiles of that query tile in turn and hand the running frame from
+// tile to tile:
 //   warp 0     lane 0: Q, the K8 tiles (4-stage ring), then the repair deltas;
 //              lane 1: the NVFP4 V tile images (scales + codes, one 9 KB bulk
 //              copy per tile, 4-stage ring) and the block-mean chunks.
@@ -21,7 +22,7 @@
 //   warp 2     issues QK^T (FP8).
 //   warps 3-10 two softmax warpgroups taking the KV tiles in turn, one thread
 //              per query row.
-// What differs from the FP8 kernel:
+// What is specific to the 4-bit products:
 //   - P lives in shared memory: the block-scaled FP4 MMA reads both operands
 //     from there. Three slots of [1 KB scales | 8 KB codes]; the PV warp copies
 //     a slot's scales into TMEM (tcgen05.cp) right before the product.
@@ -440,9 +441,13 @@ __global__ void __launch_bounds__(352, 1)
   } else {
     // ------------------------------------------------------------ softmax rows
     // Warpgroup g (warps 3+4g .. 6+4g) takes the tiles t with t % 2 == g;
-    // thread row r = 32*(warp%4) + lane. Frame hand-over (s_F, mxr) and the
-    // row-sum bookkeeping are the FP8 kernel's; only the row-sum columns differ
-    // (tile t: column 384 + t % 4, so a warpgroup owns columns g and g + 2).
+    // thread row r = 32*(warp%4) + lane. The frame is handed from tile to
+    // tile in order through s_F (mxr[t%2]). Row sums stay with the warpgroup
+    // that owns the tile: lt_own (registers) and its own slots of sLb (slot
+    // t%32 of every tile t of parity g), all in the frame of its latest tile;
+    // l_t is the difference of two reads of column 384 + t % 4 (a warpgroup
+    // owns columns g and g + 2). The two warpgroups meet only where a chunk of
+    // 32 row sums is flushed for the block-mean restore, and at the end.
     const int g = (warp - 3) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
@@ -643,9 +648,9 @@ __global__ void __launch_bounds__(352, 1)
       ok = ragged ? tile(T - 1, std::true_type{}) : tile(T - 1, std::false_type{});
 
     // ---------------------------------------------------------- end of the KV loop
-    // As in the FP8 kernel: the last tile's warpgroup takes the other's
-    // row-sum state, adds l_{T-2} and l_{T-1}, flushes the remaining restore
-    // chunks, runs the repair; both warpgroups write half of the output.
+    // The last tile's warpgroup takes the other's row-sum state, adds
+    // l_{T-2} and l_{T-1}, flushes the remaining restore chunks and runs the
+    // repair; both warpgroups write half of the output.
     const bool fin_wg = ((T - 1) & 1) == g;
     if (!fin_wg) {
       s_lto[r] = lt_own;  // frame F_{T-2}, the frame the last tile was handed

@@ -16,14 +16,10 @@ struct AttnFp8Params {
   uint32_t *status;           // device status word
 };
 
+// Grid ceil(Nb/2) x B*H: CTA x takes query tiles 2x and 2x+1.
 __global__ void k_vc_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmMu,
                               const __grid_constant__ CUtensorMap tmDT, const AttnFp8Params p);
 uint32_t attn_fp8_smem_bytes();
-// Two 128-query tiles per CTA (grid ceil(Nb/2) x B*H), same parameters.
-__global__ void k_vc_attn_fwd_2q(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmMu,
-                                 const __grid_constant__ CUtensorMap tmDT, const AttnFp8Params p);
-uint32_t attn_fp8_2q_smem_bytes();
 
 }  // namespace vc

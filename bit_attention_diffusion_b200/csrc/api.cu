@@ -219,6 +219,20 @@ void prof_mark(int i, cudaStream_t s) {
 
 vc_status last_error() { return cudaGetLastError() == cudaSuccess ? VC_OK : VC_ERR_CUDA; }
 
+// One non-blocking side stream per device for the prologue work that runs
+// concurrently with the caller's stream (created on first use, kept for the
+// life of the process; ordering with the caller's stream is by events only).
+cudaStream_t side_stream() {
+  static std::mutex m;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> g(m);
+  if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+    streams[dev] = nullptr;
+  return streams[dev];
+}
+
 // Clear the completion counters and the status word at the start of a call.
 vc_status clear_small(const Ws &w, cudaStream_t s) {
   // status and the per-(b,h) counters are the regions of the layout before perm
@@ -425,10 +439,24 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
   uint8_t *q8 = w.at<uint8_t>(w.L.q8), *k8 = w.at<uint8_t>(w.L.k8), *v8t = w.at<uint8_t>(w.L.v8t);
   float *sq = w.at<float>(w.L.sq), *sk = w.at<float>(w.L.sk), *vscale = w.at<float>(w.L.vscale);
   int32_t *rep_idx = w.at<int32_t>(w.L.rep_idx);
-  launch_quant_qk(sh, w, Qh, Kh, pm, q8, sq, k8, sk, s);
-  prof_mark(2, s);
+  // Q/K quantization on a side stream, concurrent with the V passes on the
+  // caller's stream (they touch disjoint workspace regions); the attention
+  // kernel waits for both. Per-call events, released once the work completes.
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  cudaStream_t side = side_stream();
+  if (!side || cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) != cudaSuccess)
+    return VC_ERR_CUDA;
+  cudaEventRecord(ev_fork, s);
+  cudaStreamWaitEvent(side, ev_fork, 0);
+  launch_quant_qk(sh, w, Qh, Kh, pm, q8, sq, k8, sk, side);
+  cudaEventRecord(ev_join, side);
   launch_quant_v(sh, w, Vh, pm, v8t, vscale, w.at<uint16_t>(w.L.vmean), rep_idx, w.at<uint16_t>(w.L.rep_delta), s);
+  prof_mark(2, s);
+  cudaStreamWaitEvent(s, ev_join, 0);
   prof_mark(3, s);
+  cudaEventDestroy(ev_fork);
+  cudaEventDestroy(ev_join);
 
   const bool fp4 = (sh.flags & VC_VFMT_NVFP4) != 0;
   CUtensorMap tq, tk, tv, tmu, tdt;

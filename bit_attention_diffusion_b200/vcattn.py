@@ -172,8 +172,9 @@ def vc_attn_profile(on: bool) -> int:
 
 
 def vc_attn_profile_read() -> list:
-    """Phase durations (ms) of the last profiled vc_attn_fwd call:
-    [cluster, quant_qk, quant_v, attention]; [] if none was recorded."""
+    """Mean phase durations (ms) of the profiled vc_attn_fwd calls:
+    [cluster, quant_v (Q/K quantization overlaps it on a side stream),
+    further wait for quant_qk, attention]; [] if none was recorded."""
     buf = (ctypes.c_float * 4)()
     n = lib().vc_attn_profile_read(buf, 4)
     return [float(buf[i]) for i in range(n)]

@@ -37,6 +37,7 @@ FLAG_VSMOOTH = 1
 FLAG_REPAIR = 2
 FLAG_KSMOOTH = 8
 FLAG_VFMT_NVFP4 = 32
+FLAG_QK_NVFP4 = 64  # full 4-bit path: Q and K in NVFP4 too (with FLAG_VFMT_NVFP4)
 FLAGS_DEFAULT = FLAG_VSMOOTH | FLAG_REPAIR | FLAG_KSMOOTH
 
 
@@ -94,6 +95,9 @@ def lib():
             L.orc_quant_v4_head.argtypes = [P, P, i32, i32, i32, i32, P, P, P, P, P, P, P]
             L.orc_attn_vc4_rows.argtypes = [P, P, P, P, P, P, P, P, P, P, i32, i32, i32, f32,
                                             P, i32, P, P, P]
+            L.orc_quant_qk4_head.argtypes = [P, P, P, i32, i32, i32, P, P, P, P, P, P, P]
+            L.orc_attn_vc44_rows.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, i32, i32, i32, f32,
+                                             P, i32, P, P, P]
             _lib = L
     return _lib
 
@@ -309,6 +313,42 @@ def attn_vc4_rows(qk: dict, vq: dict, N: int, rows, softmax_scale: float = DEFAU
     return out, out_l, out_F
 
 
+def quant_qk4_head(q_bits, k_bits, perm, ksmooth: bool = True):
+    """NVFP4 Q (original order) and K' (permuted, smoothed): codes [Nb*128, d]
+    (low nibble), block scale codes [Nb*128, d/16], per-128-row-block global
+    scales g [Nb] (powers of two), and the K channel means."""
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    pm = np.ascontiguousarray(perm, dtype=np.int32)
+    N, d = q.shape
+    Nb = (N + TILE - 1) // TILE
+    out = dict(qcodes=np.empty((Nb * TILE, d), np.uint8), qsfc=np.empty((Nb * TILE, d // 16), np.uint8),
+               qg=np.empty(Nb, np.float32), kcodes=np.empty((Nb * TILE, d), np.uint8),
+               ksfc=np.empty((Nb * TILE, d // 16), np.uint8), kg=np.empty(Nb, np.float32),
+               kbar=np.empty(d, np.float32))
+    lib().orc_quant_qk4_head(_p(q), _p(k), _p(pm), N, d, int(bool(ksmooth)), _p(out["qcodes"]), _p(out["qsfc"]),
+                             _p(out["qg"]), _p(out["kcodes"]), _p(out["ksfc"]), _p(out["kg"]), _p(out["kbar"]))
+    return out
+
+
+def attn_vc44_rows(qk4: dict, vq: dict, N: int, rows, softmax_scale: float = DEFAULT_SCALE):
+    """The full 4-bit path's attention for the given query rows of one head."""
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    d = qk4["qcodes"].shape[1]
+    out = np.empty((rows.size, d), np.float64)
+    out_l = np.empty(rows.size, np.float64)
+    out_F = np.empty(rows.size, np.float32)
+    R = int(vq["rep_idx"].size)
+    ri = vq["rep_idx"] if R else np.zeros(1, np.int32)
+    rd = vq["rep_delta"] if R else np.zeros((1, d), np.uint16)
+    lib().orc_attn_vc44_rows(_p(qk4["qcodes"]), _p(qk4["qsfc"]), _p(qk4["qg"]), _p(qk4["kcodes"]),
+                             _p(qk4["ksfc"]), _p(qk4["kg"]), _p(vq["codes"]), _p(vq["sfc"]), _p(vq["vscale"]),
+                             _p(vq["vmean"]), _p(np.ascontiguousarray(ri)), _p(np.ascontiguousarray(rd)), R,
+                             int(N), d, float(kappa(softmax_scale)), _p(rows), rows.size,
+                             _p(out), _p(out_l), _p(out_F))
+    return out, out_l, out_F
+
+
 # ---------------------------------------------------------------- whole path
 def head_prologue(q_bits, k_bits, v_bits, flags: int = FLAGS_DEFAULT, k: int = 8, iters: int = 3,
                   rho: float = 0.005, perm=None):
@@ -323,7 +363,11 @@ def head_prologue(q_bits, k_bits, v_bits, flags: int = FLAGS_DEFAULT, k: int = 8
             perm = np.arange(N, dtype=np.int32)
     perm = np.ascontiguousarray(perm, dtype=np.int32)
     R = repair_count(rho, N) if (flags & FLAG_REPAIR) else 0
-    qk = quant_qk_head(q_bits, k_bits, perm, ksmooth=bool(flags & FLAG_KSMOOTH))
+    if flags & FLAG_QK_NVFP4:
+        assert flags & FLAG_VFMT_NVFP4, "the full 4-bit path needs the NVFP4 residual too"
+        qk = quant_qk4_head(q_bits, k_bits, perm, ksmooth=bool(flags & FLAG_KSMOOTH))
+    else:
+        qk = quant_qk_head(q_bits, k_bits, perm, ksmooth=bool(flags & FLAG_KSMOOTH))
     quant_v = quant_v4_head if (flags & FLAG_VFMT_NVFP4) else quant_v_head
     vq = quant_v(v_bits, perm, demean=bool(flags & FLAG_VSMOOTH), R=R)
     return dict(perm=perm, cent=cent, labels=labels, qk=qk, vq=vq, R=R)
@@ -337,7 +381,9 @@ def vc_attention_head(q_bits, k_bits, v_bits, rows=None, flags: int = FLAGS_DEFA
     pro = head_prologue(q_bits, k_bits, v_bits, flags, k, iters, rho, perm)
     if rows is None:
         rows = np.arange(N, dtype=np.int32)
-    if flags & FLAG_VFMT_NVFP4:
+    if flags & FLAG_QK_NVFP4:
+        out, l, F = attn_vc44_rows(pro["qk"], pro["vq"], N, rows, softmax_scale)
+    elif flags & FLAG_VFMT_NVFP4:
         out, l, F = attn_vc4_rows(pro["qk"], pro["vq"], N, rows, softmax_scale)
     else:
         out, l, F = attn_vc_rows(pro["qk"], pro["vq"], N, rows, softmax_scale, C)

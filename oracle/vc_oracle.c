@@ -121,6 +121,10 @@ uint8_t orc_e4m3_encode(float x)
     return (uint8_t)(sign | code);
 }
 
+/* OCP FP4 E2M1, defined with the NVFP4 variant below. */
+double orc_e2m1_value(uint8_t code);
+uint8_t orc_e2m1_encode(float x);
+
 /* ------------------------------------------------------------------ */
 /* ExpCast-FP8 ([VCA] "ExpCast-FP8: eliminando o gargalo do softmax")   */
 /* ------------------------------------------------------------------ */
@@ -278,6 +282,76 @@ void orc_quant_qk_head(const uint16_t *Q, const uint16_t *K, const int32_t *perm
                 blk[(size_t)i * d + c] = orc_bf16_value(K[(size_t)src * d + c]) - kbar[c];
         }
         quant_block_rows(blk, rows, d, k8 + (size_t)r0 * d, &sk[t]);
+    }
+    free(blk);
+}
+
+/* NVFP4 Q and K' for the full 4-bit path [R]: the same smoothing and row
+ * order as orc_quant_qk_head; per 128-row block a power-of-two global scale
+ * g = 2^e, the least with amax <= 2688 * 2^e over the block (1 when the block
+ * is all zero); per row and 16 consecutive channels the E4M3 scale
+ * sf = E4M3(fl(fl(b * 2^-e) / 6)) of the block maximum b, and the codes
+ * E2M1(fl(fl(x * 2^-e) * fl(1 / sf))) (every code 0 when sf is 0): the value
+ * format of the NVFP4 residual, with the blocks along the channels (the K
+ * dimension of QK^T). Outputs: codes [Nb*128][d] (padding rows 0),
+ * sfc [Nb*128][d/16], g [Nb]. */
+static void quant4_block_rows(const float *X, int rows, int d, uint8_t *codes, uint8_t *sfc, float *g)
+{
+    float amax = 0.0f;
+    int e = 0, E, db = d / 16;
+    for (int i = 0; i < rows * d; ++i)
+        if (fabsf(X[i]) > amax)
+            amax = fabsf(X[i]);
+    if (amax > 0.0f) {
+        float f = frexpf(amax, &E); /* 2688 = 0.65625 * 2^12 */
+        e = (f > 0.65625f) ? E - 11 : E - 12;
+    }
+    *g = ldexpf(1.0f, e);
+    for (int i = 0; i < rows; ++i)
+        for (int jb = 0; jb < db; ++jb) {
+            const float *x = X + (size_t)i * d + 16 * jb;
+            float b = 0.0f, sfv, rcp;
+            uint8_t sc;
+            for (int c = 0; c < 16; ++c)
+                if (fabsf(x[c]) > b)
+                    b = fabsf(x[c]);
+            sc = orc_e4m3_encode(ldexpf(b, -e) / 6.0f);
+            sfv = (float)orc_e4m3_value(sc);
+            rcp = (sfv == 0.0f) ? 0.0f : 1.0f / sfv;
+            sfc[(size_t)i * db + jb] = sc;
+            for (int c = 0; c < 16; ++c)
+                codes[(size_t)i * d + 16 * jb + c] = (sfv == 0.0f) ? 0 : orc_e2m1_encode(ldexpf(x[c], -e) * rcp);
+        }
+}
+
+void orc_quant_qk4_head(const uint16_t *Q, const uint16_t *K, const int32_t *perm, int N, int d, int ksmooth,
+                        uint8_t *qcodes, uint8_t *qsfc, float *qg, uint8_t *kcodes, uint8_t *ksfc, float *kg,
+                        float *kbar)
+{
+    int Nb = (N + TILE - 1) / TILE, db = d / 16;
+    float *blk = (float *)malloc((size_t)TILE * d * sizeof(float));
+    for (int c = 0; c < d; ++c) {
+        double s = 0.0;
+        for (int n = 0; n < N; ++n)
+            s += (double)orc_bf16_value(K[(size_t)n * d + c]);
+        kbar[c] = ksmooth ? (float)(s / (double)N) : 0.0f;
+    }
+    memset(qcodes, 0, (size_t)Nb * TILE * d);
+    memset(kcodes, 0, (size_t)Nb * TILE * d);
+    memset(qsfc, 0, (size_t)Nb * TILE * db);
+    memset(ksfc, 0, (size_t)Nb * TILE * db);
+    for (int t = 0; t < Nb; ++t) {
+        int r0 = t * TILE, rows = (N - r0 < TILE) ? N - r0 : TILE;
+        for (int i = 0; i < rows; ++i)
+            for (int c = 0; c < d; ++c)
+                blk[(size_t)i * d + c] = orc_bf16_value(Q[(size_t)(r0 + i) * d + c]);
+        quant4_block_rows(blk, rows, d, qcodes + (size_t)r0 * d, qsfc + (size_t)r0 * db, &qg[t]);
+        for (int i = 0; i < rows; ++i) {
+            int src = perm[r0 + i];
+            for (int c = 0; c < d; ++c)
+                blk[(size_t)i * d + c] = orc_bf16_value(K[(size_t)src * d + c]) - kbar[c];
+        }
+        quant4_block_rows(blk, rows, d, kcodes + (size_t)r0 * d, ksfc + (size_t)r0 * db, &kg[t]);
     }
     free(blk);
 }
@@ -750,37 +824,21 @@ void orc_quant_v4_head(const uint16_t *V, const int32_t *perm, int N, int d, int
  * with P'_ij = bf16(fp32(2^x'_ij * 2688)) and x'_ij the exponent against the
  * final frame [R]; then O_i = num / l. Inputs: vcodes[N][d], vsfc[ceil(N/16)][d]
  * and vscale[d] = g_c as orc_quant_v4_head writes them. */
-void orc_attn_vc4_rows(const uint8_t *q8, const float *sq, const uint8_t *k8, const float *sk,
-                       const uint8_t *vcodes, const uint8_t *vsfc, const float *vscale, const uint16_t *vmean,
-                       const int32_t *rep_idx, const uint16_t *rep_delta, int R,
-                       int N, int d, float kappa, const int32_t *rows, int nrows,
-                       double *out, double *out_l, float *out_F)
+static void attn_vc4_core(const double *qd_all, const float *sq, const double *kd, const float *sk,
+                          const double *vd, const double *mud, const int32_t *rep_idx, const uint16_t *rep_delta,
+                          int R, int N, int d, float kappa, const int32_t *rows, int nrows, double *out,
+                          double *out_l, float *out_F)
 {
     int Nb = (N + TILE - 1) / TILE;
-    double *kd = (double *)malloc((size_t)N * d * sizeof(double));
-    double *vd = (double *)malloc((size_t)N * d * sizeof(double));
-    double *mud = (double *)malloc((size_t)Nb * d * sizeof(double));
-    for (int j = 0; j < N; ++j)
-        for (int c = 0; c < d; ++c) {
-            kd[(size_t)j * d + c] = orc_e4m3_value(k8[(size_t)j * d + c]);
-            vd[(size_t)j * d + c] = orc_e2m1_value(vcodes[(size_t)j * d + c]) *
-                                    orc_e4m3_value(vsfc[(size_t)(j / 16) * d + c]) * (double)vscale[c];
-        }
-    for (int t = 0; t < Nb; ++t)
-        for (int c = 0; c < d; ++c)
-            mud[(size_t)t * d + c] = (double)orc_bf16_value(vmean[(size_t)t * d + c]);
-
 #pragma omp parallel for schedule(dynamic, 1)
     for (int ir = 0; ir < nrows; ++ir) {
         int i = rows[ir];
-        double qd[TILE * 2];
+        const double *qd = qd_all + (size_t)i * d;
         double *num = (double *)calloc((size_t)d, sizeof(double));
         float *acc = (float *)malloc((size_t)TILE * sizeof(float));
         double l = 0.0;
         float m = -INFINITY, F = -INFINITY;
         float sqi = sq[i / TILE];
-        for (int c = 0; c < d; ++c)
-            qd[c] = orc_e4m3_value(q8[(size_t)i * d + c]);
         for (int t = 0; t < Nb; ++t) {
             int j0 = t * TILE, j1 = (j0 + TILE < N) ? j0 + TILE : N;
             float alpha = (sqi * sk[t]) * kappa;
@@ -841,6 +899,70 @@ void orc_attn_vc4_rows(const uint8_t *q8, const float *sq, const uint8_t *k8, co
         free(num);
         free(acc);
     }
+}
+
+/* The NVFP4 values and block means in the units the core multiplies. */
+static void v4_dequant(const uint8_t *vcodes, const uint8_t *vsfc, const float *vscale, const uint16_t *vmean,
+                       int N, int d, double *vd, double *mud)
+{
+    int Nb = (N + TILE - 1) / TILE;
+    for (int j = 0; j < N; ++j)
+        for (int c = 0; c < d; ++c)
+            vd[(size_t)j * d + c] = orc_e2m1_value(vcodes[(size_t)j * d + c]) *
+                                    orc_e4m3_value(vsfc[(size_t)(j / 16) * d + c]) * (double)vscale[c];
+    for (int t = 0; t < Nb; ++t)
+        for (int c = 0; c < d; ++c)
+            mud[(size_t)t * d + c] = (double)orc_bf16_value(vmean[(size_t)t * d + c]);
+}
+
+void orc_attn_vc4_rows(const uint8_t *q8, const float *sq, const uint8_t *k8, const float *sk,
+                       const uint8_t *vcodes, const uint8_t *vsfc, const float *vscale, const uint16_t *vmean,
+                       const int32_t *rep_idx, const uint16_t *rep_delta, int R,
+                       int N, int d, float kappa, const int32_t *rows, int nrows,
+                       double *out, double *out_l, float *out_F)
+{
+    int Nb = (N + TILE - 1) / TILE;
+    double *qd = (double *)malloc((size_t)N * d * sizeof(double));
+    double *kd = (double *)malloc((size_t)N * d * sizeof(double));
+    double *vd = (double *)malloc((size_t)N * d * sizeof(double));
+    double *mud = (double *)malloc((size_t)Nb * d * sizeof(double));
+    for (size_t i = 0; i < (size_t)N * d; ++i) {
+        qd[i] = orc_e4m3_value(q8[i]);
+        kd[i] = orc_e4m3_value(k8[i]);
+    }
+    v4_dequant(vcodes, vsfc, vscale, vmean, N, d, vd, mud);
+    attn_vc4_core(qd, sq, kd, sk, vd, mud, rep_idx, rep_delta, R, N, d, kappa, rows, nrows, out, out_l, out_F);
+    free(qd);
+    free(kd);
+    free(vd);
+    free(mud);
+}
+
+/* Full 4-bit path [R]: Q and K' in NVFP4 as well (orc_quant_qk4_head); the
+ * score is sum_c value(qcode) sfq value(kcode) sfk (exact, rounded once to
+ * binary32, as the tensor core accumulates it) and its scale the product of
+ * the two blocks' power-of-two global scales; the rest is orc_attn_vc4_rows. */
+void orc_attn_vc44_rows(const uint8_t *qcodes, const uint8_t *qsfc, const float *qg, const uint8_t *kcodes,
+                        const uint8_t *ksfc, const float *kg, const uint8_t *vcodes, const uint8_t *vsfc,
+                        const float *vscale, const uint16_t *vmean, const int32_t *rep_idx,
+                        const uint16_t *rep_delta, int R, int N, int d, float kappa, const int32_t *rows,
+                        int nrows, double *out, double *out_l, float *out_F)
+{
+    int Nb = (N + TILE - 1) / TILE, db = d / 16;
+    double *qd = (double *)malloc((size_t)N * d * sizeof(double));
+    double *kd = (double *)malloc((size_t)N * d * sizeof(double));
+    double *vd = (double *)malloc((size_t)N * d * sizeof(double));
+    double *mud = (double *)malloc((size_t)Nb * d * sizeof(double));
+    for (int j = 0; j < N; ++j)
+        for (int c = 0; c < d; ++c) {
+            qd[(size_t)j * d + c] = orc_e2m1_value(qcodes[(size_t)j * d + c]) *
+                                    orc_e4m3_value(qsfc[(size_t)j * db + c / 16]);
+            kd[(size_t)j * d + c] = orc_e2m1_value(kcodes[(size_t)j * d + c]) *
+                                    orc_e4m3_value(ksfc[(size_t)j * db + c / 16]);
+        }
+    v4_dequant(vcodes, vsfc, vscale, vmean, N, d, vd, mud);
+    attn_vc4_core(qd, qg, kd, kg, vd, mud, rep_idx, rep_delta, R, N, d, kappa, rows, nrows, out, out_l, out_F);
+    free(qd);
     free(kd);
     free(vd);
     free(mud);

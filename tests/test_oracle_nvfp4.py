@@ -307,19 +307,20 @@ def _fma32(a, b, c) -> np.float32:
     return lo if (lo.view(np.uint32) & 1) == 0 else hi
 
 
-def _direct_global_frame4(orc, pro, N, rows, scale):
+def _direct_global_frame4(orc, pro, N, rows, scale, qd_all=None, kd_all=None):
     """Every tile's probabilities quantized against its own frame F_t (by the
-    pinned block quantizer), all contributions scaled once to the final frame."""
+    pinned block quantizer), all contributions scaled once to the final frame.
+    qd_all / kd_all: the score operands (default: the E4M3 decode of q8 / k8)."""
     qk, vq = pro["qk"], pro["vq"]
     kap = np.float32(orc.kappa(scale))
     Nb = (N + 127) // 128
-    kd = orc.e4m3_value(qk["k8"][:N])
+    kd = orc.e4m3_value(qk["k8"][:N]) if kd_all is None else kd_all
     vd = _deq(orc, vq)
     mu = orc.bf16_value(vq["vmean"]).astype(np.float64)
     tile = np.arange(N) // 128
     out = []
     for i in rows:
-        qd = orc.e4m3_value(qk["q8"][i])
+        qd = orc.e4m3_value(qk["q8"][i]) if qd_all is None else qd_all[i]
         acc = (kd @ qd).astype(np.float32)
         alpha = ((np.float32(qk["sq"][i // 128]) * qk["sk"]).astype(np.float32) * kap).astype(np.float32)
         u = (acc * alpha[tile]).astype(np.float32)
@@ -370,3 +371,104 @@ def test_random_inputs_error_band_vs_exact(orc):
     e4 = np.linalg.norm(r4["out"] - ex) / np.linalg.norm(ex)
     e8 = np.linalg.norm(r8["out"] - ex) / np.linalg.norm(ex)
     assert e8 < e4 < 0.5, (e4, e8)
+
+
+# ---------------------------------------------------------------- full 4-bit path (Q and K in NVFP4 too)
+def test_quant_qk4_matches_library_roundings(orc):
+    """Per 128-row block g = the least power of two with amax <= 2688 g; per
+    row and 16 channels the scale E4M3(fl(b/g)/6) and codes
+    E2M1(fl(fl(x/g) * fl(1/sf))), from ml_dtypes roundings of the same
+    binary32 steps; K' = K - channel mean, rows through the permutation."""
+    x = synth.make_inputs(synth.custom(1, 1, 300, seed=61))
+    q, k = x["q"][0, 0], x["k"][0, 0]
+    perm = np.random.default_rng(61).permutation(300).astype(np.int32)
+    o = orc.quant_qk4_head(q, k, perm, ksmooth=True)
+    kf = synth.bf16_bits_to_f32(k).astype(np.float64)
+    kbar = (kf.sum(0) / 300).astype(np.float32)
+    assert np.array_equal(o["kbar"], kbar)
+    for name, X, codes, sfc, g in (("q", synth.bf16_bits_to_f32(q), o["qcodes"], o["qsfc"], o["qg"]),
+                                   ("k", (synth.bf16_bits_to_f32(k)[perm] - kbar).astype(np.float32), o["kcodes"],
+                                    o["ksfc"], o["kg"])):
+        for t in range(3):
+            blk = X[128 * t:128 * t + 128]
+            amax = np.abs(blk).max()
+            assert amax <= 2688 * g[t] and amax > 1344 * g[t] and np.log2(g[t]) == np.round(np.log2(g[t])), name
+            xs = (blk / g[t]).astype(np.float32)                      # exact: g is a power of two
+            b = np.abs(xs.reshape(-1, 8, 16)).max(2).astype(np.float32)
+            sf = (b / np.float32(6.0)).astype(np.float32).astype(E4M3_LIB)
+            assert np.array_equal(sf.view(np.uint8), sfc[128 * t:128 * t + len(blk)]), (name, t)
+            sfv = sf.astype(np.float32)
+            with np.errstate(divide="ignore"):
+                rcp = np.where(sfv == 0, np.float32(0), (np.float32(1.0) / sfv).astype(np.float32)).astype(np.float32)
+            want = (xs.reshape(-1, 8, 16) * rcp[:, :, None]).astype(np.float32).astype(E2M1_LIB).view(np.uint8)
+            want = np.where(sfv[:, :, None] == 0, 0, want).reshape(-1, 128)
+            assert np.array_equal(codes[128 * t:128 * t + len(blk)], want), (name, t)
+    # padding rows of the ragged last block are zero
+    assert np.all(o["qcodes"][300:] == 0) and np.all(o["ksfc"][300:] == 0)
+
+
+def _lossless_case_qk4(seed, N=300, d=128):
+    """The a10 lossless values and permutation, with Q and K on the NVFP4 grid:
+    channel block 16..31 carries everything. Q: channel 16 = 3 on every row
+    (the block maximum: g_q = 2^-9, scale 256), one of channels 17..23 = 2,
+    channel 24 = 1. K: channel 25 = 24 on every key (g_k = 2^-6, scale 256),
+    channels 17..23 in {0, -4, -8}, channel 24 = 16 on the keys at permuted
+    positions 256..271. Scores q.k lie in {0, -8, -16} (+16 for the boosted
+    keys): multiples of 8 byte units at kappa = 1."""
+    _, _, v, perm, scale = _lossless_case(seed, N, d)
+    rng = np.random.default_rng(seed + 1000)
+    q = np.zeros((N, d), np.float32)
+    q[:, 16] = 3.0
+    q[:, 24] = 1.0
+    q[np.arange(N), rng.integers(17, 24, N)] = 2.0
+    kp = np.zeros((N, d), np.float32)
+    kp[:, 25] = 24.0
+    kp[:, 17:24] = rng.choice([0.0, -4.0, -8.0], (N, 7))
+    kp[256:272, 24] = 16.0
+    k = np.empty_like(kp)
+    k[perm] = kp
+    return synth.f32_to_bf16_bits(q), synth.f32_to_bf16_bits(k), v, perm, scale
+
+
+@pytest.mark.parametrize("seed", [70, 71])
+def test_full_4bit_lossless_case_reduces_to_exact_attention(orc, seed):
+    q, k, v, perm, scale = _lossless_case_qk4(seed)
+    flags = orc.FLAG_VSMOOTH | orc.FLAG_REPAIR | orc.FLAG_VFMT_NVFP4 | orc.FLAG_QK_NVFP4
+    r = orc.vc_attention_head(q, k, v, flags=flags, rho=0.005, softmax_scale=scale, perm=perm)
+    qk = r["qk"]
+    assert np.all(qk["qg"] == 2.0 ** -9) and np.all(qk["kg"] == 2.0 ** -6)
+    # the scores' block: scale 256 on every row; the other blocks are empty
+    assert np.all(qk["qsfc"][:300, 1] == 0x78) and np.all(qk["ksfc"][:300, 1] == 0x78)   # E4M3 256
+    assert np.all(qk["qsfc"][:300, [0, 2, 3, 4, 5, 6, 7]] == 0)
+    assert np.all(r["F"] == 16.0)
+    ex = orc.exact_attention_head(q, k, v, softmax_scale=scale)
+    rel = np.abs(r["out"] - ex).max() / np.abs(ex).max()
+    assert rel < 1e-8, rel
+    # a score off the grid (one key's channel 17 at -5: between -4 and -6)
+    # breaks it
+    kb = synth.bf16_bits_to_f32(k)
+    kb[perm[10], 17] = -5.0
+    r2 = orc.vc_attention_head(q, synth.f32_to_bf16_bits(kb), v, flags=flags, softmax_scale=scale, perm=perm)
+    ex2 = orc.exact_attention_head(q, synth.f32_to_bf16_bits(kb), v, softmax_scale=scale)
+    assert np.abs(r2["out"] - ex2).max() / np.abs(ex2).max() > 1e3 * rel
+
+
+def test_full_4bit_online_rescaling_equals_global_frame_form(orc):
+    """Random inputs: the online 4-bit path equals an un-tiled evaluation that
+    takes the scores from the dequantized NVFP4 Q and K, quantizes each tile's
+    probabilities against its own frame and scales everything once."""
+    wl = synth.custom(1, 1, 400, seed=35)
+    x = synth.make_inputs(wl)
+    q, k, v = x["q"][0, 0], x["k"][0, 0], x["v"][0, 0]
+    rows = np.array([0, 5, 127, 128, 399], np.int32)
+    flags = orc.FLAGS_DEFAULT | orc.FLAG_VFMT_NVFP4 | orc.FLAG_QK_NVFP4
+    r = orc.vc_attention_head(q, k, v, rows=rows, flags=flags)
+    qk = r["qk"]
+    N = 400
+    qd = orc.e2m1_value(qk["qcodes"][:N]) * orc.e4m3_value(qk["qsfc"][:N]).repeat(16, axis=1)
+    kd = orc.e2m1_value(qk["kcodes"][:N]) * orc.e4m3_value(qk["ksfc"][:N]).repeat(16, axis=1)
+    # the FP8-path helper with the NVFP4 operands and global scales in place of
+    # the E4M3 decode and block scales
+    pro = {"qk": {"q8": None, "sq": qk["qg"], "k8": None, "sk": qk["kg"]}, "vq": r["vq"]}
+    want = _direct_global_frame4(orc, pro, N, rows, orc.DEFAULT_SCALE, qd_all=qd, kd_all=kd)
+    assert np.allclose(r["out"], want, rtol=1e-9, atol=1e-12)

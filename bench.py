@@ -11,13 +11,14 @@ attention kernel. Metric: TFLOPS = 4*B*H*N^2*d / t (the pages' attention FLOP
 count), also as % of the measured FP8 dense peak.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload NAME] [--vfmt e4m3|nvfp4]
+                  [--workload NAME] [--vfmt e4m3|nvfp4|nvfp4qk]
 
 The default line also carries "variants": the 720p video workload (B=1, H=40,
-N=75600) on the 8-bit path and on the NVFP4-residual variant (VC_VFMT_NVFP4),
-the latter with its roofline against the exp2 throughput of the special-
-function units (the variant has no ExpCast, so one 2^x per score bounds it).
---vfmt nvfp4 [--workload NAME] times the variant as the main line instead.
+N=75600) on the 8-bit path, on the NVFP4-residual variant (VC_VFMT_NVFP4) and
+on the full 4-bit path (VC_VFMT_NVFP4 | VC_QK_NVFP4), the 4-bit ones with
+their roofline against the exp2 throughput of the special-function units
+(they have no ExpCast, so one 2^x per score bounds them). --vfmt nvfp4 or
+nvfp4qk [--workload NAME] times a variant as the main line instead.
 
 N > 1 runs under torchrun: every rank owns one independent copy of the
 workload (heads are independent problems; no data-path collective), the step
@@ -43,7 +44,12 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = "image2048_b1h24n16544"
 METRIC = "vc_attn_fwd TFLOPS (4N²dH/t) at N=16544,H=24,d=128; % of B200 FP8 peak"
-VARIANT_WORKLOAD = "video720p_b1h40n75600"  # the workload the NVFP4-residual variant is timed on
+VARIANT_WORKLOAD = "video720p_b1h40n75600"  # the workload the NVFP4 variants are timed on
+VFMT_FLAGS = {"e4m3": 0, "nvfp4": 32, "nvfp4qk": 32 | 64}  # VC_VFMT_NVFP4, VC_QK_NVFP4
+ATTN_KERNEL = {"e4m3": "k_vc_attn_fwd", "nvfp4": "k_vc_attn_fwd4", "nvfp4qk": "k_vc_attn_fwd44"}
+DTYPE = {"e4m3": "fp8_e4m3 (fp32 accumulate)",
+         "nvfp4": "fp8_e4m3 QK, nvfp4 (e2m1 + e4m3 block-16 scales) PV, fp32 accumulate",
+         "nvfp4qk": "nvfp4 (e2m1 + e4m3 block-16 scales) QK and PV, fp32 accumulate"}
 SMS = 148
 EX2_PER_CLK_SM = 16  # special-function unit: 2^x results per clock per SM (CUDA throughput table, cc 10.0)
 FALLBACK_HBM_GBS = 6650.0
@@ -172,7 +178,7 @@ def _to_dev(torch, bits):
 
 
 # ---------------------------------------------------------------- CPU oracle timing
-def cpu_oracle_sample(wl, x, rows_per_head: int = 96, heads=(0,), nvfp4: bool = False):
+def cpu_oracle_sample(wl, x, rows_per_head: int = 96, heads=(0,), extra_flags: int = 0):
     """Time the oracle on a bounded sample and extrapolate to the workload.
 
     For each sampled head: the full per-head prologue (k-means, quantization,
@@ -186,11 +192,13 @@ def cpu_oracle_sample(wl, x, rows_per_head: int = 96, heads=(0,), nvfp4: bool = 
     for h in heads:
         q, k, v = x["q"][0, h], x["k"][0, h], x["v"][0, h]
         t0 = time.perf_counter()
-        flags = oracle.FLAGS_DEFAULT | (oracle.FLAG_VFMT_NVFP4 if nvfp4 else 0)
+        flags = oracle.FLAGS_DEFAULT | extra_flags
         pro = oracle.head_prologue(q, k, v, flags=flags)
         t1 = time.perf_counter()
         rows = np.linspace(0, wl.N - 1, rows_per_head).astype(np.int32)
-        if nvfp4:
+        if flags & oracle.FLAG_QK_NVFP4:
+            oracle.attn_vc44_rows(pro["qk"], pro["vq"], wl.N, rows)
+        elif flags & oracle.FLAG_VFMT_NVFP4:
             oracle.attn_vc4_rows(pro["qk"], pro["vq"], wl.N, rows)
         else:
             oracle.attn_vc_rows(pro["qk"], pro["vq"], wl.N, rows)
@@ -235,29 +243,30 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- GPU bench
-def exp2_roofline(B, H, N, attn_ms, sm_mhz):
-    """The NVFP4 variant has no ExpCast: every score goes through one 2^x on the
-    special-function unit, the kernel's bound (N^2 B H per launch)."""
+def exp2_roofline(B, H, N, attn_ms, sm_mhz, kernel="k_vc_attn_fwd4"):
+    """The NVFP4 variants have no ExpCast: every score goes through one 2^x on
+    the special-function unit, the kernel's bound (N^2 B H per launch)."""
     if not attn_ms or not sm_mhz:
         return None
     achieved = B * H * float(N) * N / (attn_ms * 1e-3) / 1e9
     peak = SMS * EX2_PER_CLK_SM * sm_mhz * 1e6 / 1e9
-    return {"kernel": "k_vc_attn_fwd4", "bound": "alu", "achieved": achieved, "peak": peak, "unit": "Gexp2/s",
+    return {"kernel": kernel, "bound": "alu", "achieved": achieved, "peak": peak, "unit": "Gexp2/s",
             "frac": achieved / peak, "traffic": None,
             "peak_source": f"{SMS} SMs x {EX2_PER_CLK_SM} ex2/clk/SM x {sm_mhz:.0f} MHz (median SM clock under load)",
             "algorithmic": "B*H*N^2 exp2 per launch"}
 
 
 def measure_video_variants(torch, vcattn, synth, stream, warmup, steps, world):
-    """The video workload on both paths: the 8-bit path and the NVFP4-residual
-    variant (vc_attn_fwd with clustering in the call, CUDA events on the stream)."""
+    """The video workload on the three paths: the 8-bit path, the NVFP4-residual
+    variant and the full 4-bit path (vc_attn_fwd with clustering in the call,
+    CUDA events on the stream)."""
     wl, x = synth.make_by_name(VARIANT_WORKLOAD)
     B, H, N = wl.B, wl.H, wl.N
     q, k, v = (_to_dev(torch, x[n]) for n in "qkv")
     del x
     out = torch.empty_like(q)
     res = {}
-    for tag, extra in (("fp8", 0), ("nvfp4", vcattn.VC_VFMT_NVFP4)):
+    for tag, extra in (("fp8", 0), ("nvfp4", VFMT_FLAGS["nvfp4"]), ("nvfp4qk", VFMT_FLAGS["nvfp4qk"])):
         p = vcattn.params(flags=vcattn.FLAGS_DEFAULT | extra)
         ws, nb = vcattn.workspace(B, H, N, p)
 
@@ -288,8 +297,8 @@ def measure_video_variants(torch, vcattn, synth, stream, warmup, steps, world):
              "value": job_tflops(world, wl.flops, ms), "unit": "TFLOPS",
              "attn_ms": attn_ms, "attn_tflops": wl.flops / (attn_ms * 1e-3) / 1e12 if attn_ms else None,
              "clocks": clk}
-        if tag == "nvfp4":
-            r["roofline"] = exp2_roofline(B, H, N, attn_ms, clk.get("sm_mhz"))
+        if tag != "fp8":
+            r["roofline"] = exp2_roofline(B, H, N, attn_ms, clk.get("sm_mhz"), ATTN_KERNEL[tag])
         res[tag] = r
         del ws
     del q, k, v, out
@@ -324,8 +333,8 @@ def run_ours(args):
     wl, x = synth.make_by_name(args.workload)
     B, H, N, d = wl.B, wl.H, wl.N, 128
     q, k, v = (_to_dev(torch, x[n]) for n in "qkv")
-    nvfp4 = args.vfmt == "nvfp4"
-    p = vcattn.params(flags=vcattn.FLAGS_DEFAULT | (vcattn.VC_VFMT_NVFP4 if nvfp4 else 0))
+    nvfp4 = args.vfmt != "e4m3"
+    p = vcattn.params(flags=vcattn.FLAGS_DEFAULT | VFMT_FLAGS[args.vfmt])
     ws, ws_bytes = vcattn.workspace(B, H, N, p)
     out = torch.empty_like(q)
 
@@ -456,7 +465,8 @@ def run_ours(args):
         # four whole heads (every query row) on the image workload: about 10-15 s
         # of oracle work; on larger workloads a bounded number of rows per head
         rows = wl.N if wl.N <= 20000 else 2048
-        tf, cores, sample, _ = cpu_oracle_sample(wl, x, rows_per_head=rows, heads=(0, 1, 2, 3), nvfp4=nvfp4)
+        tf, cores, sample, _ = cpu_oracle_sample(wl, x, rows_per_head=rows, heads=(0, 1, 2, 3),
+                                                 extra_flags=VFMT_FLAGS[args.vfmt])
         cpu = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample}
     variants = None
     if args.workload == WORKLOAD and not nvfp4:
@@ -465,9 +475,9 @@ def run_ours(args):
 
     if rank == 0:
         metric = METRIC if (args.workload == WORKLOAD and not nvfp4) else \
-            f"vc_attn_fwd TFLOPS (4N²dH/t) on {args.workload}, V residual {args.vfmt}"
+            f"vc_attn_fwd TFLOPS (4N²dH/t) on {args.workload}, format {args.vfmt}"
         if nvfp4:
-            roof = exp2_roofline(B, H, N, attn_ms, clk.get("sm_mhz"))
+            roof = exp2_roofline(B, H, N, attn_ms, clk.get("sm_mhz"), ATTN_KERNEL[args.vfmt])
         else:
             roof = {"kernel": "k_vc_attn_fwd", "bound": "tensor", "achieved": attn_tflops,
                     "peak": fp8_peak, "unit": "TFLOP/s",
@@ -480,8 +490,7 @@ def run_ours(args):
             "metric": metric, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None,
-            "dtype": ("fp8_e4m3 QK, nvfp4 (e2m1 + e4m3 block-16 scales) PV, fp32 accumulate" if nvfp4
-                      else "fp8_e4m3 (fp32 accumulate)"),
+            "dtype": DTYPE[args.vfmt],
             "data": "synthetic",
             "pct_of_fp8_peak": 100.0 * (value / world) / fp8_peak,
             "config": {"workload": args.workload, "vfmt": args.vfmt, "B": B, "H": H, "N": N, "d": d, "k": p.k,
@@ -535,8 +544,9 @@ def main():
     ap.add_argument("--only-main", action="store_true",
                     help="warm-up + the timed main loop only (the small case profiler captures wrap)")
     ap.add_argument("--workload", default=WORKLOAD, help="synthetic workload name (bit_attention_diffusion_b200.synth)")
-    ap.add_argument("--vfmt", default="e4m3", choices=["e4m3", "nvfp4"],
-                    help="V residual format: the 8-bit path (default) or the NVFP4-residual variant")
+    ap.add_argument("--vfmt", default="e4m3", choices=sorted(VFMT_FLAGS),
+                    help="the 8-bit path (e4m3, default), the NVFP4-residual variant (nvfp4) or the "
+                         "full 4-bit path (nvfp4qk: Q, K in NVFP4 too)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -152,7 +152,9 @@ vc_status check_device() {
           cudaFuncSetAttribute(k_quantv4_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, QUANTV2_SMEM) !=
               cudaSuccess ||
           cudaFuncSetAttribute(k_vc_attn_fwd4, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(attn_fp4_smem_bytes())) != cudaSuccess ||
+                               static_cast<int>(attn_fp4_smem_bytes(false))) != cudaSuccess ||
+          cudaFuncSetAttribute(k_vc_attn_fwd44, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(attn_fp4_smem_bytes(true))) != cudaSuccess ||
           cudaFuncSetAttribute(k_kmeans_pass8, cudaFuncAttributeMaxDynamicSharedMemorySize, KMEANS8_SMEM) !=
               cudaSuccess) {
         ok_cache[dev] = 0;
@@ -169,7 +171,9 @@ vc_status check_params(const vc_params *p) {
   if (!(p->rho >= 0.0f && p->rho < 1.0f)) return VC_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.0f) || !std::isfinite(p->softmax_scale)) return VC_ERR_INVALID_ARG;
   if (p->expcast_bias < 8 || p->expcast_bias > 126) return VC_ERR_INVALID_ARG;
-  if (p->flags & ~(VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH | VC_WARMSTART | VC_VFMT_NVFP4)) return VC_ERR_INVALID_ARG;
+  if (p->flags & ~(VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH | VC_WARMSTART | VC_VFMT_NVFP4 | VC_QK_NVFP4))
+    return VC_ERR_INVALID_ARG;
+  if ((p->flags & VC_QK_NVFP4) && !(p->flags & VC_VFMT_NVFP4)) return VC_ERR_INVALID_ARG;  // 4-bit QK needs 4-bit PV
   return VC_OK;
 }
 
@@ -275,7 +279,10 @@ void launch_quant_qk(const Shape &sh, const Ws &w, const uint16_t *Q, const uint
   } else {
     cudaMemsetAsync(kbar, 0, static_cast<size_t>(sh.BH) * D * sizeof(float), s);  // no K smoothing: mean 0
   }
-  k_qk_quant<<<dim3(sh.Nb, sh.BH, 2), 256, 0, s>>>(Q, K, perm, kbar, sh.N, sh.Npad, q8, sq, k8, sk);
+  if (sh.flags & VC_QK_NVFP4)
+    k_qk_quant4<<<dim3(sh.Nb, sh.BH, 2), 256, 0, s>>>(Q, K, perm, kbar, sh.N, sh.Nb, q8, sq, k8, sk);
+  else
+    k_qk_quant<<<dim3(sh.Nb, sh.BH, 2), 256, 0, s>>>(Q, K, perm, kbar, sh.N, sh.Npad, q8, sq, k8, sk);
   count_launch();
 }
 
@@ -459,6 +466,7 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
   cudaEventDestroy(ev_join);
 
   const bool fp4 = (sh.flags & VC_VFMT_NVFP4) != 0;
+  const bool qk4 = (sh.flags & VC_QK_NVFP4) != 0;
   CUtensorMap tq, tk, tv, tmu, tdt;
   const uint64_t rows = static_cast<uint64_t>(sh.BH) * sh.Npad;
   bool ok = map2d(&tq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, rows, 128, 128) &&
@@ -488,11 +496,16 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
     ap.sk = sk;
     ap.vscale = vscale;
     ap.v4img = v8t;
+    ap.qimg = qk4 ? q8 : nullptr;
+    ap.kimg = qk4 ? k8 : nullptr;
     ap.rep_idx = rep_idx;
     ap.k8 = k8;
     ap.O = static_cast<uint16_t *>(O);
     ap.status = w.at<uint32_t>(w.L.status);
-    k_vc_attn_fwd4<<<dim3(sh.Nb, sh.BH), 352, attn_fp4_smem_bytes(), s>>>(tq, tk, tmu, tdt, ap);
+    if (qk4)
+      k_vc_attn_fwd44<<<dim3(sh.Nb, sh.BH), 352, attn_fp4_smem_bytes(true), s>>>(tq, tk, tmu, tdt, ap);
+    else
+      k_vc_attn_fwd4<<<dim3(sh.Nb, sh.BH), 352, attn_fp4_smem_bytes(false), s>>>(tq, tk, tmu, tdt, ap);
     count_launch();
     prof_mark(4, s);
     if (g_prof.on) ++g_prof.calls;

@@ -29,15 +29,20 @@
 //   - Each softmax thread turns its row's 128 scores into 8 blocks of 16:
 //     x = fma(acc, alpha/8, -F/8), p = 2^x, block scale sf = E4M3(448 * max p),
 //     codes E2M1(p * fl(2688 / sf)), the multipliers from a 128-entry table.
-//   - PV is one N = 160 product: B = the V tile's 128 channel rows plus 32 rows
+//   - PV is one N = 144 product: B = the V tile's 128 channel rows plus 16 rows
 //     E holding one row of ones (E2M1 1.0, scale 1.0) at row s in ring stage s,
 //     so the row sum l_t (sum of value(code) * sf over the tile, 2688 x the
 //     dequantized probabilities) lands in accumulator column 128 + t % 4, and
 //     every PV adds exact zeros to the other three.
+//   - The full 4-bit path (QK4) takes Q and K' as NVFP4 tile images of the
+//     same layout (rows = tokens, the K dimension = channels): QK^T is two
+//     K = 64 steps of kind::mxf4nvf4, the Q tile's scales copied into TMEM
+//     once, each K' tile's into one of two slots right before its product.
 // TMEM (512 columns x 128 lanes): S double buffer [0,256); O [256,384); row
-// sums [384,388) (the N = 160 accumulator spans [256,416)); V scales of ring
-// stage s at 416 + 16 s (+8 per K step; column +4 holds the constant scale of
-// E); P scales of slot i at 480 + 8 i (+4 per K step).
+// sums [384,388) (the N = 144 accumulator spans [256,400)); V scales of ring
+// stage s at 400 + 16 s (+8 per K step; column +4 holds the constant scale of
+// E); P scales of slot i at 464 + 8 i (+4 per K step); QK4: Q scales at 488,
+// K' scales of slot j at 496 + 8 j (+4 per K step).
 // O is kept in units of 2688 x p x v / g (g the channel's global scale, a power
 // of two): O_acc = sum P * value(code) * vsf + sum_t l_t * mean_t / g +
 // sum_R P' * delta / g, and the epilogue writes O = g_c * O_acc / l.
@@ -53,38 +58,57 @@ namespace vc {
 namespace {
 using namespace attn;
 
-constexpr int KS = 4;                                          // K ring stages
-constexpr int VS = 4;                                          // V ring stages
 constexpr uint32_t SZ_TILE8 = 128 * 128;                       // one 128x128 byte tile
 constexpr uint32_t SZ_V4 = 128 * 64;                           // E2M1 codes of one V tile
-constexpr uint32_t SZ_E4 = 32 * 64;                            // E rows
+constexpr uint32_t SZ_E4 = 16 * 64;                            // E rows
 constexpr uint32_t SZ_VSTAGE = V4_SF_BYTES + SZ_V4 + SZ_E4;    // [scales | codes | E]
 constexpr uint32_t SZ_PSLOT = V4_SF_BYTES + SZ_V4;             // [scales | codes]
 constexpr int NPSLOT = 3;
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = OFF_Q + SZ_TILE8;
-constexpr uint32_t OFF_V = OFF_K + KS * SZ_TILE8;
-constexpr uint32_t OFF_P = OFF_V + VS * SZ_VSTAGE;  // right after the V ring: the repair reuses both (48 KB)
-constexpr uint32_t OFF_AR = OFF_P + NPSLOT * SZ_PSLOT;
-constexpr uint32_t OFF_MU = OFF_AR + SZ_TILE8;
-constexpr uint32_t OFF_LB = OFF_MU + 2 * SZ_TILE8;
-constexpr uint32_t SMEM_USED = OFF_LB + 32 * 128 * 4;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // alignment slack
-static_assert(SZ_VSTAGE % 1024 == 0 && SZ_PSLOT % 1024 == 0 && OFF_V % 1024 == 0 && OFF_P % 1024 == 0 &&
-                  OFF_AR % 1024 == 0 && OFF_MU % 1024 == 0,
-              "tile alignment");
-static_assert(VS * SZ_VSTAGE + NPSLOT * SZ_PSLOT >= 3 * SZ_TILE8, "repair staging fits in the V ring and P slots");
-static_assert(SMEM_BYTES + 8192 <= 232448, "shared memory budget (dynamic + static)");
 
-constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_L = 384, TM_SFB = 416, TM_SFA = 480;
+// Shared memory and TMEM of the two QK^T formats. QK4: Q and K' as NVFP4 tile
+// images ([scales | codes], 9 KB) instead of 16 KB E4M3 tiles; their scales
+// take the last 24 TMEM columns.
+template <bool QK4>
+struct Lay {
+  static constexpr int KS = 4;  // K ring stages
+  static constexpr int VS = 4;  // V ring stages: stage t % 4 holds the ones row of row-sum column t % 4
+  static constexpr uint32_t SZ_QK = QK4 ? static_cast<uint32_t>(V4_TILE_BYTES) : SZ_TILE8;
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_K = OFF_Q + SZ_QK;
+  static constexpr uint32_t OFF_V = OFF_K + KS * SZ_QK;
+  static constexpr uint32_t OFF_P = OFF_V + VS * SZ_VSTAGE;  // right after the V ring: the repair reuses both
+  static constexpr uint32_t OFF_AR = OFF_P + NPSLOT * SZ_PSLOT;
+  static constexpr uint32_t OFF_MU = OFF_AR + SZ_TILE8;
+  static constexpr uint32_t OFF_LB = OFF_MU + 2 * SZ_TILE8;
+  static constexpr uint32_t SMEM_USED = OFF_LB + 32 * 128 * 4;
+  static constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // alignment slack
+  // TMEM columns: S [0,256), O and row sums [256,400), V scales 16 per stage,
+  // P scales 8 per slot, then (QK4) Q scales 8 and K scales 8 per slot (2)
+  static constexpr uint32_t TM_SFB = 400, TM_SFA = TM_SFB + 16 * VS, TM_QSF = TM_SFA + 8 * NPSLOT,
+                            TM_KSF = TM_QSF + 8;
+  static_assert(SZ_QK % 1024 == 0 && SZ_VSTAGE % 1024 == 0 && SZ_PSLOT % 1024 == 0 && OFF_V % 1024 == 0 &&
+                    OFF_P % 1024 == 0 && OFF_AR % 1024 == 0 && OFF_MU % 1024 == 0,
+                "tile alignment");
+  // repair staging: K rows (16 KB FP8 tile or 9 KB image) then 32 KB of bf16 P at +16 KB
+  static_assert(VS * SZ_VSTAGE + NPSLOT * SZ_PSLOT >= 3 * SZ_TILE8, "repair staging fits in the V ring and P slots");
+  static_assert(KS * SZ_QK >= 2 * SZ_TILE8, "the repair deltas fit in the K ring");
+  static_assert(SMEM_BYTES + 8192 <= 232448, "shared memory budget (dynamic + static)");
+  static_assert(!QK4 || TM_KSF + 16 <= 512, "TMEM columns");
+  static_assert(QK4 || TM_SFA + 8 * NPSLOT <= 512, "TMEM columns");
+};
+
+constexpr uint32_t TM_S0 = 0, TM_O = 256, TM_L = 384;
 constexpr int NPD = 8;  // PV completion barriers, indexed t % 8
 __device__ __forceinline__ uint32_t lcol_of(int t) { return TM_L + (t & 3); }
 constexpr uint32_t IDESC_QK = idesc_make(0, 0, 128, 128, false, false);  // E4M3 x E4M3 -> f32, N = 128
-constexpr uint32_t IDESC_PV = idesc_fp4_make(128, 160);                  // NVFP4 P x NVFP4 [V | E], N = 160
+constexpr uint32_t IDESC_QK4 = idesc_fp4_make(128, 128);                 // NVFP4 Q x NVFP4 K', N = 128
+constexpr uint32_t IDESC_PV = idesc_fp4_make(128, 144);                  // NVFP4 P x NVFP4 [V | E], N = 144
 constexpr uint32_t IDESC_BF = idesc_make(1, 1, 128, 128, false, false);  // bf16 x bf16 -> f32
 constexpr float P_GLOBAL = 2688.0f;  // 6 * 448: block maximum -> E2M1 6 at scale 448
 
+template <bool QK4>
 struct Bars {
+  static constexpr int KS = Lay<QK4>::KS, VS = Lay<QK4>::VS;
   uint64_t q, kfull[KS], kempty[KS], vfull[VS], vempty[VS], mufull[2], muempty[2];
   uint64_t sfull[2], sfree[2], pfull[4], mxr[2], pvdone[NPD], bk, lflush, wgdone, main, epi, rdone, repk, reps,
       repp, repdone, dt, fin;
@@ -165,12 +189,16 @@ __device__ __forceinline__ void p_block(const float *s, float al8, float nF8, fl
   w1 = e2m1x8(q + 8);
 }
 
-}  // namespace
 
-__global__ void __launch_bounds__(352, 1)
-    k_vc_attn_fwd4(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmMu, const __grid_constant__ CUtensorMap tmDT,
-                   const AttnFp4Params p) {
+// The body of both kernels; QK4 selects the format of QK^T.
+template <bool QK4>
+__device__ __forceinline__ void attn4_body(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmMu,
+                                           const CUtensorMap &tmDT, const AttnFp4Params &p) {
+  using L = Lay<QK4>;
+  constexpr int KS = L::KS, VS = L::VS;
+  constexpr uint32_t SZ_QK = L::SZ_QK, TM_SFB = L::TM_SFB, TM_SFA = L::TM_SFA;
+  constexpr uint32_t OFF_Q = L::OFF_Q, OFF_K = L::OFF_K, OFF_V = L::OFF_V, OFF_P = L::OFF_P, OFF_AR = L::OFF_AR,
+                     OFF_MU = L::OFF_MU, OFF_LB = L::OFF_LB;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = sm + OFF_Q;
@@ -180,7 +208,7 @@ __global__ void __launch_bounds__(352, 1)
   uint8_t *sAr = sm + OFF_AR;
   uint8_t *sMu = sm + OFF_MU;
   float *sLb = reinterpret_cast<float *>(sm + OFF_LB);  // [32 slots][128 rows]
-  __shared__ Bars bars;
+  __shared__ Bars<QK4> bars;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ float s_vscale[128];
@@ -225,10 +253,10 @@ __global__ void __launch_bounds__(352, 1)
   }
   if (warp >= 3) {
     const int t = threadIdx.x - 96;  // 0..255
-    // the E rows of the four ring stages (32 rows x 64 bytes after the codes,
+    // the E rows of the four ring stages (16 rows x 64 bytes after the codes,
     // 64-byte swizzle): zero except row s of stage s, all E2M1 1.0 (0x22 = two ones)
-    for (int i = t; i < VS * 128; i += 256) {
-      const int s = i >> 7, rr = (i >> 2) & 31, ch = i & 3;
+    for (int i = t; i < VS * 64; i += 256) {
+      const int s = i >> 6, rr = (i >> 2) & 15, ch = i & 3;
       const uint32_t v = rr == s ? 0x22222222u : 0u;
       *reinterpret_cast<uint4 *>(sV + s * SZ_VSTAGE + V4_SF_BYTES + SZ_V4 + sw64_off(rr, ch)) = make_uint4(v, v, v, v);
     }
@@ -263,15 +291,23 @@ __global__ void __launch_bounds__(352, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmDT);
-      mbar_arrive_expect_tx(&bars.q, SZ_TILE8);
-      tma_load_2d(sQ, &tmQ, &bars.q, 0, bh * p.Npad + qt * 128);
+      if constexpr (QK4) {
+        mbar_arrive_expect_tx(&bars.q, SZ_QK);
+        bulk_load(sQ, p.qimg + (static_cast<size_t>(bh) * T + qt) * SZ_QK, SZ_QK, &bars.q);
+      } else {
+        mbar_arrive_expect_tx(&bars.q, SZ_QK);
+        tma_load_2d(sQ, &tmQ, &bars.q, 0, bh * p.Npad + qt * 128);
+      }
       bool ok = true;
       for (int t = 0; t < T && ok; ++t) {
         const int s = t % KS;
         ok = wait(&bars.kempty[s], ((t / KS) & 1) ^ 1);
         if (!ok) break;
-        mbar_arrive_expect_tx(&bars.kfull[s], SZ_TILE8);
-        tma_load_2d(sK + s * SZ_TILE8, &tmK, &bars.kfull[s], 0, bh * p.Npad + t * 128);
+        mbar_arrive_expect_tx(&bars.kfull[s], SZ_QK);
+        if constexpr (QK4)
+          bulk_load(sK + s * SZ_QK, p.kimg + (static_cast<size_t>(bh) * T + t) * SZ_QK, SZ_QK, &bars.kfull[s]);
+        else
+          tma_load_2d(sK + s * SZ_QK, &tmK, &bars.kfull[s], 0, bh * p.Npad + t * 128);
       }
       if (ok && nrc > 0) {
         ok = wait(&bars.main, 0);
@@ -328,8 +364,26 @@ __global__ void __launch_bounds__(352, 1)
         tc_fence_after();
         if (elect_one()) {
           const uint32_t d = tmem + TM_S0 + (t & 1) * 128;
+          if constexpr (QK4) {
+            // K scales into slot t%2: its previous reader, QK(t-2), completed
+            // before S(t-2) was read out (the sfree wait above)
+            const uint8_t *kst = sK + s * SZ_QK;
+            const uint32_t ksf = tmem + L::TM_KSF + 8 * (t & 1);
+            if (t == 0) {  // the Q tile's scales, read by every QK^T of this CTA (same thread: in issue order)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma_f8_ss(d, dQ + KSTEP * kk, dK + TSTEP * s + KSTEP * kk, IDESC_QK, kk > 0);
+              for (int kk = 0; kk < 2; ++kk) tmem_cp_sf(tmem + L::TM_QSF + 4 * kk, sdesc_sf(smem_u32(sQ + 512 * kk)));
+            }
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) tmem_cp_sf(ksf + 4 * kk, sdesc_sf(smem_u32(kst + 512 * kk)));
+            const uint64_t dq = sdesc_sw64(smem_u32(sQ + V4_SF_BYTES)), dk = sdesc_sw64(smem_u32(kst + V4_SF_BYTES));
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              mma_fp4_ss(d, dq + 2 * kk, dk + 2 * kk, IDESC_QK4, tmem + L::TM_QSF + 4 * kk, ksf + 4 * kk, kk > 0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f8_ss(d, dQ + KSTEP * kk, dK + TSTEP * s + KSTEP * kk, IDESC_QK, kk > 0);
+          }
           mma_commit(&bars.kempty[s]);
           mma_commit(&bars.sfull[t & 1]);
         }
@@ -418,8 +472,21 @@ __global__ void __launch_bounds__(352, 1)
         if (!ok) break;
         tc_fence_after();
         if (elect_one()) {
+          if constexpr (QK4) {
+            // the staged K' rows: scales into K-scale slot 0 (every QK^T of
+            // the loop completed before `main`), codes after them
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tmem + TM_S0, dQ + KSTEP * kk, dR + KSTEP * kk, IDESC_QK, kk > 0);
+            for (int kk = 0; kk < 2; ++kk) tmem_cp_sf(tmem + L::TM_KSF + 4 * kk, sdesc_sf(smem_u32(sV + 512 * kk)));
+            const uint64_t dq = sdesc_sw64(smem_u32(sQ + V4_SF_BYTES)), dk = sdesc_sw64(smem_u32(sV + V4_SF_BYTES));
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              mma_fp4_ss(tmem + TM_S0, dq + 2 * kk, dk + 2 * kk, IDESC_QK4, tmem + L::TM_QSF + 4 * kk,
+                         tmem + L::TM_KSF + 4 * kk, kk > 0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f8_ss(tmem + TM_S0, dQ + KSTEP * kk, dR + KSTEP * kk, IDESC_QK, kk > 0);
+          }
           mma_commit(&bars.reps);
         }
         __syncwarp();
@@ -701,20 +768,43 @@ __global__ void __launch_bounds__(352, 1)
       }
       const int i = rc * 128 + r;
       const int nval = min(128, p.R - rc * 128);
-      uint4 krow[8];
       float al = 0.0f;
-      if (i < p.R) {
-        const int pos = p.rep_idx[static_cast<size_t>(bh) * p.R + i];
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.k8 + (static_cast<size_t>(bh) * p.Npad + pos) * 128);
+      if constexpr (QK4) {
+        // row pos % 128 of K' tile pos / 128: 64 bytes of codes and 8 scale
+        // bytes, staged as row r of an image (rows past R: codes and scales 0)
+        uint4 krow[4];
+        uint32_t ksc[2] = {0u, 0u};
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) krow[ch] = src[ch];
-        al = __fmul_rn(__fmul_rn(sqs, skh[pos >> 7]), p.kappa);
+        for (int ch = 0; ch < 4; ++ch) krow[ch] = make_uint4(0u, 0u, 0u, 0u);
+        if (i < p.R) {
+          const int pos = p.rep_idx[static_cast<size_t>(bh) * p.R + i];
+          const uint8_t *img = p.kimg + (static_cast<size_t>(bh) * T + (pos >> 7)) * SZ_QK;
+          const int rr = pos & 127;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) krow[ch] = *reinterpret_cast<const uint4 *>(img + V4_SF_BYTES + sw64_off(rr, ch));
+#pragma unroll
+          for (int h = 0; h < 2; ++h) ksc[h] = *reinterpret_cast<const uint32_t *>(img + v4_sf_off(rr, 4 * h));
+          al = __fmul_rn(__fmul_rn(sqs, skh[pos >> 7]), p.kappa);
+        }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) *reinterpret_cast<uint4 *>(sV + V4_SF_BYTES + sw64_off(r, ch)) = krow[ch];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) *reinterpret_cast<uint32_t *>(sV + v4_sf_off(r, 4 * h)) = ksc[h];
       } else {
+        uint4 krow[8];
+        if (i < p.R) {
+          const int pos = p.rep_idx[static_cast<size_t>(bh) * p.R + i];
+          const uint4 *src = reinterpret_cast<const uint4 *>(p.k8 + (static_cast<size_t>(bh) * p.Npad + pos) * 128);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) krow[ch] = make_uint4(0u, 0u, 0u, 0u);
+          for (int ch = 0; ch < 8; ++ch) krow[ch] = src[ch];
+          al = __fmul_rn(__fmul_rn(sqs, skh[pos >> 7]), p.kappa);
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) krow[ch] = make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4 *>(sV + sw128_off(r, ch)) = krow[ch];
       }
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4 *>(sV + sw128_off(r, ch)) = krow[ch];
       s_alphaR[r] = __fmul_rn(al, 0.125f);
       fence_proxy_async_smem();
       tc_fence_before();
@@ -792,6 +882,22 @@ __global__ void __launch_bounds__(352, 1)
   }
 }
 
-uint32_t attn_fp4_smem_bytes() { return SMEM_BYTES; }
+}  // namespace
+
+__global__ void __launch_bounds__(352, 1)
+    k_vc_attn_fwd4(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmMu, const __grid_constant__ CUtensorMap tmDT,
+                   const AttnFp4Params p) {
+  attn4_body<false>(tmQ, tmK, tmMu, tmDT, p);
+}
+
+__global__ void __launch_bounds__(352, 1)
+    k_vc_attn_fwd44(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmMu, const __grid_constant__ CUtensorMap tmDT,
+                    const AttnFp4Params p) {
+  attn4_body<true>(tmQ, tmK, tmMu, tmDT, p);
+}
+
+uint32_t attn_fp4_smem_bytes(bool qk4) { return qk4 ? Lay<true>::SMEM_BYTES : Lay<false>::SMEM_BYTES; }
 
 }  // namespace vc

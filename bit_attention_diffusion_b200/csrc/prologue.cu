@@ -526,6 +526,95 @@ __global__ void __launch_bounds__(256) k_qk_quant(const uint16_t *__restrict__ Q
   if (tid == 0) (z == 0 ? sq : sk)[static_cast<size_t>(bh) * (Npad / TILE) + t] = scale;
 }
 
+// NVFP4 block quantization of the full 4-bit path, same grid and row mapping
+// as k_qk_quant (z = 0: Q rows in original order; z = 1: K rows through perm
+// minus the channel mean). Per block the power-of-two global scale g = 2^e,
+// the least with amax <= 2688 * g (g = 1 for an all-zero block); per row and
+// 16 channels sf = E4M3(fp32(b * 2^-e) / 6) of the block maximum b; codes
+// E2M1(fp32(x * 2^-e) * fp32(1/sf)), 0 where sf is 0 and in rows past N. The
+// tile image: scales, then rows of codes in the 64-byte swizzle (the layout
+// of the V tile images, rows = tokens, the K dimension = channels).
+__global__ void __launch_bounds__(256) k_qk_quant4(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
+                                                   const int32_t *__restrict__ perm, const float *__restrict__ kbar,
+                                                   int N, int Nb, uint8_t *__restrict__ q4img, float *__restrict__ gq,
+                                                   uint8_t *__restrict__ k4img, float *__restrict__ gk) {
+  __shared__ float wmax[8];
+  const int t = blockIdx.x, bh = blockIdx.y, z = blockIdx.z;
+  const int tid = threadIdx.x, g = tid >> 4, c = tid & 15;
+  const int cnt = min(TILE, N - t * TILE);
+  const uint16_t *src = (z == 0 ? Q : K) + static_cast<size_t>(bh) * N * D + 8 * c;
+  int row[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int rr = g + 16 * i, pos = t * TILE + rr;
+    row[i] = rr < cnt ? ((z == 1 && perm != nullptr) ? __ldg(perm + static_cast<size_t>(bh) * N + pos) : pos) : -1;
+  }
+  uint4 w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    w[i] = row[i] >= 0 ? __ldg(reinterpret_cast<const uint4 *>(src + static_cast<size_t>(row[i]) * D))
+                       : make_uint4(0u, 0u, 0u, 0u);
+  float kb[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (z == 1) {
+    const float4 k0 = *reinterpret_cast<const float4 *>(kbar + static_cast<size_t>(bh) * D + 8 * c);
+    const float4 k1 = *reinterpret_cast<const float4 *>(kbar + static_cast<size_t>(bh) * D + 8 * c + 4);
+    kb[0] = k0.x; kb[1] = k0.y; kb[2] = k0.z; kb[3] = k0.w;
+    kb[4] = k1.x; kb[5] = k1.y; kb[6] = k1.z; kb[7] = k1.w;
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (row[i] < 0) continue;  // rows past N do not enter the block's amax
+    float x[8];
+    bf16x8(w[i], x);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(z == 1 ? __fsub_rn(x[j], kb[j]) : x[j]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if ((tid & 31) == 0) wmax[tid >> 5] = amax;
+  __syncthreads();
+  amax = wmax[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, wmax[i]);
+  int e = 0;
+  if (amax > 0.0f) {
+    int E;
+    const float f = frexpf(amax, &E);  // amax = f * 2^E, f in [0.5, 1); 2688 = 0.65625 * 2^12
+    e = (f > 0.65625f) ? E - 11 : E - 12;
+  }
+  // x * 2^-e in two exact steps when 2^-e is past the binary32 range (tiny blocks)
+  const int eh = -e > 126 ? 64 : 0;
+  const float m_hi = ldexpf(1.0f, eh), m_lo = ldexpf(1.0f, -e - eh);
+  uint8_t *img = (z == 0 ? q4img : k4img) + (static_cast<size_t>(bh) * Nb + t) * V4_TILE_BYTES;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = g + 16 * i;
+    float x[8], y[8];
+    bf16x8(w[i], x);
+    float b = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      y[j] = __fmul_rn(__fmul_rn(z == 1 ? __fsub_rn(x[j], kb[j]) : x[j], m_hi), m_lo);
+      b = fmaxf(b, fabsf(y[j]));
+    }
+    b = fmaxf(b, __shfl_xor_sync(0xFFFFFFFFu, b, 1));  // the 16-channel block of threads c, c^1
+    uint32_t sc = e4m3x2(__fdiv_rn(b, 6.0f), 0.0f) & 0xFFu;
+    if (row[i] < 0) sc = 0u;
+    const float sfv = e4m3x2_value(static_cast<uint16_t>(sc)).x;
+    uint32_t codes = 0u;
+    if (sfv != 0.0f) {
+      const float rcp = __frcp_rn(sfv);
+#pragma unroll
+      for (int j = 0; j < 8; j += 2)
+        codes |= e2m1x2(__fmul_rn(y[j], rcp), __fmul_rn(y[j + 1], rcp)) << (4 * j);
+    }
+    *reinterpret_cast<uint32_t *>(img + V4_SF_BYTES + sw64_off(r, c >> 2) + 4 * (c & 3)) = codes;
+    if ((c & 1) == 0) img[v4_sf_off(r, c >> 1)] = static_cast<uint8_t>(sc);
+  }
+  if (tid == 0) (z == 0 ? gq : gk)[static_cast<size_t>(bh) * Nb + t] = ldexpf(1.0f, e);
+}
+
 // ============================================================== V demean + quantization
 // The block's 128 rows (gathered through perm) are copied to shared memory
 // with cp.async, row stride 272 bytes: 16-byte reads of one row per thread
@@ -766,6 +855,8 @@ __global__ void __launch_bounds__(256) k_quantv4_pass2(const uint16_t *__restric
           const float r1 = __fsub_rn(x[j + 1], smu[c + 1]);
           codes = e2m1x2(__fmul_rn(__fmul_rn(r0, smult[c]), srcp[jb][c]),
                          __fmul_rn(__fmul_rn(r1, smult[c + 1]), srcp[jb][c + 1]));
+          if (ssfv[jb][c] == 0.0f) codes &= 0xF0u;  // no scale: code 0 (not the -0 of a negative residual)
+          if (ssfv[jb][c + 1] == 0.0f) codes &= 0x0Fu;
           const float2 dq = e2m1x2_value(codes);
           const float e0 = __fsub_rn(r0, __fmul_rn(__fmul_rn(dq.x, ssfv[jb][c]), sscale[c]));
           const float e1 = __fsub_rn(r1, __fmul_rn(__fmul_rn(dq.y, ssfv[jb][c + 1]), sscale[c + 1]));

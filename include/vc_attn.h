@@ -64,6 +64,17 @@ typedef enum {
  * PV runs on the block-scaled FP4 tensor cores. QK^T stays FP8; the expcast
  * bias is not used. vc_attn_quant_v and vc_attn_fwd honour it. */
 #define VC_VFMT_NVFP4 32u
+/* The full 4-bit path ([VCA] "Por que a atenção é o gargalo": low-precision
+ * tensor cores for both products; "Benchmarks": the 4-bit V-Smooth kernel
+ * against SageAttention3): with VC_VFMT_NVFP4, Q and K' are NVFP4 too and
+ * QK^T runs on the block-scaled FP4 tensor cores. Per 128-row block of Q
+ * (original order) or K' (permuted order, K smoothing applied) a power-of-two
+ * global scale g, the least with amax <= 2688 * g (1 for an all-zero block);
+ * per row and 16 consecutive channels an E4M3 scale sf = E4M3(fp32(b / g) / 6)
+ * of the block maximum b; codes E2M1(fp32(x / g) * fp32(1 / sf)) (0 where sf
+ * is 0). The score scale is g_q * g_k * kappa. Without VC_VFMT_NVFP4 the
+ * flag is invalid. vc_attn_quant_qk and vc_attn_fwd honour it. */
+#define VC_QK_NVFP4 64u
 
 typedef struct {
   int k;             /* k-means clusters, 1..64 (default 8) */
@@ -72,7 +83,7 @@ typedef struct {
   float softmax_scale; /* 0 => 1/sqrt(d) */
   int expcast_bias;  /* C: the running row maximum maps to byte C, 8..126 (default 120) */
   unsigned flags;    /* VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH (default), optionally VC_WARMSTART,
-                        VC_VFMT_NVFP4 */
+                        VC_VFMT_NVFP4, VC_QK_NVFP4 (with VC_VFMT_NVFP4) */
 } vc_params;
 
 /* Fill the defaults listed above. */
@@ -146,6 +157,13 @@ size_t vc_attn_cluster_noalloc_max_bytes(void);
  *   Q, K  bf16 [B,H,N,d] in;  perm int32 [B,H,N] in (NULL = identity)
  *   q8, k8 uint8 [B,H,Npad,d] out (E4M3 codes; padding rows are 0)
  *   sq, sk fp32 [B,H,Nb] out (block scales)
+ * With VC_QK_NVFP4 (see there) the same buffers receive NVFP4 tile images
+ * instead, one per 128-row block, 9216 bytes each at byte (b*H+h)*Nb*9216 +
+ * t*9216 (the first 9/16 of the buffer): the E4M3 scales (byte 512*(j/4) +
+ * 16*(r%32) + 4*(r/32) + j%4 for row r and 16-channel block j), then the E2M1
+ * codes, rows of 64 bytes (channel 2i in the low nibble of byte i) in the
+ * 64-byte swizzle of the V tile images; rows past N are 0. sq, sk receive the
+ * power-of-two global scales g.
  */
 vc_status vc_attn_quant_qk(const void *Q, const void *K, const int32_t *perm, int B, int H, int N, int d,
                            const vc_params *p, uint8_t *q8, float *sq, uint8_t *k8, float *sk, void *ws,

@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(256) k_kmeans_pass8(const uint16_t *__restrict
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     if (tok < cnt) {
       const uint8_t *row = buf + tok * KM8_ROW_BYTES;
-#pragma unroll 2
+#pragma unroll 4
       for (int g8 = 0; g8 < 16; ++g8) {
         const uint4 w = *reinterpret_cast<const uint4 *>(row + 16 * g8);
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -325,17 +325,23 @@ __global__ void __launch_bounds__(256) k_kmeans_pass8(const uint16_t *__restrict
   __syncthreads();
   if (tid == 0) s_last = (atomicAdd(&counter[bh], 1u) == static_cast<unsigned>(nblk - 1));
   __syncthreads();
-  if (!s_last || tid >= 128) return;
+  if (!s_last) return;
   __threadfence();
-  for (int j = 0; j < k; ++j) {
-    double sum = 0.0;
-    long long n = 0;
+  // every (cluster, channel) of the head at once: thread (c = tid % 128,
+  // cluster parity tid / 128) takes clusters j = parity, parity + 2, ...; the
+  // partial sums are added in block order
+  {
+    const int c = tid & 127;
+    for (int j = tid >> 7; j < k; j += 2) {
+      double sum = 0.0;
+      long long n = 0;
 #pragma unroll 16
-    for (int b = 0; b < nblk; ++b) {  // loads batched by the unroll
-      sum += __ldcg(psum + ((static_cast<size_t>(bh) * nblk + b) * k + j) * D + tid);
-      n += __ldcg(pcnt + (static_cast<size_t>(bh) * nblk + b) * k + j);
+      for (int b = 0; b < nblk; ++b) {  // loads batched by the unroll
+        sum += __ldcg(psum + ((static_cast<size_t>(bh) * nblk + b) * k + j) * D + c);
+        n += __ldcg(pcnt + (static_cast<size_t>(bh) * nblk + b) * k + j);
+      }
+      if (n > 0) cent_h[j * D + c] = static_cast<float>(sum / static_cast<double>(n));
     }
-    if (n > 0) cent_h[j * D + tid] = static_cast<float>(sum / static_cast<double>(n));
   }
   if (tid == 0) counter[bh] = 0u;
 }
@@ -707,7 +713,10 @@ __global__ void __launch_bounds__(256) k_quantv_pass1(const uint16_t *__restrict
 // bf16 block means pre-divided by the channel scale for the in-kernel restore
 // (mut2[bh][chunk][c][0..63]: slots 0..31 and 32..63 both hold tile
 // chunk*32 + slot; unused slots of the last chunk are zero). Thread r < 128
-// owns token r: its error is fmaf-accumulated in channel order.
+// owns token r: its error is fmaf-accumulated in channel order; the residual,
+// scaling and dequantization of a channel pair are packed f32x2 operations
+// (each lane rounds as the scalar one; differences are sums with negated
+// operands, exactly the same values).
 __global__ void __launch_bounds__(256) k_quantv_pass2(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
                                                       int N, int Nb, int Npad, int nch32,
                                                       const uint16_t *__restrict__ vmean,
@@ -717,17 +726,17 @@ __global__ void __launch_bounds__(256) k_quantv_pass2(const uint16_t *__restrict
   extern __shared__ __align__(16) uint8_t dsm[];
   uint8_t *sv = dsm;                            // 128 rows x 272 bytes
   uint8_t *codeT = dsm + TILE * VQ_ROW_BYTES;   // 128 channels x 144 bytes
-  __shared__ __align__(16) float smu[D], smult[D], sscale[D];
+  __shared__ __align__(16) float snmu[D], smult[D], snscale[D];  // -mean, 2^-e, -scale
   const int t = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
   const int p0 = t * TILE, cnt = min(TILE, N - p0);
   gather_tile(sv, V + static_cast<size_t>(bh) * N * D, perm ? perm + static_cast<size_t>(bh) * N : nullptr, p0, cnt);
   if (tid < 128) {
     const int c = tid;
     const uint16_t mu = vmean[(static_cast<size_t>(bh) * Nb + t) * D + c];
-    smu[c] = bf16_to_f32(mu);
+    snmu[c] = -bf16_to_f32(mu);
     const int e = vexpo[static_cast<size_t>(bh) * D + c];
     smult[c] = ldexpf(1.0f, -e);
-    sscale[c] = vscale[static_cast<size_t>(bh) * D + c];
+    snscale[c] = -vscale[static_cast<size_t>(bh) * D + c];
     // block mean / scale for the restore MMA (exact: bf16 divided by a power of two)
     const uint16_t ms = f32_to_bf16_rn(__fmul_rn(bf16_to_f32(mu), ldexpf(1.0f, -e)));
     const int ch = t / CHUNK32, slot = t % CHUNK32;
@@ -754,14 +763,13 @@ __global__ void __launch_bounds__(256) k_quantv_pass2(const uint16_t *__restrict
         const int c = c0 + j;
         uint16_t codes = 0;
         if (r < cnt) {
-          const float r0 = __fsub_rn(x[j], smu[c]);
-          const float r1 = __fsub_rn(x[j + 1], smu[c + 1]);
-          codes = e4m3x2(__fmul_rn(r0, smult[c]), __fmul_rn(r1, smult[c + 1]));
-          const float2 dq = e4m3x2_value(codes);
-          const float e0 = __fsub_rn(r0, __fmul_rn(dq.x, sscale[c]));
-          const float e1 = __fsub_rn(r1, __fmul_rn(dq.y, sscale[c + 1]));
-          acc = __fmaf_rn(e0, e0, acc);
-          acc = __fmaf_rn(e1, e1, acc);
+          const float2 rr = __fadd2_rn(make_float2(x[j], x[j + 1]), *reinterpret_cast<const float2 *>(&snmu[c]));
+          const float2 sr = __fmul2_rn(rr, *reinterpret_cast<const float2 *>(&smult[c]));
+          codes = e4m3x2(sr.x, sr.y);
+          const float2 nd = __fmul2_rn(e4m3x2_value(codes), *reinterpret_cast<const float2 *>(&snscale[c]));
+          const float2 ee = __fadd2_rn(rr, nd);
+          acc = __fmaf_rn(ee.x, ee.x, acc);
+          acc = __fmaf_rn(ee.y, ee.y, acc);
         }
         codeT[c * 144 + r] = static_cast<uint8_t>(codes & 0xFF);
         codeT[(c + 1) * 144 + r] = static_cast<uint8_t>(codes >> 8);

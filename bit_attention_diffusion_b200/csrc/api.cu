@@ -267,22 +267,28 @@ void launch_cluster(const Shape &sh, const Ws &w, const uint16_t *V, int32_t *pe
   count_launch();
 }
 
+// parts: QK_Q = the K channel means and Q (no permutation needed), QK_K = K'
+// through perm (after QK_Q on the same stream); both in one launch for QK_QK.
+enum { QK_Q = 1, QK_K = 2, QK_QK = 3 };
 void launch_quant_qk(const Shape &sh, const Ws &w, const uint16_t *Q, const uint16_t *K, const int32_t *perm,
-                     uint8_t *q8, float *sq, uint8_t *k8, float *sk, cudaStream_t s) {
+                     uint8_t *q8, float *sq, uint8_t *k8, float *sk, cudaStream_t s, int parts = QK_QK) {
   const int ks = (sh.flags & VC_KSMOOTH) ? 1 : 0;
   double *part = w.at<double>(w.L.kbar_part);
   float *kbar = w.at<float>(w.L.kbar);
-  if (ks) {
+  if (!(parts & QK_Q)) {
+    // K' alone: the means were computed by an earlier QK_Q launch on this stream
+  } else if (ks) {
     k_kbar<<<dim3(sh.kb_nchunk, sh.BH), 256, 0, s>>>(K, sh.N, sh.kb_nchunk, 1, part, w.at<unsigned>(w.L.kb_counter),
                                                      kbar);
     count_launch();
   } else {
     cudaMemsetAsync(kbar, 0, static_cast<size_t>(sh.BH) * D * sizeof(float), s);  // no K smoothing: mean 0
   }
+  const int zbase = (parts & QK_Q) ? 0 : 1, nz = parts == QK_QK ? 2 : 1;
   if (sh.flags & VC_QK_NVFP4)
-    k_qk_quant4<<<dim3(sh.Nb, sh.BH, 2), 256, 0, s>>>(Q, K, perm, kbar, sh.N, sh.Nb, q8, sq, k8, sk);
+    k_qk_quant4<<<dim3(sh.Nb, sh.BH, nz), 256, 0, s>>>(Q, K, perm, kbar, sh.N, sh.Nb, zbase, q8, sq, k8, sk);
   else
-    k_qk_quant<<<dim3(sh.Nb, sh.BH, 2), 256, 0, s>>>(Q, K, perm, kbar, sh.N, sh.Npad, q8, sq, k8, sk);
+    k_qk_quant<<<dim3(sh.Nb, sh.BH, nz), 256, 0, s>>>(Q, K, perm, kbar, sh.N, sh.Npad, zbase, q8, sq, k8, sk);
   count_launch();
 }
 
@@ -435,35 +441,46 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
                  *Vh = static_cast<const uint16_t *>(V);
   if ((st = clear_small(w, s)) != VC_OK) return st;
   prof_mark(0, s);
+  uint8_t *q8 = w.at<uint8_t>(w.L.q8), *k8 = w.at<uint8_t>(w.L.k8), *v8t = w.at<uint8_t>(w.L.v8t);
+  float *sq = w.at<float>(w.L.sq), *sk = w.at<float>(w.L.sk), *vscale = w.at<float>(w.L.vscale);
+  int32_t *rep_idx = w.at<int32_t>(w.L.rep_idx);
+  // Q/K quantization on a side stream (disjoint workspace regions). When this
+  // call clusters, the K channel means and Q (which do not depend on the
+  // permutation) start with the call, concurrent with the clustering, and K'
+  // follows once the permutation is known; otherwise Q and K' are one launch.
+  // Either way they run concurrently with the V passes, and the attention
+  // kernel waits for both streams. Per-call events, released once the work
+  // completes.
+  const bool clusters = !perm && (sh.flags & VC_VSMOOTH);
+  cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};  // fork, permutation ready, join
+  cudaStream_t side = side_stream();
+  bool evok = side != nullptr;
+  for (int i = 0; i < 3 && evok; ++i) evok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+  if (!evok) {
+    for (cudaEvent_t e : ev)
+      if (e) cudaEventDestroy(e);
+    return VC_ERR_CUDA;
+  }
+  cudaEventRecord(ev[0], s);
+  cudaStreamWaitEvent(side, ev[0], 0);
+  if (clusters) launch_quant_qk(sh, w, Qh, Kh, nullptr, q8, sq, k8, sk, side, QK_Q);
   const int32_t *pm = perm;
-  if (!pm && (sh.flags & VC_VSMOOTH)) {
+  if (clusters) {
     Shape cold = sh;  // vc_attn_fwd has no centroid input: always the default start
     cold.flags &= ~VC_WARMSTART;
     launch_cluster(cold, w, Vh, w.at<int32_t>(w.L.perm), w.at<float>(w.L.cent), s);
     pm = w.at<int32_t>(w.L.perm);
   }
   prof_mark(1, s);
-  uint8_t *q8 = w.at<uint8_t>(w.L.q8), *k8 = w.at<uint8_t>(w.L.k8), *v8t = w.at<uint8_t>(w.L.v8t);
-  float *sq = w.at<float>(w.L.sq), *sk = w.at<float>(w.L.sk), *vscale = w.at<float>(w.L.vscale);
-  int32_t *rep_idx = w.at<int32_t>(w.L.rep_idx);
-  // Q/K quantization on a side stream, concurrent with the V passes on the
-  // caller's stream (they touch disjoint workspace regions); the attention
-  // kernel waits for both. Per-call events, released once the work completes.
-  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
-  cudaStream_t side = side_stream();
-  if (!side || cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) != cudaSuccess)
-    return VC_ERR_CUDA;
-  cudaEventRecord(ev_fork, s);
-  cudaStreamWaitEvent(side, ev_fork, 0);
-  launch_quant_qk(sh, w, Qh, Kh, pm, q8, sq, k8, sk, side);
-  cudaEventRecord(ev_join, side);
+  cudaEventRecord(ev[1], s);
+  cudaStreamWaitEvent(side, ev[1], 0);
+  launch_quant_qk(sh, w, Qh, Kh, pm, q8, sq, k8, sk, side, clusters ? QK_K : QK_QK);
+  cudaEventRecord(ev[2], side);
   launch_quant_v(sh, w, Vh, pm, v8t, vscale, w.at<uint16_t>(w.L.vmean), rep_idx, w.at<uint16_t>(w.L.rep_delta), s);
   prof_mark(2, s);
-  cudaStreamWaitEvent(s, ev_join, 0);
+  cudaStreamWaitEvent(s, ev[2], 0);
   prof_mark(3, s);
-  cudaEventDestroy(ev_fork);
-  cudaEventDestroy(ev_join);
+  for (cudaEvent_t e : ev) cudaEventDestroy(e);
 
   const bool fp4 = (sh.flags & VC_VFMT_NVFP4) != 0;
   const bool qk4 = (sh.flags & VC_QK_NVFP4) != 0;

@@ -467,14 +467,16 @@ __global__ void __launch_bounds__(256) k_kbar(const uint16_t *__restrict__ K, in
 }
 
 // Block quantization: z = 0 -> Q rows [128t, 128t+128) in original order;
-// z = 1 -> K rows perm[128t + r] minus the channel mean. scale = amax/448,
+// z = 1 -> K rows perm[128t + r] minus the channel mean (z = blockIdx.z +
+// zbase: one launch may take both, or Q and K separately). scale = amax/448,
 // codes = E4M3(x * (448/amax)); rows past N get code 0.
 __global__ void __launch_bounds__(256) k_qk_quant(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                                                   const int32_t *__restrict__ perm, const float *__restrict__ kbar,
-                                                  int N, int Npad, uint8_t *__restrict__ q8, float *__restrict__ sq,
-                                                  uint8_t *__restrict__ k8, float *__restrict__ sk) {
+                                                  int N, int Npad, int zbase, uint8_t *__restrict__ q8,
+                                                  float *__restrict__ sq, uint8_t *__restrict__ k8,
+                                                  float *__restrict__ sk) {
   __shared__ float wmax[8];
-  const int t = blockIdx.x, bh = blockIdx.y, z = blockIdx.z;
+  const int t = blockIdx.x, bh = blockIdx.y, z = blockIdx.z + zbase;
   const int tid = threadIdx.x, g = tid >> 4, c = tid & 15;
   const int cnt = min(TILE, N - t * TILE);
   const uint16_t *src = (z == 0 ? Q : K) + static_cast<size_t>(bh) * N * D + 8 * c;
@@ -542,10 +544,11 @@ __global__ void __launch_bounds__(256) k_qk_quant(const uint16_t *__restrict__ Q
 // of the V tile images, rows = tokens, the K dimension = channels).
 __global__ void __launch_bounds__(256) k_qk_quant4(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                                                    const int32_t *__restrict__ perm, const float *__restrict__ kbar,
-                                                   int N, int Nb, uint8_t *__restrict__ q4img, float *__restrict__ gq,
-                                                   uint8_t *__restrict__ k4img, float *__restrict__ gk) {
+                                                   int N, int Nb, int zbase, uint8_t *__restrict__ q4img,
+                                                   float *__restrict__ gq, uint8_t *__restrict__ k4img,
+                                                   float *__restrict__ gk) {
   __shared__ float wmax[8];
-  const int t = blockIdx.x, bh = blockIdx.y, z = blockIdx.z;
+  const int t = blockIdx.x, bh = blockIdx.y, z = blockIdx.z + zbase;
   const int tid = threadIdx.x, g = tid >> 4, c = tid & 15;
   const int cnt = min(TILE, N - t * TILE);
   const uint16_t *src = (z == 0 ? Q : K) + static_cast<size_t>(bh) * N * D + 8 * c;

@@ -13,9 +13,9 @@ __global__ void k_perm_sort(const int32_t *labels, int N, int k, int32_t *perm);
 __global__ void k_kbar(const uint16_t *K, int N, int nchunk, int ksmooth, double *part, unsigned *counter,
                        float *kbar);
 __global__ void k_qk_quant(const uint16_t *Q, const uint16_t *K, const int32_t *perm, const float *kbar, int N,
-                           int Npad, uint8_t *q8, float *sq, uint8_t *k8, float *sk);
+                           int Npad, int zbase, uint8_t *q8, float *sq, uint8_t *k8, float *sk);
 __global__ void k_qk_quant4(const uint16_t *Q, const uint16_t *K, const int32_t *perm, const float *kbar, int N,
-                            int Nb, uint8_t *q4img, float *gq, uint8_t *k4img, float *gk);
+                            int Nb, int zbase, uint8_t *q4img, float *gq, uint8_t *k4img, float *gk);
 __global__ void k_quantv_pass1(const uint16_t *V, const int32_t *perm, int N, int Nb, int demean, int fp4, uint16_t *vmean,
                                float *amax_part, float *vscale, int *vexpo, unsigned *counter);
 __global__ void k_quantv_pass2(const uint16_t *V, const int32_t *perm, int N, int Nb, int Npad, int nch32,

@@ -223,9 +223,12 @@ vc_status vc_attn_quant_v(const void *V, const int32_t *perm, int B, int H, int 
  * Restore) on the tensor cores in bf16; repair adds p * delta for the listed
  * tokens; O = scale_c * acc / l.
  * Q/K quantization runs on an internal non-blocking stream of the library
- * (one per device, created on first use) between two per-call events, so it
- * overlaps the V passes; the call stays stream-ordered with respect to the
- * caller's stream and can be captured into a CUDA graph.
+ * (one per device, created on first use), ordered by per-call events: when
+ * the call clusters, the K channel means and Q start with the call (they do
+ * not depend on the permutation) and K' follows the clustering; otherwise Q
+ * and K' are one launch. Either way it overlaps the V passes; the call stays
+ * stream-ordered with respect to the caller's stream and can be captured
+ * into a CUDA graph.
  * With VC_VFMT_NVFP4 (the 4-bit variant): the same frames, then per 16 keys
  * x = fma(acc, alpha/8, -F/8), p = 2^x, block scale sf = E4M3(448 * max p),
  * codes E2M1(p * fl(2688/sf)); O += P V4 on the block-scaled FP4 tensor cores
@@ -310,10 +313,11 @@ vc_status vc_attn_wait_selftest(void *ws, long long limit_cycles, void *stream);
  * once per device when profiling is first switched on, and switching it on
  * again restarts the count. vc_attn_profile_read() waits for the recorded
  * calls and writes their mean phase durations in milliseconds to ms[0..3]:
- * clustering (0 when a permutation was passed); V quantization + repair
- * selection (on the caller's stream, while Q/K quantization runs on an
- * internal side stream); the further wait for Q/K quantization (0 when it
- * finished first); and the fused attention kernel. Returns
+ * clustering (0 when a permutation was passed; Q quantization may run
+ * beside it on the internal side stream); V quantization + repair selection
+ * (on the caller's stream, while K' quantization runs on the side stream);
+ * the further wait for Q/K quantization (0 when it finished first); and the
+ * fused attention kernel. Returns
  * the number of values written (4), or 0 if nothing was recorded or
  * max_n < 4. */
 vc_status vc_attn_profile(int on);

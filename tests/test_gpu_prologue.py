@@ -42,6 +42,49 @@ def test_cluster_bit_exact(torch, B, H, N, k, iters):
             assert np.array_equal(cent[b, h].view(np.uint32), c_o.view(np.uint32)), (b, h)
 
 
+def _tie_inputs(N=600, seed=5):
+    """V with exact and near ties for the first assignment (initial centroids
+    are the tokens j*N/8: 0, 75, 150, ...): centroids 0 and 1 differ only in
+    channel 0 (0 and 2); tokens 1-74 are token 0 with channel 0 = 1
+    (equidistant: ties go to cluster 0), tokens 76-149 the same with channel
+    0 one bf16 step above or below 1 (a gap far below the estimate's error
+    bound); tokens 400-419 repeat cluster 3's initial centroid exactly."""
+    x = _inputs(1, 2, N, seed=seed)
+    v = synth.bf16_bits_to_f32(x["v"]).astype(np.float32)
+    one_up, one_dn = np.float32(1.0078125), np.float32(0.99609375)   # bf16 neighbours of 1
+    for h in range(2):
+        base = v[0, h, 0].copy()
+        base[0] = 0.0
+        v[0, h, 0] = base
+        v[0, h, N // 8] = base
+        v[0, h, N // 8, 0] = 2.0
+        v[0, h, 1:N // 8] = base
+        v[0, h, 1:N // 8, 0] = 1.0
+        v[0, h, N // 8 + 1:2 * N // 8] = base
+        v[0, h, N // 8 + 1:N // 8 + 38, 0] = one_up
+        v[0, h, N // 8 + 38:2 * N // 8, 0] = one_dn
+        v[0, h, 400:420] = v[0, h, 3 * N // 8]
+    x["v"] = synth.f32_to_bf16_bits(v)
+    return x
+
+
+@pytest.mark.parametrize("k,iters", [(8, 0), (8, 3), (5, 2)])
+def test_cluster_ties_and_near_ties_bit_exact(torch, k, iters):
+    """The clustering kernel labels by a certified estimate and falls back to
+    the pinned distances where the estimate cannot decide: exact ties and
+    near ties must come out as the oracle's (lowest cluster on a tie)."""
+    x = _tie_inputs()
+    p = vcattn.params(k=k, iters=iters)
+    perm, cent = vcattn.cluster(to_dev_bf16(x["v"]), p)
+    perm, cent = perm.cpu().numpy(), cent.cpu().numpy()
+    for h in range(2):
+        c_o, lab_o = oracle.kmeans_head(x["v"][0, h], k, iters)
+        if iters == 0:
+            assert np.all(lab_o[1:75] == 0) and np.all(lab_o[76:113] == 1) and np.all(lab_o[113:150] == 0)
+        assert np.array_equal(perm[0, h], oracle.stable_sort_labels(lab_o, k)), h
+        assert np.array_equal(cent[0, h].view(np.uint32), c_o.view(np.uint32)), h
+
+
 @pytest.mark.parametrize("B,H,N", SHAPES)
 @pytest.mark.parametrize("ksmooth", [True, False])
 def test_quant_qk_bit_exact(torch, B, H, N, ksmooth):

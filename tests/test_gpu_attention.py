@@ -1,6 +1,6 @@
 """GPU parity of the fused VC-Attention FP8 forward against the oracle.
 
-Bar (the benchmark spec): relative L2 <= 1e-3 between the kernel's bf16 output and the
+Bar: relative L2 <= 1e-3 between the kernel's bf16 output and the
 oracle's output rounded the same way (fp64 -> fp32 -> bf16), on every row for
 small and ragged shapes and on sampled rows (first, last, tail-tile and random
 rows) at the full workload sizes, in the launch configuration the bench times

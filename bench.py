@@ -425,6 +425,34 @@ def run_ours(args):
     ms_plain = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
     del ws_plain
 
+    # ---- the one-launch prologue (VC_FUSED_PROLOGUE), with clustering and with the
+    # cached permutation (E4M3 path only; the flag is ignored by the 4-bit variants)
+    fused = None
+    if not nvfp4:
+        p_f = vcattn.params(flags=vcattn.FLAGS_DEFAULT | vcattn.VC_FUSED_PROLOGUE)
+        ws_f, ws_f_bytes = vcattn.workspace(B, H, N, p_f)
+
+        def step_fused(pm=None):
+            st = vcattn.vc_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d,
+                                    None if pm is None else pm.data_ptr(), p_f, out.data_ptr(), ws_f.data_ptr(),
+                                    ws_f_bytes, sptr)
+            if st != 0:
+                raise vcattn.VcError(st, "vc_attn_fwd")
+
+        fused = {}
+        for tag, pm in (("with_clustering", None), ("cached_perm", perm)):
+            for _ in range(args.warmup):
+                step_fused(pm)
+            barrier()
+            e0.record(stream)
+            for _ in range(args.steps):
+                step_fused(pm)
+            e1.record(stream)
+            e1.synchronize()
+            fused[tag + "_ms_per_step"] = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+        fused["note"] = "vc_attn_fwd with VC_FUSED_PROLOGUE: the prologue as one cooperative persistent launch"
+        del ws_f
+
     # ---- BF16 comparator kernel
     for _ in range(args.warmup):
         vcattn.fwd_ref_bf16(q, k, v, out=out)
@@ -539,6 +567,7 @@ def run_ours(args):
                 "note": "share of the forward time that V-Smooth and repair add: the same call with "
                         "flags = VC_KSMOOTH (no grouping, demean, restore or repair) is the plain FP8 "
                         "forward; clustering runs only in the first 25% of denoising steps"},
+            "fused_prologue": fused,
             "ref_bf16": {"value": world * flops / (ms_ref * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms_ref,
                          "pct_of_bf16_peak": 100.0 * (flops / (ms_ref * 1e-3) / 1e12) / bf16_peak},
             "roofline": roof,

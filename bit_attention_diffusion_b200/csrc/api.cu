@@ -48,6 +48,7 @@ WsLayout make_layout(const Shape &s) {
   const size_t BH = static_cast<size_t>(s.BH), N = static_cast<size_t>(s.N), Nb = static_cast<size_t>(s.Nb),
                Npad = static_cast<size_t>(s.Npad), k = static_cast<size_t>(s.k);
   L.status = take(256);
+  L.gsync = take(256);  // grid-barrier counter of the one-launch prologue
   L.km_counter = take(BH * 4);
   L.vq_counter = take(BH * 4);
   L.kb_counter = take(BH * 4);
@@ -156,6 +157,8 @@ vc_status check_device() {
           cudaFuncSetAttribute(k_vc_attn_fwd44, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(attn_fp4_smem_bytes(true))) != cudaSuccess ||
           cudaFuncSetAttribute(k_kmeans_pass8, cudaFuncAttributeMaxDynamicSharedMemorySize, KMEANS8_SMEM) !=
+              cudaSuccess ||
+          cudaFuncSetAttribute(k_prologue_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, FUSED_SMEM) !=
               cudaSuccess) {
         ok_cache[dev] = 0;
         return VC_ERR_CUDA;
@@ -171,7 +174,8 @@ vc_status check_params(const vc_params *p) {
   if (!(p->rho >= 0.0f && p->rho < 1.0f)) return VC_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.0f) || !std::isfinite(p->softmax_scale)) return VC_ERR_INVALID_ARG;
   if (p->expcast_bias < 8 || p->expcast_bias > 126) return VC_ERR_INVALID_ARG;
-  if (p->flags & ~(VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH | VC_WARMSTART | VC_VFMT_NVFP4 | VC_QK_NVFP4))
+  if (p->flags & ~(VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH | VC_WARMSTART | VC_VFMT_NVFP4 | VC_QK_NVFP4 |
+                   VC_FUSED_PROLOGUE))
     return VC_ERR_INVALID_ARG;
   if ((p->flags & VC_QK_NVFP4) && !(p->flags & VC_VFMT_NVFP4)) return VC_ERR_INVALID_ARG;  // 4-bit QK needs 4-bit PV
   return VC_OK;
@@ -328,6 +332,56 @@ void launch_quant_v(const Shape &sh, const Ws &w, const uint16_t *V, const int32
   }
 }
 
+// Blocks of the one-launch prologue: every block must be resident at once
+// (cooperative launch), so the grid is the occupancy limit times the SMs.
+int fused_grid() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (!cache[dev]) {
+    int per_sm = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_prologue_fused, 256, FUSED_SMEM) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return 0;
+    cache[dev] = per_sm * sms;
+  }
+  return cache[dev];
+}
+
+// The whole prologue of vc_attn_fwd (E4M3 path, k <= 8) as one launch.
+vc_status launch_prologue_fused(const Shape &sh, const Ws &w, const uint16_t *Q, const uint16_t *K,
+                                const uint16_t *V, const int32_t *perm, bool cluster, cudaStream_t s) {
+  FusedPrologueParams fp{};
+  fp.Q = Q; fp.K = K; fp.V = V;
+  fp.BH = sh.BH; fp.N = sh.N; fp.Nb = sh.Nb; fp.Npad = sh.Npad; fp.nch32 = sh.nch32; fp.k = sh.k;
+  fp.iters = sh.iters; fp.R = sh.R; fp.Rpad = sh.Rpad; fp.km_cpb = sh.km_cpb; fp.km_nblk = sh.km_nblk;
+  fp.kb_nchunk = sh.kb_nchunk;
+  fp.demean = (sh.flags & VC_VSMOOTH) ? 1 : 0;
+  fp.ksmooth = (sh.flags & VC_KSMOOTH) ? 1 : 0;
+  fp.cluster = cluster ? 1 : 0;
+  fp.perm_in = perm;
+  fp.perm = w.at<int32_t>(w.L.perm); fp.labels = w.at<int32_t>(w.L.labels); fp.cent = w.at<float>(w.L.cent);
+  fp.km_psum = w.at<double>(w.L.km_psum); fp.km_pcnt = w.at<int>(w.L.km_pcnt);
+  fp.km_counter = w.at<unsigned>(w.L.km_counter);
+  fp.kb_part = w.at<double>(w.L.kbar_part); fp.kb_counter = w.at<unsigned>(w.L.kb_counter);
+  fp.kbar = w.at<float>(w.L.kbar);
+  fp.q8 = w.at<uint8_t>(w.L.q8); fp.k8 = w.at<uint8_t>(w.L.k8); fp.v8t = w.at<uint8_t>(w.L.v8t);
+  fp.sq = w.at<float>(w.L.sq); fp.sk = w.at<float>(w.L.sk); fp.amax_part = w.at<float>(w.L.amax_part);
+  fp.vscale = w.at<float>(w.L.vscale); fp.err = w.at<float>(w.L.err); fp.vexpo = w.at<int>(w.L.vexpo);
+  fp.vmean = w.at<uint16_t>(w.L.vmean); fp.mut2 = w.at<uint16_t>(w.L.mut2);
+  fp.rep_delta = w.at<uint16_t>(w.L.rep_delta); fp.deltat = w.at<uint16_t>(w.L.deltat);
+  fp.vq_counter = w.at<unsigned>(w.L.vq_counter); fp.rep_idx = w.at<int32_t>(w.L.rep_idx);
+  fp.gsync = w.at<unsigned>(w.L.gsync); fp.status = w.at<uint32_t>(w.L.status);
+  const int grid = fused_grid();
+  if (grid <= 0) return VC_ERR_CUDA;
+  void *args[] = {&fp};
+  if (cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(k_prologue_fused), dim3(grid), dim3(256), args,
+                                  FUSED_SMEM, s) != cudaSuccess)
+    return VC_ERR_CUDA;
+  count_launch();
+  return VC_OK;
+}
+
 float kappa_of(float softmax_scale) {
   return static_cast<float>(8.0 * 1.4426950408889634074 * static_cast<double>(softmax_scale));
 }
@@ -444,43 +498,53 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
   uint8_t *q8 = w.at<uint8_t>(w.L.q8), *k8 = w.at<uint8_t>(w.L.k8), *v8t = w.at<uint8_t>(w.L.v8t);
   float *sq = w.at<float>(w.L.sq), *sk = w.at<float>(w.L.sk), *vscale = w.at<float>(w.L.vscale);
   int32_t *rep_idx = w.at<int32_t>(w.L.rep_idx);
-  // Q/K quantization on a side stream (disjoint workspace regions). When this
-  // call clusters, the K channel means and Q (which do not depend on the
-  // permutation) start with the call, concurrent with the clustering, and K'
-  // follows once the permutation is known; otherwise Q and K' are one launch.
-  // Either way they run concurrently with the V passes, and the attention
-  // kernel waits for both streams. Per-call events, released once the work
-  // completes.
   const bool clusters = !perm && (sh.flags & VC_VSMOOTH);
-  cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};  // fork, permutation ready, join
-  cudaStream_t side = side_stream();
-  bool evok = side != nullptr;
-  for (int i = 0; i < 3 && evok; ++i) evok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
-  if (!evok) {
-    for (cudaEvent_t e : ev)
-      if (e) cudaEventDestroy(e);
-    return VC_ERR_CUDA;
+  const bool fused = (sh.flags & VC_FUSED_PROLOGUE) && sh.k <= 8 &&
+                     !(sh.flags & (VC_VFMT_NVFP4 | VC_QK_NVFP4));
+  if (fused) {
+    // the whole prologue in one launch; its time is reported as the first phase
+    if ((st = launch_prologue_fused(sh, w, Qh, Kh, Vh, perm, clusters, s)) != VC_OK) return st;
+    prof_mark(1, s);
+    prof_mark(2, s);
+    prof_mark(3, s);
+  } else {
+    // Q/K quantization on a side stream (disjoint workspace regions). When this
+    // call clusters, the K channel means and Q (which do not depend on the
+    // permutation) start with the call, concurrent with the clustering, and K'
+    // follows once the permutation is known; otherwise Q and K' are one launch.
+    // Either way they run concurrently with the V passes, and the attention
+    // kernel waits for both streams. Per-call events, released once the work
+    // completes.
+    cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};  // fork, permutation ready, join
+    cudaStream_t side = side_stream();
+    bool evok = side != nullptr;
+    for (int i = 0; i < 3 && evok; ++i) evok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!evok) {
+      for (cudaEvent_t e : ev)
+        if (e) cudaEventDestroy(e);
+      return VC_ERR_CUDA;
+    }
+    cudaEventRecord(ev[0], s);
+    cudaStreamWaitEvent(side, ev[0], 0);
+    if (clusters) launch_quant_qk(sh, w, Qh, Kh, nullptr, q8, sq, k8, sk, side, QK_Q);
+    const int32_t *pm = perm;
+    if (clusters) {
+      Shape cold = sh;  // vc_attn_fwd has no centroid input: always the default start
+      cold.flags &= ~VC_WARMSTART;
+      launch_cluster(cold, w, Vh, w.at<int32_t>(w.L.perm), w.at<float>(w.L.cent), s);
+      pm = w.at<int32_t>(w.L.perm);
+    }
+    prof_mark(1, s);
+    cudaEventRecord(ev[1], s);
+    cudaStreamWaitEvent(side, ev[1], 0);
+    launch_quant_qk(sh, w, Qh, Kh, pm, q8, sq, k8, sk, side, clusters ? QK_K : QK_QK);
+    cudaEventRecord(ev[2], side);
+    launch_quant_v(sh, w, Vh, pm, v8t, vscale, w.at<uint16_t>(w.L.vmean), rep_idx, w.at<uint16_t>(w.L.rep_delta), s);
+    prof_mark(2, s);
+    cudaStreamWaitEvent(s, ev[2], 0);
+    prof_mark(3, s);
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
   }
-  cudaEventRecord(ev[0], s);
-  cudaStreamWaitEvent(side, ev[0], 0);
-  if (clusters) launch_quant_qk(sh, w, Qh, Kh, nullptr, q8, sq, k8, sk, side, QK_Q);
-  const int32_t *pm = perm;
-  if (clusters) {
-    Shape cold = sh;  // vc_attn_fwd has no centroid input: always the default start
-    cold.flags &= ~VC_WARMSTART;
-    launch_cluster(cold, w, Vh, w.at<int32_t>(w.L.perm), w.at<float>(w.L.cent), s);
-    pm = w.at<int32_t>(w.L.perm);
-  }
-  prof_mark(1, s);
-  cudaEventRecord(ev[1], s);
-  cudaStreamWaitEvent(side, ev[1], 0);
-  launch_quant_qk(sh, w, Qh, Kh, pm, q8, sq, k8, sk, side, clusters ? QK_K : QK_QK);
-  cudaEventRecord(ev[2], side);
-  launch_quant_v(sh, w, Vh, pm, v8t, vscale, w.at<uint16_t>(w.L.vmean), rep_idx, w.at<uint16_t>(w.L.rep_delta), s);
-  prof_mark(2, s);
-  cudaStreamWaitEvent(s, ev[2], 0);
-  prof_mark(3, s);
-  for (cudaEvent_t e : ev) cudaEventDestroy(e);
 
   const bool fp4 = (sh.flags & VC_VFMT_NVFP4) != 0;
   const bool qk4 = (sh.flags & VC_QK_NVFP4) != 0;

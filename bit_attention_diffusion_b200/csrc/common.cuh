@@ -31,7 +31,7 @@ struct Shape {
 
 // Byte offsets of the workspace arrays (all 256-byte aligned).
 struct WsLayout {
-  size_t perm, labels, cent, km_psum, km_pcnt, km_counter, kb_counter;
+  size_t gsync, perm, labels, cent, km_psum, km_pcnt, km_counter, kb_counter;
   size_t kbar_part, kbar;
   size_t q8, sq, k8, sk;
   size_t v8t, vscale, vexpo, vmean, amax_part, vq_counter, mut2, err;

@@ -10,19 +10,23 @@
 // art); page "VC-Attention et FLUX 3 accélèrent la génération d'images sur
 // Blackwell", section "Le compromis entre vitesse et fidélité" (rho = 0.005).
 #include "common.cuh"
+#include "sm100.cuh"
 #include "prologue.cuh"
 
 namespace vc {
 
 // ============================================================== k-means
 // Init c_j = V[floor(j*N/k)].
-__global__ void k_kmeans_init(const uint16_t *__restrict__ V, int N, int k, float *__restrict__ cent) {
-  const int bh = blockIdx.x;
+__device__ __forceinline__ void kmeans_init_body(const uint16_t *__restrict__ V, int N, int k, float *__restrict__ cent, int bx, int by, int bz) {
+  const int bh = bx;
   for (int j = 0; j < k; ++j) {
     const long long src = (static_cast<long long>(j) * N) / k;
     cent[(static_cast<size_t>(bh) * k + j) * D + threadIdx.x] =
         bf16_to_f32(V[(static_cast<size_t>(bh) * N + src) * D + threadIdx.x]);
   }
+}
+__global__ void k_kmeans_init(const uint16_t *__restrict__ V, int N, int k, float *__restrict__ cent) {
+  kmeans_init_body(V, N, k, cent, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 // One Lloyd pass over `cpb` consecutive 128-token chunks per block: assign
@@ -177,18 +181,18 @@ __device__ __forceinline__ void km8_load_chunk(uint8_t *buf, const uint16_t *Vh,
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-__global__ void __launch_bounds__(256) k_kmeans_pass8(const uint16_t *__restrict__ V, int N, int k, int cpb,
+__device__ __forceinline__ void kmeans_pass8_body(const uint16_t *__restrict__ V, int N, int k, int cpb,
                                                       int nblk, float *__restrict__ cent,
                                                       int32_t *__restrict__ labels, double *__restrict__ psum,
                                                       int *__restrict__ pcnt, unsigned *__restrict__ counter,
-                                                      int accumulate) {
+                                                      int accumulate, int bx, int by, int bz) {
   extern __shared__ __align__(16) uint8_t dsm[];
   __shared__ __align__(16) float scent[D * 8];  // [c][j]; j >= k unused
   __shared__ int slab[TILE];
   __shared__ int slist[TILE];
   __shared__ int sstart[9];
   __shared__ int s_last;
-  const int bh = blockIdx.y, blk = blockIdx.x, tid = threadIdx.x;
+  const int bh = by, blk = bx, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const uint16_t *Vh = V + static_cast<size_t>(bh) * N * D;
   float *cent_h = cent + static_cast<size_t>(bh) * k * D;
@@ -345,21 +349,29 @@ __global__ void __launch_bounds__(256) k_kmeans_pass8(const uint16_t *__restrict
   }
   if (tid == 0) counter[bh] = 0u;
 }
+__global__ void __launch_bounds__(256) k_kmeans_pass8(const uint16_t *__restrict__ V, int N, int k, int cpb,
+                                                      int nblk, float *__restrict__ cent,
+                                                      int32_t *__restrict__ labels, double *__restrict__ psum,
+                                                      int *__restrict__ pcnt, unsigned *__restrict__ counter,
+                                                      int accumulate) {
+  kmeans_pass8_body(V, N, k, cpb, nblk, cent, labels, psum, pcnt, counter, accumulate, blockIdx.x, blockIdx.y, blockIdx.z);
+}
 
 // Stable counting sort of token indices by label, one block per (b,h): a
-// histogram gives each label's start; then rounds of 1024 tokens scatter in
+// histogram gives each label's start; then rounds of NT tokens scatter in
 // order (rank among equal labels = earlier lanes of the warp + earlier warps).
-__global__ void __launch_bounds__(1024) k_perm_sort(const int32_t *__restrict__ labels, int N, int k,
-                                                    int32_t *__restrict__ perm) {
+template <int NT>
+__device__ __forceinline__ void perm_sort_body(const int32_t *__restrict__ labels, int N, int k,
+                                                    int32_t *__restrict__ perm, int bx, int by, int bz) {
   __shared__ int base[64];
   __shared__ int tot[64];
-  __shared__ int wcnt[32][64];
-  const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __shared__ int wcnt[NT / 32][64];
+  const int bh = bx, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int32_t *lab = labels + static_cast<size_t>(bh) * N;
   int32_t *out = perm + static_cast<size_t>(bh) * N;
   if (tid < 64) base[tid] = 0;
   __syncthreads();
-  for (int n = tid; n < N; n += 1024) atomicAdd(&base[lab[n]], 1);
+  for (int n = tid; n < N; n += NT) atomicAdd(&base[lab[n]], 1);
   __syncthreads();
   if (tid == 0) {
     int run = 0;
@@ -369,8 +381,8 @@ __global__ void __launch_bounds__(1024) k_perm_sort(const int32_t *__restrict__ 
       run += c;
     }
   }
-  for (int n0 = 0; n0 < N; n0 += 1024) {
-    for (int i = tid; i < 32 * 64; i += 1024) (&wcnt[0][0])[i] = 0;
+  for (int n0 = 0; n0 < N; n0 += NT) {
+    for (int i = tid; i < (NT / 32) * 64; i += NT) (&wcnt[0][0])[i] = 0;
     __syncthreads();
     const int n = n0 + tid;
     const int L = n < N ? lab[n] : -1;
@@ -380,7 +392,7 @@ __global__ void __launch_bounds__(1024) k_perm_sort(const int32_t *__restrict__ 
     __syncthreads();
     if (tid < k) {
       int run = 0;
-      for (int w = 0; w < 32; ++w) {
+      for (int w = 0; w < NT / 32; ++w) {
         const int c = wcnt[w][tid];
         wcnt[w][tid] = run;
         run += c;
@@ -392,6 +404,10 @@ __global__ void __launch_bounds__(1024) k_perm_sort(const int32_t *__restrict__ 
     __syncthreads();
     if (tid < k) base[tid] += tot[tid];
   }
+}
+__global__ void __launch_bounds__(1024) k_perm_sort(const int32_t *__restrict__ labels, int N, int k,
+                                                    int32_t *__restrict__ perm) {
+  perm_sort_body<1024>(labels, N, k, perm, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 // ============================================================== streaming helpers
@@ -418,12 +434,12 @@ __device__ __forceinline__ void bf16x8(const uint4 &w, float *x) {
 // Channel sums of K in fp64 over a row range (one block per (chunk, b,h));
 // the last block of a (b,h) adds the chunk sums in chunk order and writes the
 // channel mean (0 without K smoothing).
-__global__ void __launch_bounds__(256) k_kbar(const uint16_t *__restrict__ K, int N, int nchunk, int ksmooth,
+__device__ __forceinline__ void kbar_body(const uint16_t *__restrict__ K, int N, int nchunk, int ksmooth,
                                               double *__restrict__ part, unsigned *__restrict__ counter,
-                                              float *__restrict__ kbar) {
+                                              float *__restrict__ kbar, int bx, int by, int bz) {
   __shared__ double red[16][128];
   __shared__ int s_last;
-  const int bh = blockIdx.y, ch = blockIdx.x, tid = threadIdx.x;
+  const int bh = by, ch = bx, tid = threadIdx.x;
   const int g = tid >> 4, c = tid & 15;
   const int rows = (N + nchunk - 1) / nchunk;
   const int r0 = ch * rows, r1 = min(N, r0 + rows);
@@ -465,18 +481,23 @@ __global__ void __launch_bounds__(256) k_kbar(const uint16_t *__restrict__ K, in
   }
   if (tid == 0) counter[bh] = 0u;
 }
+__global__ void __launch_bounds__(256) k_kbar(const uint16_t *__restrict__ K, int N, int nchunk, int ksmooth,
+                                              double *__restrict__ part, unsigned *__restrict__ counter,
+                                              float *__restrict__ kbar) {
+  kbar_body(K, N, nchunk, ksmooth, part, counter, kbar, blockIdx.x, blockIdx.y, blockIdx.z);
+}
 
 // Block quantization: z = 0 -> Q rows [128t, 128t+128) in original order;
 // z = 1 -> K rows perm[128t + r] minus the channel mean (z = blockIdx.z +
 // zbase: one launch may take both, or Q and K separately). scale = amax/448,
 // codes = E4M3(x * (448/amax)); rows past N get code 0.
-__global__ void __launch_bounds__(256) k_qk_quant(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
+__device__ __forceinline__ void qk_quant_body(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                                                   const int32_t *__restrict__ perm, const float *__restrict__ kbar,
                                                   int N, int Npad, int zbase, uint8_t *__restrict__ q8,
                                                   float *__restrict__ sq, uint8_t *__restrict__ k8,
-                                                  float *__restrict__ sk) {
+                                                  float *__restrict__ sk, int bx, int by, int bz) {
   __shared__ float wmax[8];
-  const int t = blockIdx.x, bh = blockIdx.y, z = blockIdx.z + zbase;
+  const int t = bx, bh = by, z = bz + zbase;
   const int tid = threadIdx.x, g = tid >> 4, c = tid & 15;
   const int cnt = min(TILE, N - t * TILE);
   const uint16_t *src = (z == 0 ? Q : K) + static_cast<size_t>(bh) * N * D + 8 * c;
@@ -532,6 +553,13 @@ __global__ void __launch_bounds__(256) k_qk_quant(const uint16_t *__restrict__ Q
     *reinterpret_cast<uint2 *>(dst + static_cast<size_t>(g + 16 * i) * D) = make_uint2(lo, hi);
   }
   if (tid == 0) (z == 0 ? sq : sk)[static_cast<size_t>(bh) * (Npad / TILE) + t] = scale;
+}
+__global__ void __launch_bounds__(256) k_qk_quant(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
+                                                  const int32_t *__restrict__ perm, const float *__restrict__ kbar,
+                                                  int N, int Npad, int zbase, uint8_t *__restrict__ q8,
+                                                  float *__restrict__ sq, uint8_t *__restrict__ k8,
+                                                  float *__restrict__ sk) {
+  qk_quant_body(Q, K, perm, kbar, N, Npad, zbase, q8, sq, k8, sk, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 // NVFP4 block quantization of the full 4-bit path, same grid and row mapping
@@ -654,16 +682,16 @@ __device__ __forceinline__ float sv_at(const uint8_t *sv, int r, int c) {
 // residual amax; the last block of a (b,h) turns the channel amax into the
 // power-of-two scale (the least with amax <= 448 * scale for E4M3 residuals,
 // amax <= 2688 * scale, the NVFP4 global scale, for 4-bit ones). Thread (h, c): channel c over rows [64h, 64h+64).
-__global__ void __launch_bounds__(256) k_quantv_pass1(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
+__device__ __forceinline__ void quantv_pass1_body(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
                                                       int N, int Nb, int demean, int fp4, uint16_t *__restrict__ vmean,
                                                       float *__restrict__ amax_part, float *__restrict__ vscale,
-                                                      int *__restrict__ vexpo, unsigned *__restrict__ counter) {
+                                                      int *__restrict__ vexpo, unsigned *__restrict__ counter, int bx, int by, int bz) {
   extern __shared__ __align__(16) uint8_t dsm[];
   uint8_t *sv = dsm;  // 128 rows x 272 bytes
   __shared__ double ssum[2][128];
   __shared__ float smax[2][128];
   __shared__ int s_last;
-  const int t = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int t = bx, bh = by, tid = threadIdx.x;
   const int p0 = t * TILE, cnt = min(TILE, N - p0);
   gather_tile(sv, V + static_cast<size_t>(bh) * N * D, perm ? perm + static_cast<size_t>(bh) * N : nullptr, p0, cnt);
   __syncthreads();
@@ -711,6 +739,12 @@ __global__ void __launch_bounds__(256) k_quantv_pass1(const uint16_t *__restrict
   vexpo[static_cast<size_t>(bh) * D + c] = e;
   if (c == 0) counter[bh] = 0u;
 }
+__global__ void __launch_bounds__(256) k_quantv_pass1(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
+                                                      int N, int Nb, int demean, int fp4, uint16_t *__restrict__ vmean,
+                                                      float *__restrict__ amax_part, float *__restrict__ vscale,
+                                                      int *__restrict__ vexpo, unsigned *__restrict__ counter) {
+  quantv_pass1_body(V, perm, N, Nb, demean, fp4, vmean, amax_part, vscale, vexpo, counter, blockIdx.x, blockIdx.y, blockIdx.z);
+}
 
 // Pass 2: residual codes (written channel-major), per-token error, and the
 // bf16 block means pre-divided by the channel scale for the in-kernel restore
@@ -720,17 +754,17 @@ __global__ void __launch_bounds__(256) k_quantv_pass1(const uint16_t *__restrict
 // scaling and dequantization of a channel pair are packed f32x2 operations
 // (each lane rounds as the scalar one; differences are sums with negated
 // operands, exactly the same values).
-__global__ void __launch_bounds__(256) k_quantv_pass2(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
+__device__ __forceinline__ void quantv_pass2_body(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
                                                       int N, int Nb, int Npad, int nch32,
                                                       const uint16_t *__restrict__ vmean,
                                                       const float *__restrict__ vscale, const int *__restrict__ vexpo,
                                                       uint8_t *__restrict__ v8t, float *__restrict__ err,
-                                                      uint16_t *__restrict__ mut2) {
+                                                      uint16_t *__restrict__ mut2, int bx, int by, int bz) {
   extern __shared__ __align__(16) uint8_t dsm[];
   uint8_t *sv = dsm;                            // 128 rows x 272 bytes
   uint8_t *codeT = dsm + TILE * VQ_ROW_BYTES;   // 128 channels x 144 bytes
   __shared__ __align__(16) float snmu[D], smult[D], snscale[D];  // -mean, 2^-e, -scale
-  const int t = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int t = bx, bh = by, tid = threadIdx.x;
   const int p0 = t * TILE, cnt = min(TILE, N - p0);
   gather_tile(sv, V + static_cast<size_t>(bh) * N * D, perm ? perm + static_cast<size_t>(bh) * N : nullptr, p0, cnt);
   if (tid < 128) {
@@ -789,6 +823,14 @@ __global__ void __launch_bounds__(256) k_quantv_pass2(const uint16_t *__restrict
     for (int i = 0; i < 4; ++i)
       *reinterpret_cast<uint4 *>(dst + 16 * i) = *reinterpret_cast<const uint4 *>(srcT + 16 * i);
   }
+}
+__global__ void __launch_bounds__(256) k_quantv_pass2(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
+                                                      int N, int Nb, int Npad, int nch32,
+                                                      const uint16_t *__restrict__ vmean,
+                                                      const float *__restrict__ vscale, const int *__restrict__ vexpo,
+                                                      uint8_t *__restrict__ v8t, float *__restrict__ err,
+                                                      uint16_t *__restrict__ mut2) {
+  quantv_pass2_body(V, perm, N, Nb, Npad, nch32, vmean, vscale, vexpo, v8t, err, mut2, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 // NVFP4 pass 2 (page "VC-Attention acelera atenção…", "V-Smooth: corrigindo
@@ -912,13 +954,14 @@ __global__ void __launch_bounds__(256) k_quantv4_pass2(const uint16_t *__restric
 // Top-R by error (float >= 0, so the bit pattern orders like the value), ties
 // to the lowest permuted position; output ascending. One block per (b,h):
 // radix select of the R-th largest key, then an ordered compaction.
-__global__ void __launch_bounds__(1024) k_repair_select(const float *__restrict__ err, int N, int R,
-                                                        int32_t *__restrict__ rep_idx) {
+template <int NT>
+__device__ __forceinline__ void repair_select_body(const float *__restrict__ err, int N, int R,
+                                                        int32_t *__restrict__ rep_idx, int bx, int by, int bz) {
   __shared__ unsigned hist[256];
   __shared__ unsigned s_prefix, s_need;
-  __shared__ int wgt[32], weq[32];
+  __shared__ int wgt[NT / 32], weq[NT / 32];
   __shared__ int s_base_gt, s_base_eq;
-  const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = bx, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const unsigned *key = reinterpret_cast<const unsigned *>(err + static_cast<size_t>(bh) * N);
   int32_t *out = rep_idx + static_cast<size_t>(bh) * R;
   if (tid == 0) {
@@ -930,7 +973,7 @@ __global__ void __launch_bounds__(1024) k_repair_select(const float *__restrict_
     if (tid < 256) hist[tid] = 0u;
     __syncthreads();
     const unsigned prefix = s_prefix;
-    for (int n = tid; n < N; n += 1024) {
+    for (int n = tid; n < N; n += NT) {
       const unsigned kv = key[n];
       if ((kv & mask) == prefix) atomicAdd(&hist[(kv >> shift) & 0xFFu], 1u);
     }
@@ -958,7 +1001,7 @@ __global__ void __launch_bounds__(1024) k_repair_select(const float *__restrict_
     s_base_eq = 0;
   }
   __syncthreads();
-  for (int n0 = 0; n0 < N; n0 += 1024) {
+  for (int n0 = 0; n0 < N; n0 += NT) {
     const int n = n0 + tid;
     const unsigned kv = n < N ? key[n] : 0u;
     const bool gt = n < N && kv > T;
@@ -984,7 +1027,7 @@ __global__ void __launch_bounds__(1024) k_repair_select(const float *__restrict_
     __syncthreads();
     if (tid == 0) {
       int tg = 0, te = 0;
-      for (int w = 0; w < 32; ++w) {
+      for (int w = 0; w < NT / 32; ++w) {
         tg += wgt[w];
         te += weq[w];
       }
@@ -993,6 +1036,10 @@ __global__ void __launch_bounds__(1024) k_repair_select(const float *__restrict_
     }
     __syncthreads();
   }
+}
+__global__ void __launch_bounds__(1024) k_repair_select(const float *__restrict__ err, int N, int R,
+                                                        int32_t *__restrict__ rep_idx) {
+  repair_select_body<1024>(err, N, R, rep_idx, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 // Same selection for N <= 32768, with no serial step: the keys stay in
@@ -1095,14 +1142,14 @@ __global__ void __launch_bounds__(RS_T) k_repair_select_reg(const float *__restr
 // delta = bf16(r - value(code)*scale) for every repaired token; also the
 // channel-major copy divided by the channel scale (deltat[bh][c][r], zero for
 // r in [R, Rpad)) that the attention kernel's repair MMA reads.
-__global__ void __launch_bounds__(256) k_repair_delta(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
+__device__ __forceinline__ void repair_delta_body(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
                                                       int N, int Nb, int R, int Rpad,
                                                       const int32_t *__restrict__ rep_idx,
                                                       const uint16_t *__restrict__ vmean,
                                                       const float *__restrict__ vscale, const int *__restrict__ vexpo,
-                                                      uint16_t *__restrict__ rep_delta, uint16_t *__restrict__ deltat) {
-  const int bh = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * 8 + warp;
+                                                      uint16_t *__restrict__ rep_delta, uint16_t *__restrict__ deltat, int bx, int by, int bz) {
+  const int bh = by, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = bx * 8 + warp;
   if (r >= Rpad) return;
   if (r >= R) {
     for (int i = 0; i < 4; ++i) deltat[(static_cast<size_t>(bh) * D + 4 * lane + i) * Rpad + r] = 0;
@@ -1136,6 +1183,14 @@ __global__ void __launch_bounds__(256) k_repair_delta(const uint16_t *__restrict
     const int c = 4 * lane + i;
     deltat[(static_cast<size_t>(bh) * D + c) * Rpad + r] = f32_to_bf16_rn(__fmul_rn(bf16_to_f32(dl[i]), mult[i]));
   }
+}
+__global__ void __launch_bounds__(256) k_repair_delta(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
+                                                      int N, int Nb, int R, int Rpad,
+                                                      const int32_t *__restrict__ rep_idx,
+                                                      const uint16_t *__restrict__ vmean,
+                                                      const float *__restrict__ vscale, const int *__restrict__ vexpo,
+                                                      uint16_t *__restrict__ rep_delta, uint16_t *__restrict__ deltat) {
+  repair_delta_body(V, perm, N, Nb, R, Rpad, rep_idx, vmean, vscale, vexpo, rep_delta, deltat, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 // The repair deltas of the NVFP4 residual: the token's codes are recomputed
@@ -1189,6 +1244,125 @@ __global__ void __launch_bounds__(256) k_repair_delta4(const uint16_t *__restric
 }
 
 // ============================================================== misc
+// ============================================================== one-launch prologue
+// Grid-wide barrier of a cooperative launch: every block adds one to the
+// counter (zeroed at the start of the call) and waits until it holds
+// `target` = (barriers passed so far) x gridDim.x. Bounded: a wait that runs
+// out sets the timeout bit in the status word and the block leaves the kernel
+// (the other blocks then run out as well); nothing spins for ever.
+__device__ bool grid_barrier(unsigned *count, unsigned target, uint32_t *status) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(count, 1u);
+    const long long t0 = clock64();
+    int ok = 1;
+    while (true) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(count) : "memory");
+      if (v >= target) break;
+      if (clock64() - t0 > VC_WAIT_LIMIT_CYCLES) {
+        atomicOr(status, ST_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      __nanosleep(100);
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+// The prologue of vc_attn_fwd (E4M3 path, k <= 8) as one persistent launch:
+// the bodies of the separate kernels, each work item one of their blocks,
+// with a grid barrier wherever a step reads what the previous one wrote.
+//   1. k-means init (if clustering), the K channel means, Q quantization
+//   2. each Lloyd pass (iters updates, then the final labels)
+//   3. the stable permutation
+//   4. K' quantization and V pass 1 (block means, channel scales)
+//   5. V pass 2 (codes, token errors, restore operands)
+//   6. repair selection, 7. repair deltas
+// Every (b,h) step is the one the separate kernels compute, so every output
+// is bit-identical to theirs.
+__global__ void __launch_bounds__(256) k_prologue_fused(const FusedPrologueParams p) {
+  unsigned passed = 0;
+  auto sync = [&]() -> bool {
+    ++passed;
+    return grid_barrier(p.gsync, passed * gridDim.x, p.status);
+  };
+  const int BH = p.BH, Nb = p.Nb;
+  {
+    const int n_init = p.cluster ? BH : 0;
+    const int n_kbar = p.ksmooth ? p.kb_nchunk * BH : BH;
+    const int n_q = Nb * BH;
+    for (int it = blockIdx.x; it < n_init + n_kbar + n_q; it += gridDim.x) {
+      int i = it;
+      if (i < n_init) {
+        if (threadIdx.x < D) kmeans_init_body(p.V, p.N, p.k, p.cent, i, 0, 0);
+      } else if ((i -= n_init) < n_kbar) {
+        if (p.ksmooth)
+          kbar_body(p.K, p.N, p.kb_nchunk, 1, p.kb_part, p.kb_counter, p.kbar, i % p.kb_nchunk, i / p.kb_nchunk, 0);
+        else if (threadIdx.x < D)
+          p.kbar[static_cast<size_t>(i) * D + threadIdx.x] = 0.0f;  // no K smoothing: mean 0
+      } else {
+        i -= n_kbar;
+        qk_quant_body(p.Q, p.K, nullptr, p.kbar, p.N, p.Npad, 0, p.q8, p.sq, p.k8, p.sk, i % Nb, i / Nb, 0);
+      }
+      __syncthreads();
+    }
+  }
+  if (!sync()) return;
+  const int32_t *pm = p.perm_in;
+  if (p.cluster) {
+    for (int pass = 0; pass <= p.iters; ++pass) {
+      for (int it = blockIdx.x; it < p.km_nblk * BH; it += gridDim.x) {
+        kmeans_pass8_body(p.V, p.N, p.k, p.km_cpb, p.km_nblk, p.cent, p.labels, p.km_psum, p.km_pcnt,
+                          p.km_counter, pass < p.iters ? 1 : 0, it % p.km_nblk, it / p.km_nblk, 0);
+        __syncthreads();
+      }
+      if (!sync()) return;
+    }
+    for (int it = blockIdx.x; it < BH; it += gridDim.x) {
+      perm_sort_body<256>(p.labels, p.N, p.k, p.perm, it, 0, 0);
+      __syncthreads();
+    }
+    if (!sync()) return;
+    pm = p.perm;
+  }
+  for (int it = blockIdx.x; it < 2 * Nb * BH; it += gridDim.x) {
+    if (it < Nb * BH) {
+      qk_quant_body(p.Q, p.K, pm, p.kbar, p.N, p.Npad, 1, p.q8, p.sq, p.k8, p.sk, it % Nb, it / Nb, 0);
+    } else {
+      const int i = it - Nb * BH;
+      quantv_pass1_body(p.V, pm, p.N, Nb, p.demean, 0, p.vmean, p.amax_part, p.vscale, p.vexpo, p.vq_counter,
+                        i % Nb, i / Nb, 0);
+    }
+    __syncthreads();
+  }
+  if (!sync()) return;
+  for (int it = blockIdx.x; it < Nb * BH; it += gridDim.x) {
+    quantv_pass2_body(p.V, pm, p.N, Nb, p.Npad, p.nch32, p.vmean, p.vscale, p.vexpo, p.v8t, p.err, p.mut2, it % Nb,
+                      it / Nb, 0);
+    __syncthreads();
+  }
+  if (p.R == 0) return;
+  if (!sync()) return;
+  for (int it = blockIdx.x; it < BH; it += gridDim.x) {
+    repair_select_body<256>(p.err, p.N, p.R, p.rep_idx, it, 0, 0);
+    __syncthreads();
+  }
+  if (!sync()) return;
+  const int nrb = (p.Rpad + 7) / 8;
+  for (int it = blockIdx.x; it < nrb * BH; it += gridDim.x) {
+    repair_delta_body(p.V, pm, p.N, Nb, p.R, p.Rpad, p.rep_idx, p.vmean, p.vscale, p.vexpo, p.rep_delta, p.deltat,
+                      it % nrb, it / nrb, 0);
+    __syncthreads();
+  }
+}
+
 __global__ void k_identity_perm(int32_t *perm, int N, long long total) {
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i < total) perm[i] = static_cast<int32_t>(i % N);

@@ -33,9 +33,38 @@ __global__ void k_repair_delta4(const uint16_t *V, const int32_t *perm, int N, i
                                 const uint8_t *v4img, uint16_t *rep_delta, uint16_t *deltat);
 __global__ void k_identity_perm(int32_t *perm, int N, long long total);
 
+// Arguments of the one-launch prologue (k_prologue_fused): the workspace
+// arrays of the separate kernels and the sizes they are launched with.
+struct FusedPrologueParams {
+  const uint16_t *Q, *K, *V;
+  int BH, N, Nb, Npad, nch32, k, iters, R, Rpad, km_cpb, km_nblk, kb_nchunk;
+  int demean, ksmooth, cluster;  // cluster: k-means + permutation in this launch
+  const int32_t *perm_in;        // the permutation when not clustering (null: identity)
+  int32_t *perm, *labels;
+  float *cent;
+  double *km_psum;
+  int *km_pcnt;
+  unsigned *km_counter;
+  double *kb_part;
+  unsigned *kb_counter;
+  float *kbar;
+  uint8_t *q8, *k8, *v8t;
+  float *sq, *sk, *amax_part, *vscale, *err;
+  int *vexpo;
+  uint16_t *vmean, *mut2, *rep_delta, *deltat;
+  unsigned *vq_counter;
+  int32_t *rep_idx;
+  unsigned *gsync;   // grid-barrier counter, zero at launch
+  uint32_t *status;  // device status word
+};
+// Cooperative launch only (every block resident): 256 threads, FUSED_SMEM of
+// dynamic shared memory.
+__global__ void k_prologue_fused(const FusedPrologueParams p);
+
 constexpr int QUANTV1_SMEM = 128 * 272;              // gathered rows
 constexpr int QUANTV2_SMEM = 128 * 272 + 128 * 144;  // rows + transposed codes
 constexpr int KMEANS8_SMEM = 2 * 128 * 272;  // double-buffered chunk rows
+constexpr int FUSED_SMEM = KMEANS8_SMEM > QUANTV2_SMEM ? KMEANS8_SMEM : QUANTV2_SMEM;  // the largest phase
 constexpr int KMEANS_SMEM_FIXED = 128 * 66 * 4;  // chunk rows; + k*128*(4+8) for centroids and sums
 
 }  // namespace vc

@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libvcattn.so")
 
 VC_OK, VC_ERR_INVALID_ARG, VC_ERR_UNSUPPORTED, VC_ERR_WORKSPACE, VC_ERR_CUDA, VC_ERR_TIMEOUT = range(6)
 VC_VSMOOTH, VC_REPAIR, VC_KSMOOTH, VC_WARMSTART, VC_VFMT_NVFP4, VC_QK_NVFP4 = 1, 2, 8, 16, 32, 64
+VC_FUSED_PROLOGUE = 128
 FLAGS_DEFAULT = VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH
 D = 128
 

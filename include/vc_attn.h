@@ -75,6 +75,16 @@ typedef enum {
  * is 0). The score scale is g_q * g_k * kappa. Without VC_VFMT_NVFP4 the
  * flag is invalid. vc_attn_quant_qk and vc_attn_fwd honour it. */
 #define VC_QK_NVFP4 64u
+/* The prologue of vc_attn_fwd (clustering when no permutation is passed,
+ * Q/K smoothing and quantization, V demean + quantization, repair list and
+ * deltas) as one cooperative persistent launch instead of one launch per
+ * step: every block of the grid is resident, the steps follow each other
+ * behind grid-wide barriers (bounded: a barrier that runs out sets
+ * VC_ERR_TIMEOUT in the device status word). Bit-identical results. Applies
+ * to the E4M3 path with k <= 8; otherwise the flag is ignored. vc_attn_fwd
+ * honours it; its profile then reports the whole prologue as the first
+ * phase. */
+#define VC_FUSED_PROLOGUE 128u
 
 typedef struct {
   int k;             /* k-means clusters, 1..64 (default 8) */
@@ -83,7 +93,7 @@ typedef struct {
   float softmax_scale; /* 0 => 1/sqrt(d) */
   int expcast_bias;  /* C: the running row maximum maps to byte C, 8..126 (default 120) */
   unsigned flags;    /* VC_VSMOOTH | VC_REPAIR | VC_KSMOOTH (default), optionally VC_WARMSTART,
-                        VC_VFMT_NVFP4, VC_QK_NVFP4 (with VC_VFMT_NVFP4) */
+                        VC_VFMT_NVFP4, VC_QK_NVFP4 (with VC_VFMT_NVFP4), VC_FUSED_PROLOGUE */
 } vc_params;
 
 /* Fill the defaults listed above. */

@@ -70,7 +70,7 @@ FAKE = 1 << 20  # a 256-aligned non-null address; never dereferenced in these ca
     (dict(p=dict(rho=-0.1)), vcattn.VC_ERR_INVALID_ARG),
     (dict(p=dict(expcast_bias=127)), vcattn.VC_ERR_INVALID_ARG),
     (dict(p=dict(flags=4)), vcattn.VC_ERR_INVALID_ARG),
-    (dict(p=dict(flags=128)), vcattn.VC_ERR_INVALID_ARG),
+    (dict(p=dict(flags=256)), vcattn.VC_ERR_INVALID_ARG),
     (dict(p=dict(flags=vcattn.FLAGS_DEFAULT | vcattn.VC_QK_NVFP4)), vcattn.VC_ERR_INVALID_ARG),  # needs VFMT_NVFP4
     (dict(p=dict(softmax_scale=-1.0)), vcattn.VC_ERR_INVALID_ARG),
 ])

@@ -584,9 +584,9 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
     ap.O = static_cast<uint16_t *>(O);
     ap.status = w.at<uint32_t>(w.L.status);
     if (qk4)
-      k_vc_attn_fwd44<<<dim3(sh.Nb, sh.BH), 352, attn_fp4_smem_bytes(true), s>>>(tq, tk, tmu, tdt, ap);
+      k_vc_attn_fwd44<<<dim3((sh.Nb + 1) / 2, sh.BH), 352, attn_fp4_smem_bytes(true), s>>>(tq, tk, tmu, tdt, ap);
     else
-      k_vc_attn_fwd4<<<dim3(sh.Nb, sh.BH), 352, attn_fp4_smem_bytes(false), s>>>(tq, tk, tmu, tdt, ap);
+      k_vc_attn_fwd4<<<dim3((sh.Nb + 1) / 2, sh.BH), 352, attn_fp4_smem_bytes(false), s>>>(tq, tk, tmu, tdt, ap);
     count_launch();
     prof_mark(4, s);
     if (g_prof.on) ++g_prof.calls;

@@ -19,7 +19,7 @@ struct AttnFp4Params {
   uint32_t *status;           // device status word
 };
 
-// QK^T from the E4M3 tiles (tmQ, tmK).
+// Grid ceil(Nb/2) x B*H: CTA x takes query tiles 2x and 2x+1. QK^T from the E4M3 tiles (tmQ, tmK).
 __global__ void k_vc_attn_fwd4(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                                const __grid_constant__ CUtensorMap tmMu, const __grid_constant__ CUtensorMap tmDT,
                                const AttnFp4Params p);

@@ -803,29 +803,12 @@ __device__ __forceinline__ void attn4_body(const CUtensorMap &tmQ, const CUtenso
     if (ok) ok = wwait(&bars.fin, 0);
     if (ok) {
       tc_fence_after();
-      const int row = qt * 128 + r;
-      uint16_t *orow = p.O + (static_cast<size_t>(bh) * p.N + row) * 128;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint32_t v[32];
-        tmem_ld32(lrow + tm_o(g) + 32 * i, v);
-        tmem_wait_ld();
-        if (row < p.N) {
-#pragma unroll
-          for (int gg = 0; gg < 4; ++gg) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 32 * i + 8 * gg + 2 * e;
-              const float o0 = __fdiv_rn(__uint_as_float(v[8 * gg + 2 * e]) * s_vscale[c], lt);
-              const float o1 = __fdiv_rn(__uint_as_float(v[8 * gg + 2 * e + 1]) * s_vscale[c + 1], lt);
-              const __nv_bfloat162 ob = __floats2bfloat162_rn(o0, o1);
-              w[e] = *reinterpret_cast<const uint32_t *>(&ob);
-            }
-            *reinterpret_cast<uint4 *>(orow + 32 * i + 8 * gg) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
-      }
+      // every product is complete: a stages over the K ring, b over the
+      // restore operands
+      const int row0 = qt * 128 + q4 * 32;
+      uint8_t *stg = (g == 0 ? sK : sAr) + q4 * 32 * 256;
+      store_o_rows(lrow + tm_o(g), s_vscale, lt, stg, p.O + (static_cast<size_t>(bh) * p.N + row0) * 128,
+                   p.N - row0);
     }
   }
   tc_fence_before();

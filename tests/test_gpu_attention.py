@@ -214,3 +214,24 @@ def test_fwd_host_equals_device_call(torch, groups):
     hout = vcattn.fwd_host(hq, hk, hv, groups, p=vcattn.params())
     torch.cuda.synchronize()
     assert torch.equal(hout, ref.cpu())
+
+
+@pytest.mark.parametrize("extra", ["VC_VFMT_NVFP4", "VC_QK_NVFP4", "VC_FUSED_PROLOGUE", "VC_KSMOOTH"])
+def test_fwd_host_equals_device_call_variants(torch, extra):
+    """The host-buffer entry point runs the same per-run pipeline for the
+    4-bit variants and the one-launch prologue: bit-identical output to the
+    device call with the same flags (B=2 so that runs cross a batch)."""
+    flags = vcattn.FLAGS_DEFAULT | getattr(vcattn, extra)
+    if extra == "VC_QK_NVFP4":
+        flags |= vcattn.VC_VFMT_NVFP4
+    if extra == "VC_KSMOOTH":
+        flags = vcattn.VC_KSMOOTH
+    p = vcattn.params(flags=flags)
+    B, H, N = 2, 3, 900
+    x = synth.make_inputs(synth.custom(B, H, N, seed=820 + len(extra)))
+    q, k, v = (to_dev_bf16(x[n]) for n in "qkv")
+    ref = vcattn.fwd(q, k, v, p=p)
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hout = vcattn.fwd_host(hq, hk, hv, 4, p=p)
+    torch.cuda.synchronize()
+    assert torch.equal(hout, ref.cpu())

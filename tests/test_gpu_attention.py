@@ -235,3 +235,39 @@ def test_fwd_host_equals_device_call_variants(torch, extra):
     hout = vcattn.fwd_host(hq, hk, hv, 4, p=p)
     torch.cuda.synchronize()
     assert torch.equal(hout, ref.cpu())
+
+
+@pytest.mark.parametrize("extra", ["", "VC_VFMT_NVFP4", "VC_QK_NVFP4"])
+def test_fwd_constant_values_are_reproduced_exactly(torch, extra):
+    """Every value token of a head is one bf16 vector (head 0: zeros). The
+    block means are that vector and every residual, code and repair delta is
+    zero, so each output row is sum_t l_t * mean / sum_t l_t: the vector
+    itself, bit for bit in bf16 (the row sums' bf16 hi/lo split and fp32 sums
+    leave a relative error near 1e-5, far below half a bf16 ulp). N = 4300:
+    a ragged last tile, 34 KV tiles, two block-mean restore chunks."""
+    flags = vcattn.FLAGS_DEFAULT
+    if extra:
+        flags |= vcattn.VC_VFMT_NVFP4
+    if extra == "VC_QK_NVFP4":
+        flags |= vcattn.VC_QK_NVFP4
+    B, H, N = 1, 2, 4300
+    x = synth.make_inputs(synth.custom(B, H, N, seed=850))
+    row = x["v"][0, 1, 0].copy()
+    assert (bf16_vals(row) != 0).all()
+    x["v"][0, 0] = 0
+    x["v"][0, 1] = row[None, :]
+    out = _run_gpu(torch, x, vcattn.params(flags=flags))
+    assert (out[0, 0] == 0).all()
+    assert (out[0, 1] == row[None, :]).all()
+
+
+def test_fwd_large_repair_budget(torch):
+    """rho = 0.9: 270 of 300 tokens repaired, as many repair chunks (3) as KV
+    tiles; every row against the oracle."""
+    B, H, N = 1, 2, 300
+    x = synth.make_inputs(synth.custom(B, H, N, seed=860))
+    out = _run_gpu(torch, x, vcattn.params(rho=0.9))
+    for h in range(H):
+        r = oracle.vc_attention_head(x["q"][0, h], x["k"][0, h], x["v"][0, h], rho=0.9)
+        ref = bf16_vals(oracle.to_bf16_bits(r["out"]))
+        assert rel_l2(bf16_vals(out[0, h]), ref) <= TOL

@@ -271,3 +271,28 @@ def test_fwd_large_repair_budget(torch):
         r = oracle.vc_attention_head(x["q"][0, h], x["k"][0, h], x["v"][0, h], rho=0.9)
         ref = bf16_vals(oracle.to_bf16_bits(r["out"]))
         assert rel_l2(bf16_vals(out[0, h]), ref) <= TOL
+
+
+@pytest.mark.parametrize("extra", ["", "VC_VFMT_NVFP4", "VC_QK_NVFP4"])
+def test_fwd_dominant_key_moves_the_frame_past_fp32_range(torch, extra):
+    """One key (position 1500, KV tile 11) is 2000 times the unit direction of
+    the summed query rows. For about a third of the rows its log2-domain score
+    lies more than 150 units above the earlier tiles' maximum, so the frame
+    jumps by more than 1200 byte units at once and the rescale factor of
+    everything accumulated so far is below fp32's range (the kernels flush it
+    to zero); for about half the rows that key takes all the probability
+    mass. Every row against the oracle."""
+    flags = vcattn.FLAGS_DEFAULT
+    if extra:
+        flags |= vcattn.VC_VFMT_NVFP4
+    if extra == "VC_QK_NVFP4":
+        flags |= vcattn.VC_QK_NVFP4
+    B, H, N = 1, 1, 2000
+    x = synth.make_inputs(synth.custom(B, H, N, seed=880))
+    u = bf16_vals(x["q"][0, 0]).sum(axis=0)
+    x["k"][0, 0, 1500] = oracle.to_bf16_bits(2000.0 * u / np.linalg.norm(u))
+    out = _run_gpu(torch, x, vcattn.params(flags=flags))
+    r = oracle.vc_attention_head(x["q"][0, 0], x["k"][0, 0], x["v"][0, 0], flags=flags)
+    ref = bf16_vals(oracle.to_bf16_bits(r["out"]))
+    assert np.isfinite(bf16_vals(out[0, 0])).all()
+    assert rel_l2(bf16_vals(out[0, 0]), ref) <= TOL

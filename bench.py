@@ -178,6 +178,19 @@ def _to_dev(torch, bits):
 
 
 # ---------------------------------------------------------------- CPU oracle timing
+def _cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), else the platform's."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown CPU"
+
+
 def cpu_oracle_sample(wl, x, rows_per_head: int = 96, heads=(0,), extra_flags: int = 0):
     """Time the oracle on a bounded sample and extrapolate to the workload.
 
@@ -211,7 +224,8 @@ def cpu_oracle_sample(wl, x, rows_per_head: int = 96, heads=(0,), extra_flags: i
     tflops = wl.flops / t_full / 1e12
     sample = (f"{nh} head(s): full per-head prologue + {rows_per_head} of {wl.N} query rows each, "
               f"extrapolated linearly in rows and heads to B={wl.B},H={wl.H} "
-              f"({t_pro + t_rows:.1f} s measured, {t_full:.0f} s extrapolated)")
+              f"({t_pro + t_rows:.1f} s measured, {t_full:.0f} s extrapolated) "
+              f"on {cores} threads of {_cpu_model()} ({os.cpu_count()} logical CPUs)")
     return tflops, cores, sample, t_pro + t_rows
 
 

@@ -181,3 +181,24 @@ def test_exactv_diagnostic_equals_method_when_values_are_lossless(orc):
     assert np.allclose(ev, r["out"], rtol=1e-9, atol=1e-9)
     r2 = orc.vc_attention_head(q, k, v, flags=flags & ~orc.FLAG_REPAIR, softmax_scale=scale, perm=perm)
     assert not np.allclose(ev, r2["out"], rtol=1e-9, atol=1e-9)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "nvfp4", "nvfp4qk"])
+def test_constant_values_are_reproduced_exactly(orc, fmt):
+    """Every value token of a head is one bf16 vector: the block means are
+    that vector and every residual is zero, so each output row is
+    sum_t l_t * mu / sum_t l_t = mu whatever the scores (the restore through
+    the row sums, in closed form); an all-zero head gives zeros. A dropped
+    restore, a normalizer other than the decoded row sum, or frames applied
+    to O and l differently break it. 300 tokens: three KV tiles, the last
+    one ragged."""
+    extra = {"e4m3": 0, "nvfp4": orc.FLAG_VFMT_NVFP4,
+             "nvfp4qk": orc.FLAG_VFMT_NVFP4 | orc.FLAG_QK_NVFP4}[fmt]
+    N = 300
+    x = synth.make_inputs(synth.custom(1, 1, N, seed=905))
+    row = x["v"][0, 0, 7].copy()
+    assert (synth.bf16_bits_to_f32(row) != 0).all()
+    for vrow in (row, np.zeros_like(row)):
+        v = np.broadcast_to(vrow, (N, 128)).copy()
+        r = orc.vc_attention_head(x["q"][0, 0], x["k"][0, 0], v, flags=orc.FLAGS_DEFAULT | extra)
+        assert np.array_equal(orc.to_bf16_bits(r["out"]), np.broadcast_to(vrow, (N, 128)))

@@ -202,3 +202,36 @@ def test_constant_values_are_reproduced_exactly(orc, fmt):
         v = np.broadcast_to(vrow, (N, 128)).copy()
         r = orc.vc_attention_head(x["q"][0, 0], x["k"][0, 0], v, flags=orc.FLAGS_DEFAULT | extra)
         assert np.array_equal(orc.to_bf16_bits(r["out"]), np.broadcast_to(vrow, (N, 128)))
+
+
+def test_dominant_key_rows_return_its_reconstructed_value(orc):
+    """One key (token 1500, 2000 times the unit direction of the summed query
+    rows) outscores every other key by more than 64 log2 units on many rows
+    (exact scores; FP8 rounding of Q and K' moves them by a few units). That
+    is far beyond the byte range (C = 120 byte units = 15 log2 units), so
+    every later key's byte is 0. The earlier tiles, at most N keys of at most
+    2^8.75 each, survive only scaled by about 2^-60 after the frame jump.
+    Those rows' output is then the dominant token's reconstructed value
+    mu_t + value(code) * s (+ its repair delta) to within 1e-9. This pins the
+    clamp at 0, a frame jump of hundreds of byte units, and the value
+    reconstruction of a single key."""
+    N = 2000
+    x = synth.make_inputs(synth.custom(1, 1, N, seed=880))
+    q = orc.bf16_value(x["q"][0, 0]).astype(np.float64)
+    u = q.sum(axis=0)
+    kb = x["k"][0, 0].copy()
+    kb[1500] = orc.to_bf16_bits(2000.0 * u / np.linalg.norm(u))
+    k = orc.bf16_value(kb).astype(np.float64)
+    s = q @ (k - k.mean(axis=0)).T / np.sqrt(128.0) * np.log2(np.e)
+    gap = s[:, 1500] - np.delete(s, 1500, axis=1).max(axis=1)
+    rows = np.nonzero(gap > 64.0)[0].astype(np.int32)
+    assert rows.size > 100
+    r = orc.vc_attention_head(x["q"][0, 0], kb, x["v"][0, 0], rows=rows)
+    vq = r["vq"]
+    pos = int(np.nonzero(r["perm"] == 1500)[0][0])  # its permuted position
+    vhat = (orc.bf16_value(vq["vmean"][pos // 128]).astype(np.float64)
+            + orc.e4m3_value(vq["v8"][pos]).astype(np.float64) * vq["vscale"].astype(np.float64))
+    hit = np.nonzero(vq["rep_idx"] == pos)[0]
+    if hit.size:
+        vhat = vhat + orc.bf16_value(vq["rep_delta"][hit[0]]).astype(np.float64)
+    assert np.allclose(r["out"], np.broadcast_to(vhat, r["out"].shape), rtol=1e-9, atol=1e-12)

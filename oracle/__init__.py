@@ -86,6 +86,7 @@ def lib():
             L.orc_e4m3_value_n.argtypes = [P, i64, P]
             L.orc_bf16_round_n.argtypes = [P, i64, P]
             L.orc_expcast_n.argtypes = [P, P, P, i64, P]
+            L.orc_expcast_bits_n.argtypes = [ctypes.c_uint32, i64, i32, f32, f32, P]
             L.orc_e2m1_value.restype = ctypes.c_double
             L.orc_e2m1_value.argtypes = [ctypes.c_uint8]
             L.orc_e2m1_encode.restype = ctypes.c_uint8
@@ -141,6 +142,15 @@ def expcast(acc, alpha, c) -> np.ndarray:
                              dtype=np.float32)
     out = np.empty(acc.shape, np.uint8)
     lib().orc_expcast_n(_p(acc), _p(alpha), _p(c), acc.size, _p(out))
+    return out
+
+
+def expcast_bits(first: int, n: int, negative: bool, alpha: float, c: float) -> np.ndarray:
+    """ExpCast bytes of the n consecutive binary32 bit patterns first, first+1, ...
+    (sign bit set when `negative`), one alpha and c: the exhaustive sweeps."""
+    out = np.empty(int(n), np.uint8)
+    lib().orc_expcast_bits_n(int(first), int(n), int(bool(negative)), float(np.float32(alpha)),
+                             float(np.float32(c)), _p(out))
     return out
 
 

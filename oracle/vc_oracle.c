@@ -1018,3 +1018,22 @@ void orc_expcast_n(const float *acc, const float *alpha, const float *c, long lo
     for (long long i = 0; i < n; ++i)
         out[i] = (uint8_t)orc_expcast_byte(acc[i], alpha[i], c[i]);
 }
+
+/* ExpCast of a run of consecutive binary32 bit patterns, for the exhaustive
+ * sweeps of the tests: acc = the float whose bit pattern is first + i (with
+ * the sign bit set when `negative`), one alpha and c for the whole run. A
+ * plain loop over orc_expcast_byte, split over threads. */
+void orc_expcast_bits_n(uint32_t first, long long n, int negative, float alpha, float c, uint8_t *out)
+{
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (long long i = 0; i < n; ++i) {
+        uint32_t b = first + (uint32_t)i;
+        float a;
+        if (negative)
+            b |= 0x80000000u;
+        memcpy(&a, &b, 4);
+        out[i] = (uint8_t)orc_expcast_byte(a, alpha, c);
+    }
+}

@@ -1,10 +1,11 @@
 """GPU parity of the fused VC-Attention FP8 forward against the oracle.
 
 Bar: relative L2 <= 1e-3 between the kernel's bf16 output and the
-oracle's output rounded the same way (fp64 -> fp32 -> bf16), on every row for
-small and ragged shapes and on sampled rows (first, last, tail-tile and random
-rows) at the full workload sizes, in the launch configuration the bench times
-(vc_attn_fwd with default parameters, clustering inside the call).
+oracle's output rounded the same way (fp64 -> fp32 -> bf16), over the checked
+rows of every head (each head on its own, and all heads together), on every
+row for small and ragged shapes, in the launch configuration the bench times
+(vc_attn_fwd with default parameters, clustering inside the call). The full
+workload sizes are in test_gpu_fullsize.py.
 
 Against exact fp64 attention the 8-bit path sits at the FP8 noise floor on
 i.i.d. Gaussian inputs (about 5-6% relative L2, cosine ~0.998, the value the
@@ -79,7 +80,7 @@ def test_fwd_matches_oracle_all_rows(torch, B, H, N):
     out = _run_gpu(torch, x, vcattn.params())
     heads = [(b, h) for b in range(B) for h in range(H)]
     rel, worst = _compare(x, out, heads, _all_rows, oracle.FLAGS_DEFAULT)
-    assert rel <= TOL and worst <= 2 * TOL, (rel, worst)
+    assert rel <= TOL and worst <= TOL, (rel, worst)
 
 
 @pytest.mark.parametrize("flags", [oracle.FLAG_KSMOOTH, oracle.FLAG_KSMOOTH | oracle.FLAG_REPAIR,
@@ -90,7 +91,7 @@ def test_fwd_flag_variants(torch, flags):
     x = synth.make_inputs(synth.custom(B, H, N, seed=400 + flags))
     out = _run_gpu(torch, x, vcattn.params(flags=flags))
     rel, worst = _compare(x, out, [(0, 0), (0, 1)], _all_rows, flags)
-    assert rel <= TOL and worst <= 2 * TOL, (rel, worst)
+    assert rel <= TOL and worst <= TOL, (rel, worst)
 
 
 def test_fwd_other_parameters(torch):
@@ -137,19 +138,16 @@ def test_fwd_lossless_case_equals_exact_attention(torch):
 
 @pytest.mark.parametrize("name,rows_per_head,heads", [
     ("tiny_b1h2n1024", None, [(0, 0), (0, 1)]),
-    ("image1024_b1h24n4256", 48, [(0, 0), (0, 11), (0, 23)]),
-    ("image2048_b1h24n16544", 24, [(0, 0), (0, 23)]),
-    ("i2i2048_b2h24n32928", 12, [(0, 5), (1, 17)]),
-    ("video720p_b1h40n75600", 8, [(0, 0), (0, 39)]),
 ])
 def test_fwd_workloads_match_oracle(torch, name, rows_per_head, heads):
-    """All five workloads at full size, default parameters, clustering inside
-    vc_attn_fwd (the call the bench times)."""
+    """The tiny workload, every row, default parameters, clustering inside
+    vc_attn_fwd (the call the bench times); the four larger workloads are
+    checked at full size in test_gpu_fullsize.py."""
     wl, x = synth.make_by_name(name)
     out = _run_gpu(torch, x, vcattn.params())
     rows_fn = _all_rows if rows_per_head is None else (lambda N: _sampled_rows(N, rows_per_head))
     rel, worst = _compare(x, out, heads, rows_fn, oracle.FLAGS_DEFAULT)
-    assert rel <= TOL and worst <= 2 * TOL, (rel, worst)
+    assert rel <= TOL and worst <= TOL, (rel, worst)
     # every row of every head is finite
     assert np.isfinite(bf16_vals(out)).all()
 
@@ -198,7 +196,7 @@ def test_fwd_restore_chunk_boundaries(torch, N):
     x = synth.make_inputs(synth.custom(1, 2, N, seed=600 + N))
     out = _run_gpu(torch, x, vcattn.params())
     rel, worst = _compare(x, out, [(0, 0), (0, 1)], lambda n: _sampled_rows(n, 48), oracle.FLAGS_DEFAULT)
-    assert rel <= TOL and worst <= 2 * TOL, (rel, worst)
+    assert rel <= TOL and worst <= TOL, (rel, worst)
 
 
 @pytest.mark.parametrize("groups", [1, 2, 7])

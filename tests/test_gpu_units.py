@@ -59,6 +59,35 @@ def test_expcast_dense_sweep_over_byte_range(torch):
     assert np.array_equal(got, want)
 
 
+@pytest.mark.parametrize("alpha,c", [(1.0, 120.0), (0.0553709, 112.0)])
+def test_expcast_exhaustive_matches_oracle(torch, alpha, c):
+    """Every binary32 score acc <= 0 with acc*alpha >= -(c+1) (about 1.1e9
+    inputs per case, the range the oracle's exhaustive pin covers: every score
+    that can reach a nonzero byte): the device bytes equal the oracle's, byte
+    for byte. alpha = 1, c = 120 is the score in byte units against the row
+    maximum's frame; the second case has a non-power-of-two alpha, so the
+    fused product's rounding decides bytes."""
+    alpha = float(np.float32(alpha))
+    last = int(np.float32((c + 1.0) / alpha).view(np.uint32))
+    while float(np.uint32(last).view(np.float32)) * alpha < c + 1.0:
+        last += 1
+    total = last + 1
+    chunk = 1 << 27
+    a_dev = torch.full((chunk,), alpha, dtype=torch.float32, device="cuda")
+    c_dev = torch.full((chunk,), c, dtype=torch.float32, device="cuda")
+    checked = 0
+    for lo in range(0, total, chunk):
+        n = min(chunk, total - lo)
+        n += n & 1  # the entry point takes pairs; one extra input past the range is harmless
+        acc = torch.arange(lo, lo + n, dtype=torch.int64, device="cuda").to(torch.int32).view(torch.float32).neg()
+        got = vcattn.expcast(acc, a_dev[:n], c_dev[:n]).cpu().numpy()
+        want = oracle.expcast_bits(lo, n, True, alpha, c)
+        bad = np.nonzero(got != want)[0]
+        assert bad.size == 0, [(lo + int(i), int(got[i]), int(want[i])) for i in bad[:8]]
+        checked += n
+    assert checked >= total > 1_000_000_000
+
+
 def test_e4m3_encoder_bit_exact(torch):
     rng = np.random.default_rng(101)
     n = 1 << 22

@@ -30,10 +30,14 @@ def _dev_bf16(torch, bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def _noalloc(torch, v, p):
+def _noalloc(torch, v, p, init=None):
     B, H, N, d = (int(s) for s in v.shape)
     perm = torch.empty((B, H, N), dtype=torch.int32, device="cuda")
-    cent = torch.empty((B, H, p.k, 128), dtype=torch.float32, device="cuda")
+    if init is None:
+        cent = torch.empty((B, H, p.k, 128), dtype=torch.float32, device="cuda")
+    else:
+        cent = init.clone()
+        p = vcattn.VcParams(p.k, p.iters, p.rho, p.softmax_scale, p.expcast_bias, p.flags | vcattn.VC_WARMSTART)
     st = vcattn.vc_attn_cluster_noalloc(v.data_ptr(), B, H, N, d, p, perm.data_ptr(), cent.data_ptr(),
                                         torch.cuda.current_stream().cuda_stream)
     assert st == vcattn.VC_OK, vcattn.status_str(st)
@@ -51,6 +55,41 @@ def test_noalloc_cluster_matches_workspace_cluster_twice_in_a_row(torch):
         torch.cuda.synchronize()
         assert torch.equal(perm, perm_ref)
         assert torch.equal(cent.view(torch.int32), cent_ref.view(torch.int32))
+
+
+def test_noalloc_more_clusters_and_warm_start_match_back_to_back(torch):
+    """k = 16 (the general k-means kernel, its own shared-memory sizing) and a
+    warm start from given centroids (VC_WARMSTART: the centroids are an input),
+    run back to back on the shared array, each against vc_attn_cluster."""
+    x = synth.make_inputs(synth.custom(1, 4, 3000, seed=73))
+    v = _dev_bf16(torch, x["v"])
+    p16 = vcattn.params(k=16, iters=2)
+    perm_ref, cent_ref = vcattn.cluster(v, p16)
+    perm, cent = _noalloc(torch, v, p16)
+    torch.cuda.synchronize()
+    assert torch.equal(perm, perm_ref) and torch.equal(cent.view(torch.int32), cent_ref.view(torch.int32))
+    _, c2 = vcattn.cluster(v, vcattn.params(iters=2))
+    p3 = vcattn.params(iters=3)
+    perm_ref, cent_ref = vcattn.cluster(v, p3, init=c2)
+    perm, cent = _noalloc(torch, v, p3, init=c2)
+    torch.cuda.synchronize()
+    assert torch.equal(perm, perm_ref) and torch.equal(cent.view(torch.int32), cent_ref.view(torch.int32))
+
+
+def test_noalloc_video_workload_shape(torch):
+    """The 720p video shape (B=1, H=40, N=75600: 3.0 M tokens) fits the array:
+    equal to vc_attn_cluster, and head 0 equal to the oracle."""
+    import oracle
+    wl, x = synth.make_by_name("video720p_b1h40n75600")
+    p = vcattn.params()
+    v = _dev_bf16(torch, x["v"])
+    perm_ref, cent_ref = vcattn.cluster(v, p)
+    perm, cent = _noalloc(torch, v, p)
+    torch.cuda.synchronize()
+    assert torch.equal(perm, perm_ref) and torch.equal(cent.view(torch.int32), cent_ref.view(torch.int32))
+    c_o, lab_o = oracle.kmeans_head(x["v"][0, 0], p.k, p.iters)
+    assert np.array_equal(perm[0, 0].cpu().numpy(), oracle.stable_sort_labels(lab_o, p.k))
+    assert np.array_equal(cent[0, 0].cpu().numpy().view(np.uint32), c_o.view(np.uint32))
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(torch):

@@ -52,6 +52,7 @@ DTYPE = {"e4m3": "fp8_e4m3 (fp32 accumulate)",
          "nvfp4qk": "nvfp4 (e2m1 + e4m3 block-16 scales) QK and PV, fp32 accumulate"}
 SMS = 148
 EX2_PER_CLK_SM = 16  # special-function unit: 2^x results per clock per SM (CUDA throughput table, cc 10.0)
+NOMINAL_FP8_TFLOPS = 4500.0  # B200 dense FP8 (no sparsity), nominal
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -65,6 +66,73 @@ def _peaks():
     except Exception:
         return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
                 "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class NvmlClockSampler:
+    """SM clock, power and clock-event reasons sampled in-process every 2 ms
+    through NVML's read-only queries during the timed region (a thread; the
+    GPU is the torch device, matched by UUID)."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
+    PERIOD_S = 0.002
+
+    def __init__(self, torch_device: int):
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        import torch
+        uuid = str(torch.cuda.get_device_properties(torch_device).uuid)
+        try:
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(torch_device)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.rows = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _sample(self):
+        nv = self.nv
+        sm = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+        bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        return (time.monotonic(), sm, pw, [nm for nm, b in self.REASONS if bits & b])
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.rows.append(self._sample())
+            except Exception:
+                pass
+            time.sleep(self.PERIOD_S)
+
+    def start(self):
+        self.rows.append(self._sample())
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self.t_begin = time.monotonic()
+        self._t.start()
+
+    def stop(self) -> dict:
+        t_end = time.monotonic()
+        self._stop.set()
+        self._t.join(timeout=2)
+        inside = [r for r in self.rows if self.t_begin <= r[0] <= t_end] or self.rows[-3:]
+        sm = [r[1] for r in inside]
+        power = [r[2] for r in inside]
+        load = [x for x, pw in zip(sm, power) if pw > 200] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": self.max_mhz, "samples": len(inside),
+                "sampler": f"NVML in-process, every {self.PERIOD_S * 1e3:.0f} ms",
+                "region_ms": round(1e3 * (t_end - self.t_begin), 1), "power_w_max": max(power),
+                "sm_mhz_min": min(sm), "reasons": sorted(set(nm for r in inside for nm in r[3]))}
+
+
+def clock_sampler(torch_device: int):
+    """The NVML sampler when NVML answers, else nvidia-smi's 20 ms sampling."""
+    try:
+        return NvmlClockSampler(torch_device)
+    except Exception:
+        return ClockSampler(torch_device)
 
 
 class ClockSampler:
@@ -191,19 +259,40 @@ def _cpu_model() -> str:
     return platform.processor() or "unknown CPU"
 
 
+# The method's parameters both arms run with (vc_params_default, the oracle's defaults).
+METHOD_PARAMS = {"k": 8, "iters": 3, "rho": 0.005, "expcast_bias": 120}
+
+
+def bench_config(wl, vfmt: str, world: int) -> dict:
+    """The workload description printed by both arms (the same dict)."""
+    mb = 3 * wl.B * wl.H * wl.N * 128 * 2 / 1e6
+    return {"workload": wl.name, "vfmt": vfmt, "B": wl.B, "H": wl.H, "N": wl.N, "d": 128, **METHOD_PARAMS,
+            "step": "vc_attn_fwd with clustering in the call",
+            "l2": (f"inputs larger than L2 (Q, K, V bf16 = {mb:.0f} MB > 126 MB)" if mb > 126 else
+                   f"inputs fit in L2 (Q, K, V bf16 = {mb:.1f} MB): L2-warm timing"),
+            "parallelism": f"replicas x{world} (independent heads, no collective)"}
+
+
+def oracle_rows_per_head(N: int) -> int:
+    """The CPU legs' sampling rule: whole heads (every query row) up to N = 20000,
+    else 2048 evenly spaced rows per head."""
+    return N if N <= 20000 else 2048
+
+
 def cpu_oracle_sample(wl, x, rows_per_head: int = 96, heads=(0,), extra_flags: int = 0):
     """Time the oracle on a bounded sample and extrapolate to the workload.
 
-    For each sampled head: the full per-head prologue (k-means, quantization,
-    repair) plus `rows_per_head` query rows of the attention (all host cores).
-    Returns (TFLOPS extrapolated to the whole workload, cores, sample text,
-    seconds spent)."""
+    For each sampled head (flat index b*H + h): the full per-head prologue
+    (k-means, quantization, repair) plus `rows_per_head` query rows of the
+    attention (all host cores). Returns (TFLOPS extrapolated to the whole
+    workload, cores, sample text, seconds spent)."""
     import numpy as np
     import oracle
     cores = oracle.set_threads(os.cpu_count() or 1)
     t_pro = t_rows = 0.0
-    for h in heads:
-        q, k, v = x["q"][0, h], x["k"][0, h], x["v"][0, h]
+    for hf in heads:
+        b, h = divmod(hf, wl.H)
+        q, k, v = x["q"][b, h], x["k"][b, h], x["v"][b, h]
         t0 = time.perf_counter()
         flags = oracle.FLAGS_DEFAULT | extra_flags
         pro = oracle.head_prologue(q, k, v, flags=flags)
@@ -230,25 +319,33 @@ def cpu_oracle_sample(wl, x, rows_per_head: int = 96, heads=(0,), extra_flags: i
 
 
 def run_reference(args):
+    """The CPU oracle as the reference arm: every step times whole heads of the
+    workload (the cpu_baseline leg's sampling rule), cycling through the heads,
+    extrapolated per head to the workload; the value is the median over the
+    timed steps."""
     world, rank, _ = _dist_env()
     if world > 1 and rank != 0:
         return 0
     from bit_attention_diffusion_b200 import synth
-    wl, x = synth.make_by_name(WORKLOAD)
+    wl, x = synth.make_by_name(args.workload)
     vals = []
     cores = 1
     sample = ""
+    rows = oracle_rows_per_head(wl.N)
     for i in range(args.warmup + args.steps):
-        # one head's prologue + 512 query rows per step (enough rows to occupy every core)
-        tflops, cores, sample, secs = cpu_oracle_sample(wl, x, rows_per_head=512)
+        tflops, cores, sample, secs = cpu_oracle_sample(wl, x, rows_per_head=rows, heads=(i % (wl.B * wl.H),),
+                                                        extra_flags=VFMT_FLAGS[args.vfmt])
         if i >= args.warmup:
             vals.append(tflops)
     v = statistics.median(vals)
+    sample = (f"median of {args.steps} timed steps after {args.warmup} warm-up steps; each step: " + sample)
     line = {
-        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC if args.workload == WORKLOAD and args.vfmt == "e4m3" else
+        f"vc_attn_fwd TFLOPS (4N²dH/t) on {args.workload}, format {args.vfmt}",
+        "value": v, "unit": "TFLOPS", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.flops / (v * 1e12) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": WORKLOAD, "B": wl.B, "H": wl.H, "N": wl.N, "d": 128},
+        "data": "synthetic", "config": bench_config(wl, args.vfmt, 1),
         "cpu_baseline": {"value": v, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -294,7 +391,7 @@ def measure_video_variants(torch, vcattn, synth, stream, warmup, steps, world):
             step()
         vcattn.vc_attn_profile(True)
         torch.cuda.synchronize()
-        clocks = ClockSampler(torch.cuda.current_device())
+        clocks = clock_sampler(torch.cuda.current_device())
         clocks.start()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -349,6 +446,7 @@ def run_ours(args):
     q, k, v = (_to_dev(torch, x[n]) for n in "qkv")
     nvfp4 = args.vfmt != "e4m3"
     p = vcattn.params(flags=vcattn.FLAGS_DEFAULT | VFMT_FLAGS[args.vfmt])
+    assert (p.k, p.iters, round(p.rho, 6), p.expcast_bias) == tuple(METHOD_PARAMS.values()), "bench_config"
     ws, ws_bytes = vcattn.workspace(B, H, N, p)
     out = torch.empty_like(q)
 
@@ -371,7 +469,7 @@ def run_ours(args):
         step()
     vcattn.vc_attn_profile(True)
     barrier()
-    clocks = ClockSampler(dev)
+    clocks = clock_sampler(dev)
     clocks.start()
     launches0 = vcattn.vc_attn_launch_count()
     e0 = torch.cuda.Event(enable_timing=True)
@@ -529,9 +627,8 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu:
         # four whole heads (every query row) on the image workload: about 10-15 s
         # of oracle work; on larger workloads a bounded number of rows per head
-        rows = wl.N if wl.N <= 20000 else 2048
-        tf, cores, sample, _ = cpu_oracle_sample(wl, x, rows_per_head=rows, heads=(0, 1, 2, 3),
-                                                 extra_flags=VFMT_FLAGS[args.vfmt])
+        tf, cores, sample, _ = cpu_oracle_sample(wl, x, rows_per_head=oracle_rows_per_head(wl.N),
+                                                 heads=(0, 1, 2, 3), extra_flags=VFMT_FLAGS[args.vfmt])
         cpu = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample}
     variants = None
     if args.workload == WORKLOAD and not nvfp4:
@@ -548,8 +645,11 @@ def run_ours(args):
                     "peak": fp8_peak, "unit": "TFLOP/s",
                     "frac": (attn_tflops / fp8_peak) if attn_tflops else None,
                     "traffic": traffic,
-                    "peak_source": f"{peak_src}: 2 x {'sustained' if long_region else 'burst'} "
-                                   f"cuBLAS bf16 ({bf16_peak:.1f} TFLOP/s)",
+                    "peak_source": f"derived from {peak_src}: 2 x the {'sustained' if long_region else 'burst'} "
+                                   f"cuBLAS bf16 figure ({bf16_peak:.1f} TFLOP/s; nominal dense ratio FP8 : BF16 "
+                                   f"= 4.5 : 2.25 PFLOP/s)",
+                    "frac_of_nominal": (attn_tflops / NOMINAL_FP8_TFLOPS) if attn_tflops else None,
+                    "nominal_peak": NOMINAL_FP8_TFLOPS,
                     "algorithmic": "4*B*H*N^2*d FLOP per launch"}
         line = {
             "metric": metric, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
@@ -558,12 +658,7 @@ def run_ours(args):
             "dtype": DTYPE[args.vfmt],
             "data": "synthetic",
             "pct_of_fp8_peak": 100.0 * (value / world) / fp8_peak,
-            "config": {"workload": args.workload, "vfmt": args.vfmt, "B": B, "H": H, "N": N, "d": d, "k": p.k,
-                       "iters": p.iters,
-                       "rho": round(p.rho, 6), "expcast_bias": p.expcast_bias,
-                       "step": "vc_attn_fwd with clustering in the call",
-                       "l2": f"inputs larger than L2 (Q, K, V bf16 = {3 * q.numel() * 2 / 1e6:.0f} MB > 126 MB)",
-                       "parallelism": f"replicas x{world} (independent heads, no collective)"},
+            "config": bench_config(wl, args.vfmt, world),
             "phases_ms": {"cluster": float(ph_mean[0]), "quant_v_repair": float(ph_mean[1]),
                           "quant_qk_extra": float(ph_mean[2]), "attention": attn_ms,
                           "note": "quant_qk runs on a side stream during quant_v_repair; "

@@ -52,6 +52,7 @@ WsLayout make_layout(const Shape &s) {
   L.km_counter = take(BH * 4);
   L.vq_counter = take(BH * 4);
   L.kb_counter = take(BH * 4);
+  L.cleared = o;
   L.perm = take(BH * N * 4);
   L.labels = take(BH * N * 4);
   L.cent = take(BH * k * D * 4);
@@ -73,6 +74,28 @@ WsLayout make_layout(const Shape &s) {
   L.rep_idx = take(BH * std::max(s.R, 1) * 4);
   L.rep_delta = take(BH * std::max(s.R, 1) * D * 2);
   L.deltat = take(BH * D * std::max(s.Rpad, 1) * 2);
+  L.total = o;
+  return L;
+}
+
+// The scratch of the clustering alone, when the permutation and the centroids
+// are the caller's buffers: the status word and the k-means completion
+// counters (zeroed per call), the labels and the k-means partial sums.
+WsLayout make_cluster_layout(const Shape &s) {
+  WsLayout L{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + std::max<size_t>(bytes, 1));
+    return at;
+  };
+  const size_t BH = static_cast<size_t>(s.BH), N = static_cast<size_t>(s.N), k = static_cast<size_t>(s.k);
+  L.status = take(256);
+  L.km_counter = take(BH * 4);
+  L.cleared = o;
+  L.labels = take(BH * N * 4);
+  L.km_psum = take(BH * s.km_nblk * k * D * 8);
+  L.km_pcnt = take(BH * s.km_nblk * k * 4);
   L.total = o;
   return L;
 }
@@ -227,24 +250,42 @@ void prof_mark(int i, cudaStream_t s) {
 
 vc_status last_error() { return cudaGetLastError() == cudaSuccess ? VC_OK : VC_ERR_CUDA; }
 
-// One non-blocking side stream per device for the prologue work that runs
-// concurrently with the caller's stream (created on first use, kept for the
-// life of the process; ordering with the caller's stream is by events only).
-cudaStream_t side_stream() {
-  static std::mutex m;
-  static cudaStream_t streams[64] = {};
+// Streams and events the library keeps per device for the life of the
+// process, created on first use with that device current: the side stream of
+// vc_attn_fwd (Q/K quantization beside the clustering and the V passes) with
+// its fork, permutation-ready and join events, and the copy-in / copy-out
+// streams of vc_attn_fwd_host with their events. Ordering with the caller's
+// stream is by events only. Every call re-records the events, so a call holds
+// the device's mutex while it enqueues work on them: concurrent calls from
+// several host threads serialize on these streams.
+struct DevCtx {
+  std::mutex m_fwd, m_host;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev[3] = {};  // fork, permutation ready, join
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t hev[4] = {};  // start, copy-in done, compute done, last copy-out done
+};
+DevCtx g_devctx[64];
+
+DevCtx *dev_ctx() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> g(m);
-  if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
-    streams[dev] = nullptr;
-  return streams[dev];
+  return &g_devctx[dev];
+}
+
+// Create the missing streams / events (caller holds the matching mutex).
+bool make_stream(cudaStream_t *s) {
+  return *s || cudaStreamCreateWithFlags(s, cudaStreamNonBlocking) == cudaSuccess;
+}
+bool make_events(cudaEvent_t *ev, int n) {
+  for (int i = 0; i < n; ++i)
+    if (!ev[i] && cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) return false;
+  return true;
 }
 
 // Clear the completion counters and the status word at the start of a call.
 vc_status clear_small(const Ws &w, cudaStream_t s) {
-  // status and the per-(b,h) counters are the regions of the layout before perm
-  if (cudaMemsetAsync(w.base, 0, w.L.perm, s) != cudaSuccess) return VC_ERR_CUDA;
+  if (cudaMemsetAsync(w.base, 0, w.L.cleared, s) != cudaSuccess) return VC_ERR_CUDA;
   return VC_OK;
 }
 
@@ -515,17 +556,14 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
     // Either way they run concurrently with the V passes, and the attention
     // kernel waits for both streams. Per-call events, released once the work
     // completes.
-    cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};  // fork, permutation ready, join
-    cudaStream_t side = side_stream();
-    bool evok = side != nullptr;
-    for (int i = 0; i < 3 && evok; ++i) evok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
-    if (!evok) {
-      for (cudaEvent_t e : ev)
-        if (e) cudaEventDestroy(e);
+    DevCtx *dc = dev_ctx();
+    if (!dc) return VC_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(dc->m_fwd);
+    if (!make_stream(&dc->side) || !make_events(dc->ev, 3)) return VC_ERR_CUDA;
+    cudaStream_t side = dc->side;
+    const cudaEvent_t *ev = dc->ev;
+    if (cudaEventRecord(ev[0], s) != cudaSuccess || cudaStreamWaitEvent(side, ev[0], 0) != cudaSuccess)
       return VC_ERR_CUDA;
-    }
-    cudaEventRecord(ev[0], s);
-    cudaStreamWaitEvent(side, ev[0], 0);
     if (clusters) launch_quant_qk(sh, w, Qh, Kh, nullptr, q8, sq, k8, sk, side, QK_Q);
     const int32_t *pm = perm;
     if (clusters) {
@@ -535,15 +573,17 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
       pm = w.at<int32_t>(w.L.perm);
     }
     prof_mark(1, s);
-    cudaEventRecord(ev[1], s);
-    cudaStreamWaitEvent(side, ev[1], 0);
-    launch_quant_qk(sh, w, Qh, Kh, pm, q8, sq, k8, sk, side, clusters ? QK_K : QK_QK);
-    cudaEventRecord(ev[2], side);
-    launch_quant_v(sh, w, Vh, pm, v8t, vscale, w.at<uint16_t>(w.L.vmean), rep_idx, w.at<uint16_t>(w.L.rep_delta), s);
+    // from here on a failed record or wait returns after joining what was
+    // already forked, so that no work of this call stays unordered
+    bool evok = cudaEventRecord(ev[1], s) == cudaSuccess && cudaStreamWaitEvent(side, ev[1], 0) == cudaSuccess;
+    if (evok) launch_quant_qk(sh, w, Qh, Kh, pm, q8, sq, k8, sk, side, clusters ? QK_K : QK_QK);
+    const bool joined = cudaEventRecord(ev[2], side) == cudaSuccess;
+    if (evok && joined)
+      launch_quant_v(sh, w, Vh, pm, v8t, vscale, w.at<uint16_t>(w.L.vmean), rep_idx, w.at<uint16_t>(w.L.rep_delta),
+                     s);
     prof_mark(2, s);
-    cudaStreamWaitEvent(s, ev[2], 0);
+    if (!joined || cudaStreamWaitEvent(s, ev[2], 0) != cudaSuccess || !evok) return VC_ERR_CUDA;
     prof_mark(3, s);
-    for (cudaEvent_t e : ev) cudaEventDestroy(e);
   }
 
   const bool fp4 = (sh.flags & VC_VFMT_NVFP4) != 0;
@@ -672,25 +712,12 @@ vc_status vc_attn_fwd_host(const void *hQ, const void *hK, const void *hV, int B
   st = check_device();
   if (st != VC_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaStream_t s_in = nullptr, s_out = nullptr;
-  cudaEvent_t ev_start = nullptr, ev_in = nullptr, ev_out = nullptr, ev_done = nullptr;
-  auto release = [&]() {
-    if (ev_start) cudaEventDestroy(ev_start);
-    if (ev_in) cudaEventDestroy(ev_in);
-    if (ev_out) cudaEventDestroy(ev_out);
-    if (ev_done) cudaEventDestroy(ev_done);
-    if (s_in) cudaStreamDestroy(s_in);  // released once its work completes
-    if (s_out) cudaStreamDestroy(s_out);
-  };
-  if (cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) != cudaSuccess ||
-      cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) != cudaSuccess ||
-      cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&ev_out, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming) != cudaSuccess) {
-    release();
-    return VC_ERR_CUDA;
-  }
+  DevCtx *dc = dev_ctx();
+  if (!dc) return VC_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(dc->m_host);
+  if (!make_stream(&dc->s_in) || !make_stream(&dc->s_out) || !make_events(dc->hev, 4)) return VC_ERR_CUDA;
+  cudaStream_t s_in = dc->s_in, s_out = dc->s_out;
+  cudaEvent_t ev_start = dc->hev[0], ev_in = dc->hev[1], ev_out = dc->hev[2], ev_done = dc->hev[3];
   bool ok = cudaEventRecord(ev_start, s) == cudaSuccess && cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess &&
             cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess;
   const size_t head_bytes = static_cast<size_t>(N) * d * sizeof(uint16_t);
@@ -714,7 +741,6 @@ vc_status vc_attn_fwd_host(const void *hQ, const void *hK, const void *hV, int B
   // the caller's stream resumes after the last copy-out (also on an error path,
   // so that nothing of this call is left running unordered)
   const bool tail_ok = cudaEventRecord(ev_done, s_out) == cudaSuccess && cudaStreamWaitEvent(s, ev_done, 0) == cudaSuccess;
-  release();
   if (st != VC_OK) return st;
   return (ok && tail_ok) ? VC_OK : VC_ERR_CUDA;
 }
@@ -796,11 +822,9 @@ extern "C" vc_status vc_attn_cluster_noalloc(const void *V, int B, int H, int N,
   if (!V || !perm || !centroids || !aligned(V, 16) || !aligned(perm, 16) || !aligned(centroids, 16))
     return VC_ERR_INVALID_ARG;
   Shape sh = make_shape(B, H, N, *p, vc_attn_repair_count(N, p));
-  WsLayout L = make_layout(sh);
-  // clustering touches only the leading regions of the layout (status,
-  // counters, permutation, labels, centroids, k-means partial sums)
-  const size_t need = L.kbar_part;
-  if (need > kNoAllocScratchBytes) return VC_ERR_WORKSPACE;
+  // the clustering's own scratch only: perm and centroids are the caller's
+  WsLayout L = make_cluster_layout(sh);
+  if (L.total > kNoAllocScratchBytes) return VC_ERR_WORKSPACE;
   if ((st = check_device()) != VC_OK) return st;
   void *scratch = nullptr;
   if ((st = noalloc_scratch(&scratch)) != VC_OK) return st;
@@ -811,7 +835,16 @@ extern "C" vc_status vc_attn_cluster_noalloc(const void *V, int B, int H, int N,
   // the completion counters must start at zero; the array keeps the previous call's contents
   if ((st = clear_small(w, s)) != VC_OK) return st;
   launch_cluster(sh, w, static_cast<const uint16_t *>(V), perm, centroids, s);
-  return last_error();
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaErrorContextIsDestroyed || e == cudaErrorDeviceUninitialized || e == cudaErrorInvalidResourceHandle) {
+    // the context that held the array is gone: look its address up again next time
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+      std::lock_guard<std::mutex> lock(g_noalloc_mu);
+      g_noalloc_ptr[dev] = nullptr;
+    }
+  }
+  return e == cudaSuccess ? VC_OK : VC_ERR_CUDA;
 }
 
 extern "C" size_t vc_attn_cluster_noalloc_max_bytes(void) { return kNoAllocScratchBytes; }

@@ -37,6 +37,7 @@ struct WsLayout {
   size_t v8t, vscale, vexpo, vmean, amax_part, vq_counter, mut2, err;
   size_t rep_idx, rep_delta, deltat;
   size_t status;
+  size_t cleared;  // bytes [0, cleared) hold the status word and counters: zeroed when a call starts
   size_t total;
 };
 
@@ -44,6 +45,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 
 Shape make_shape(int B, int H, int N, const vc_params &p, int repair_count);
 WsLayout make_layout(const Shape &s);
+WsLayout make_cluster_layout(const Shape &s);
 
 // Bookkeeping: every launch in the library goes through this counter.
 void count_launch();

@@ -1248,8 +1248,10 @@ __global__ void __launch_bounds__(256) k_repair_delta4(const uint16_t *__restric
 // Grid-wide barrier of a cooperative launch: every block adds one to the
 // counter (zeroed at the start of the call) and waits until it holds
 // `target` = (barriers passed so far) x gridDim.x. Bounded: a wait that runs
-// out sets the timeout bit in the status word and the block leaves the kernel
-// (the other blocks then run out as well); nothing spins for ever.
+// out sets the timeout bit in the status word and the block leaves the
+// kernel; every waiting block reads that bit in its wait loop and leaves as
+// soon as it is set, so a failed call ends about one limit after the first
+// block gave up; nothing spins for ever.
 __device__ bool grid_barrier(unsigned *count, unsigned target, uint32_t *status) {
   __shared__ int s_ok;
   __syncthreads();
@@ -1264,6 +1266,12 @@ __device__ bool grid_barrier(unsigned *count, unsigned target, uint32_t *status)
       if (v >= target) break;
       if (clock64() - t0 > VC_WAIT_LIMIT_CYCLES) {
         atomicOr(status, ST_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      unsigned st;
+      asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(st) : "l"(status) : "memory");
+      if (st & ST_TIMEOUT) {  // another block already gave up: this barrier cannot complete
         ok = 0;
         break;
       }

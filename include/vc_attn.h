@@ -141,13 +141,20 @@ vc_status vc_attn_cluster(const void *V, int B, int H, int N, int d, const vc_pa
  * fixed 32 MiB array in device memory that the library reserves on every
  * GPU that loads it, until the process exits.
  *   Output: identical to vc_attn_cluster with the same arguments.
- *   Limit: shapes whose clustering scratch exceeds 32 MiB (see
- *   vc_attn_cluster_noalloc_max_bytes; about B*H*N <= 3.5 M tokens at k = 8,
- *   the 720p video workload included) return VC_ERR_WORKSPACE before any
- *   launch.
+ *   Limit: the scratch is 4 bytes per token (labels) plus the k-means
+ *   partial sums (8*k*128 bytes per k-means block, about max(B*H, 444)
+ *   blocks in all: 3.6 MB at k = 8 for up to 444 heads) and 256-byte-aligned
+ *   counters. Shapes
+ *   whose scratch exceeds 32 MiB (vc_attn_cluster_noalloc_max_bytes) return
+ *   VC_ERR_WORKSPACE before any launch: about B*H*N <= 7.4 M tokens at k = 8
+ *   (the 720p video workload, 3.0 M tokens, fits).
  *   Set-up: the first call on each device looks up the array's device
  *   address (cudaGetSymbolAddress) with that device current; make that first
- *   call before any stream capture.
+ *   call before any stream capture. cudaDeviceReset() ends the context that
+ *   holds the array and makes that address stale: a process that resets a
+ *   device must not call this entry point on it again. (A call that sees the
+ *   context gone drops the cached address, so the next call looks it up
+ *   again.)
  *   Calls allocate no memory (no cudaMalloc, cudaFree or allocating library
  *   routine). All calls share the one array and each call starts by clearing
  *   its counters; calls whose executions overlap on the GPU (other streams,
@@ -233,12 +240,14 @@ vc_status vc_attn_quant_v(const void *V, const int32_t *perm, int B, int H, int 
  * Restore) on the tensor cores in bf16; repair adds p * delta for the listed
  * tokens; O = scale_c * acc / l.
  * Q/K quantization runs on an internal non-blocking stream of the library
- * (one per device, created on first use), ordered by per-call events: when
- * the call clusters, the K channel means and Q start with the call (they do
- * not depend on the permutation) and K' follows the clustering; otherwise Q
- * and K' are one launch. Either way it overlaps the V passes; the call stays
- * stream-ordered with respect to the caller's stream and can be captured
- * into a CUDA graph.
+ * (one per device, created on first use with three events), ordered by
+ * events: when the call clusters, the K channel means and Q start with the
+ * call (they do not depend on the permutation) and K' follows the
+ * clustering; otherwise Q and K' are one launch. Either way it overlaps the
+ * V passes; the call stays stream-ordered with respect to the caller's
+ * stream and can be captured into a CUDA graph. Concurrent calls from
+ * several host threads on one device serialize on that side stream (a
+ * per-device lock is held while a call enqueues its work).
  * With VC_VFMT_NVFP4 (the 4-bit variant): the same frames, then per 16 keys
  * x = fma(acc, alpha/8, -F/8), p = 2^x, block scale sf = E4M3(448 * max p),
  * codes E2M1(p * fl(2688/sf)); O += P V4 on the block-scaled FP4 tensor cores
@@ -258,8 +267,10 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
  *   1. copies the run's Q, K and V slices host -> device;
  *   2. runs the forward on that run;
  *   3. copies the run's O slice back device -> host.
- * The copies go on two streams the call creates and releases, so the copy-in of
- * one run and the copy-out of another overlap the computation of a third.
+ * The copies go on two non-blocking streams the library keeps per device
+ * (created by the first call, with their events), so the copy-in of one run
+ * and the copy-out of another overlap the computation of a third. Concurrent
+ * calls from several host threads on one device serialize on them.
  *
  * Host buffers: hQ, hK, hV, hO, [B][H][N][d] bf16. They should be page-locked
  * (cudaHostAlloc or cudaHostRegister); pageable memory works but does not

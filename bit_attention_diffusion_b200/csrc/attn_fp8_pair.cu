@@ -16,8 +16,7 @@
 // probabilities), 128-255 from CTA 1; B split along N, the first half in CTA
 // 0's shared memory and the second in CTA 1's (each SM stages half of every K
 // and V tile); D in each SM's own TMEM. Per SM the TMEM holds one query tile:
-//   S0 [0,128), S1 [128,256)   two score buffers: QK^T(t+1) runs while the
-//                              softmax reads S(t)
+//   S0 [0,128), S1 [128,256)   two score buffers, S(t % 2) for KV tile t
 //   O  [256,384), RS [384,400) PV is one N = 144 product, B = [V | E], E a
 //                              16-row block whose row s (s = the V ring stage)
 //                              is E4M3 ones: column RS+s accumulates the row
@@ -31,12 +30,13 @@
 //   warp 1     allocates TMEM for the pair; in CTA 0 issues PV, the restores
 //              and the repair products.
 //   warp 2     in CTA 0 issues QK^T.
-//   warps 3-10 softmax: two warpgroups, thread (row r, half g) takes the 64
-//              keys [64g, 64g+64) of row r of every KV tile; the two halves of
-//              a row exchange their maxima through shared memory (an mbarrier
-//              per pair of warps, so that the wait is bounded) and take the
-//              same frame. Warpgroup 0 also keeps the row sums and the restore
-//              operands.
+//   warps 3-10 softmax: warpgroup w takes the KV tiles t = w, w+2, ... (score
+//              buffer S(w), probability slot P(w)), one thread per query row,
+//              all 128 keys; while one warpgroup turns the scores of tile t
+//              into bytes, the other reads tile t+1. The running frame goes
+//              from tile to tile through shared memory (published as soon as
+//              a warpgroup has its tile's maximum), each warpgroup keeps the
+//              row sums of its own tiles with their frames.
 // O is kept in "code units": O_acc = sum p * code + sum_t l_t * mean_t/s +
 // sum_R p * delta/s, and the epilogue writes O = s_c * O_acc / l.
 #include "common.cuh"
@@ -69,8 +69,10 @@ constexpr uint32_t OFF_MU = OFF_V + VS * SZ_VH;   // block-mean chunk; the repai
 constexpr uint32_t OFF_AR = OFF_MU + SZ_MUH;
 constexpr uint32_t OFF_LB = OFF_AR + SZ_AR;       // [LSLOTS][128] fp32 row sums
 constexpr uint32_t OFF_PREV = OFF_LB + LSLOTS * 128 * 4;  // [VS][128] last value read per row-sum column
-constexpr uint32_t OFF_XM = OFF_PREV + VS * 128 * 4;     // [2 tiles][2 halves][128] partial maxima
-constexpr uint32_t SMEM_USED = OFF_XM + 2 * 2 * 128 * 4;
+constexpr uint32_t OFF_FS = OFF_PREV + VS * 128 * 4;     // [LSLOTS][128] frame of each row-sum slot
+constexpr uint32_t OFF_F = OFF_FS + LSLOTS * 128 * 4;     // [3][128] frame hand-over (two tiles, final)
+constexpr uint32_t OFF_LT1 = OFF_F + 3 * 128 * 4;         // [2][128] warpgroup 1's row sum and its frame
+constexpr uint32_t SMEM_USED = OFF_LT1 + 2 * 128 * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // alignment slack
 static_assert(VS <= 16, "one row-sum column per V stage");
 static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && SZ_VH % 1024 == 0 && OFF_MU % 1024 == 0 &&
@@ -92,7 +94,8 @@ constexpr uint16_t PAIR = 3;                                              // bot
 struct BarsPair {
   uint64_t q, kfull[KS], kempty[KS], vfull[VS], vempty[VS], mufull, muempty;
   uint64_t sfull[2], sfree[2], pfull[2], pvdone[2];
-  uint64_t xbar[2][4];  // per score buffer and pair of softmax warps: both halves' maxima written
+  uint64_t fbar[2][4];   // per warpgroup and 32-row group: the frame of its latest tile published
+  uint64_t lslot[4];     // per 32-row group: warpgroup 0 wrote the row sum that completes a chunk
   uint64_t epi, rdone, repk, repp, repdone, dt, main, fin, drain;
 };
 
@@ -159,7 +162,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
   uint8_t *sAr = sm + OFF_AR;
   float *sLb = reinterpret_cast<float *>(sm + OFF_LB);      // [LSLOTS][128]
   float *sPrev = reinterpret_cast<float *>(sm + OFF_PREV);  // [VS][128]
-  float *sXm = reinterpret_cast<float *>(sm + OFF_XM);      // [2][2][128]
+  float *sFs = reinterpret_cast<float *>(sm + OFF_FS);      // [LSLOTS][128]
+  float *sF = reinterpret_cast<float *>(sm + OFF_F);        // [3][128]
+  float *sLt1 = reinterpret_cast<float *>(sm + OFF_LT1);    // [2][128]
   __shared__ BarsPair bars;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
@@ -194,11 +199,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
     mbar_init(&bars.muempty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.sfull[i], 1);
-      mbar_init(&bars.sfree[i], 16);  // 8 softmax warps x 2 CTAs
-      mbar_init(&bars.pfull[i], 16);
+      mbar_init(&bars.sfree[i], 8);  // one warpgroup (4 warps) x 2 CTAs
+      mbar_init(&bars.pfull[i], 8);
       mbar_init(&bars.pvdone[i], 1);
-      for (int j = 0; j < 4; ++j) mbar_init(&bars.xbar[i][j], 2);  // the two warps of a row pair
+      for (int j = 0; j < 4; ++j) mbar_init(&bars.fbar[i][j], 1);  // the warp of those rows
     }
+    for (int j = 0; j < 4; ++j) mbar_init(&bars.lslot[j], 1);
     mbar_init(&bars.epi, 8);   // warpgroup 0 of both CTAs
     mbar_init(&bars.rdone, 1);
     mbar_init(&bars.repk, 8);
@@ -235,12 +241,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
   tc_fence_after();
   const uint32_t tmem = s_tmem;
 
-  // Bounded wait, cluster-scope acquire; the abort flag (set by a warp whose
-  // wait ran out) is read only when the phase is not complete yet.
+  // Bounded wait; the abort flag (set by a warp whose wait ran out) is read
+  // only when the phase is not complete yet.
   auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
-    if (mbar_try_wait_cl(smem_u32(bar), parity)) return true;
+    if (mbar_try_wait(smem_u32(bar), parity)) return true;
     if (s_abort) return false;
-    if (!mbar_wait_cl(bar, parity)) {
+    if (!mbar_wait(bar, parity)) {
       s_abort = 1;
       atomicOr(p.status, ST_TIMEOUT);
       return false;
@@ -405,45 +411,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax (both CTAs)
-    const int g = (warp - 3) >> 2;  // key half
+    // Warpgroup w takes the KV tiles t = w, w+2, w+4, ... (score buffer and
+    // probability slot w), one thread per query row and all 128 keys. The
+    // running frame is handed from tile to tile through shared memory: the
+    // warpgroup of tile t publishes F_t as soon as it has the tile maximum.
+    const int w = (warp - 3) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lrow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);  // this warp's lanes
     const float sqs = active ? p.sq[static_cast<size_t>(bh) * T + qt] : 0.0f;
     const float *skh = p.sk + static_cast<size_t>(bh) * T;
     const int tail = p.N - (T - 1) * 128;  // valid keys in the last tile
-    const uint32_t sfree_cl[2] = {at0(&bars.sfree[0]), at0(&bars.sfree[1])};
-    const uint32_t pfull_cl[2] = {at0(&bars.pfull[0]), at0(&bars.pfull[1])};
+    const uint32_t sfree_cl = at0(&bars.sfree[w]), pfull_cl = at0(&bars.pfull[w]);
     bool ok = true;
-    float F = -INFINITY;  // frame of the latest tile
-    float lt = 0.0f;      // warpgroup 0: the row sums read so far, frame F
-    int nread = 0;        // warpgroup 0: tiles whose row sum has been read
+    float Fown = -INFINITY;  // frame of this warpgroup's latest tile
+    float lt = 0.0f;         // row sums of this warpgroup's tiles read so far, in frame Flt
+    float Flt = -INFINITY;
     auto wwait = [&](uint64_t *bar, uint32_t parity) -> bool {
-      const bool w = wait(bar, parity);
-      return __all_sync(0xFFFFFFFFu, w);
+      const bool v = wait(bar, parity);
+      return __all_sync(0xFFFFFFFFu, v);
     };
-    // l_u: what PV(u) added to row-sum column u % VS (PV(u) complete, PV(u+VS)
-    // not issued), into slot u % LSLOTS and lt
-    auto read_l = [&](int u) {
-      const int col = u % VS;
+    // l_u of this warpgroup's tile u (PV(u) complete, PV(u+VS) not issued):
+    // what PV(u) added to row-sum column u % VS, into slot u % LSLOTS with
+    // its frame Fu, and into lt
+    auto read_l = [&](int u, float Fu) {
+      const int col = u % VS;  // columns of even tiles are warpgroup 0's, of odd tiles warpgroup 1's
       const float v = __uint_as_float(tmem_ld1(lrow + TM_RS + col));
       tmem_wait_ld();
       const float l = __fsub_rn(v, sPrev[col * 128 + r]);
       sPrev[col * 128 + r] = v;
       sLb[(u % LSLOTS) * 128 + r] = l;
+      sFs[(u % LSLOTS) * 128 + r] = Fu;
+      if (Fu != Flt) {
+        lt = Flt == -INFINITY ? 0.0f : lt * frame_scale(Flt, Fu);
+        Flt = Fu;
+      }
       lt += l;
     };
-    // restore A operand, row r = [hi(l) | lo(l)] of the chunk's 32 tiles in bf16
-    auto flush = [&](int X, int nvalid) {
+    // restore A operand, row r = [hi(l) | lo(l)] of the chunk's tiles in bf16,
+    // every slot moved from its own frame into frame Fto (O's frame when the
+    // restore runs)
+    auto flush = [&](int X, int nvalid, float Fto) {
       uint32_t hw[16], lw[16];
-      const float *base = sLb + ((32 * X) % LSLOTS) * 128 + r;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float l0 = (2 * i < nvalid) ? base[(2 * i) * 128] : 0.0f;
-        const float l1 = (2 * i + 1 < nvalid) ? base[(2 * i + 1) * 128] : 0.0f;
-        const __nv_bfloat16 h0 = __float2bfloat16_rn(l0), h1 = __float2bfloat16_rn(l1);
-        const __nv_bfloat16 o0 = __float2bfloat16_rn(__fsub_rn(l0, __bfloat162float(h0)));
-        const __nv_bfloat16 o1 = __float2bfloat16_rn(__fsub_rn(l1, __bfloat162float(h1)));
+        float lv[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int slot = (32 * X + 2 * i + e) % LSLOTS;
+          lv[e] = (2 * i + e < nvalid) ? sLb[slot * 128 + r] * frame_scale(sFs[slot * 128 + r], Fto) : 0.0f;
+        }
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(lv[0]), h1 = __float2bfloat16_rn(lv[1]);
+        const __nv_bfloat16 o0 = __float2bfloat16_rn(__fsub_rn(lv[0], __bfloat162float(h0)));
+        const __nv_bfloat16 o1 = __float2bfloat16_rn(__fsub_rn(lv[1], __bfloat162float(h1)));
         hw[i] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
         lw[i] = static_cast<uint32_t>(__bfloat16_as_ushort(o0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(o1)) << 16);
       }
@@ -456,125 +476,155 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
       }
     };
 
-    // One KV tile t. LAST: the ragged last tile.
+    // One KV tile t (t % 2 == w). LAST: the ragged last tile.
     auto tile = [&](int t, auto last_tag) -> bool {
       constexpr bool LAST = decltype(last_tag)::value;
-      const int b = t & 1;
       const float skt = skh[t];
-      if (!wwait(&bars.sfull[b], (t >> 1) & 1)) return false;
+      if (!wwait(&bars.sfull[w], (t >> 1) & 1)) return false;
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(lrow + tm_s(b) + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(lrow + tm_s(b) + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      uint32_t sr[128];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tmem_ld32(lrow + tm_s(w) + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * i]));
       tmem_wait_ld();
       tc_fence_before();
-      warp_arrive_cl(sfree_cl[b]);  // S(b) may take the scores of tile t+2
-      float s[64];
+      warp_arrive_cl(sfree_cl);  // S(w) may take the scores of tile t+2
+      const float Fprev_own = Fown;  // frame of this warpgroup's previous tile, t-2
+      float s[128];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) s[j] = __uint_as_float(sr[j]);
+      for (int j = 0; j < 128; ++j) s[j] = __uint_as_float(sr[j]);
       if constexpr (LAST) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j)
-          if (64 * g + j >= tail) s[j] = -INFINITY;
+        for (int j = 0; j < 128; ++j)
+          if (j >= tail) s[j] = -INFINITY;
       }
-      float pm;
+      float mx;
       {
-        float mm[22];
+        float mm[43];
 #pragma unroll
-        for (int j = 0; j < 21; ++j) mm[j] = max3(s[3 * j], s[3 * j + 1], s[3 * j + 2]);
-        mm[21] = s[63];
+        for (int j = 0; j < 42; ++j) mm[j] = max3(s[3 * j], s[3 * j + 1], s[3 * j + 2]);
+        mm[42] = fmaxf(s[126], s[127]);
 #pragma unroll
-        for (int j = 0; j < 7; ++j) mm[j] = max3(mm[3 * j], mm[3 * j + 1], mm[3 * j + 2]);
-        mm[7] = mm[21];
-        pm = fmaxf(max3(mm[0], mm[1], mm[2]), max3(mm[3], mm[4], max3(mm[5], mm[6], mm[7])));
+        for (int j = 0; j < 14; ++j) mm[j] = max3(mm[3 * j], mm[3 * j + 1], mm[3 * j + 2]);
+        mm[14] = mm[42];
+#pragma unroll
+        for (int j = 0; j < 5; ++j) mm[j] = max3(mm[3 * j], mm[3 * j + 1], mm[3 * j + 2]);
+        mx = max3(mm[0], mm[1], fmaxf(mm[2], fmaxf(mm[3], mm[4])));
       }
-      // the row's maximum: this half's and the other half's (the two warps
-      // that share these rows meet on a barrier of their own)
-      sXm[(b * 2 + g) * 128 + r] = pm;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.xbar[b][q4]);
-      if (!wwait(&bars.xbar[b][q4], (t >> 1) & 1)) return false;
-      const float mx = fmaxf(pm, sXm[(b * 2 + (g ^ 1)) * 128 + r]);
       const float alpha = __fmul_rn(__fmul_rn(sqs, skt), p.kappa);
-      // F_t = max(F_{t-1}, 8 ceil(m_t / 8)): 8 ceil(running max / 8)
-      const float Fn = fmaxf(F, 8.0f * ceilf(__fmul_rn(mx, alpha) * 0.125f));
-      const bool need = t > 0 && Fn != F;
-      const float sc = need ? frame_scale(F, Fn) : 1.0f;
-      uint32_t w[16];
+      // F_t = max(F_{t-1}, 8 ceil(m_t / 8)): 8 ceil(running max / 8), with
+      // F_{t-1} from the other warpgroup
+      float Fp = -INFINITY;
+      if (t > 0) {
+        if (!wwait(&bars.fbar[w ^ 1][q4], ((t - 1) >> 1) & 1)) return false;
+        Fp = sF[(w ^ 1) * 128 + r];
+      }
+      const float Fn = fmaxf(Fp, 8.0f * ceilf(__fmul_rn(mx, alpha) * 0.125f));
+      sF[w * 128 + r] = Fn;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.fbar[w][q4]);
+      uint32_t wb[32];
       {
         const float al24 = alpha * TWO_M24;
         const float c24 = (static_cast<float>(p.C) - Fn) * TWO_M24;
 #pragma unroll
-        for (int q = 0; q < 16; ++q) w[q] = expcast4(&s[4 * q], al24, c24);
+        for (int q = 0; q < 32; ++q) wb[q] = expcast4(&s[4 * q], al24, c24);
         if constexpr (LAST) {
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
+          for (int q = 0; q < 32; ++q) {
             uint32_t keep = 0u;
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              if (64 * g + 4 * q + e < tail) keep |= 0xFFu << (8 * e);
-            w[q] &= keep;
+              if (4 * q + e < tail) keep |= 0xFFu << (8 * e);
+            wb[q] &= keep;
           }
         }
       }
-      // PV(t-2) complete: slot P(b) is free and l_{t-2} can be read
-      if (t >= 2 && !wwait(&bars.pvdone[b], ((t >> 1) - 1) & 1)) return false;
+      // this warpgroup's previous tile: PV(t-2) complete, slot P(w) free, its
+      // row sum readable (waited for only now, so that the PV has had the
+      // whole tile to complete)
+      if (t >= 2) {
+        if (!wwait(&bars.pvdone[w], ((t >> 1) - 1) & 1)) return false;
+        tc_fence_after();
+        read_l(t - 2, Fprev_own);
+        if (w == 0 && t >= 32 && ((t - 32) & 31) == 0) {
+          // l_{t-2} completes chunk (t-32)/32 on this side; warpgroup 1
+          // flushes it at tile t+1
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.lslot[q4]);
+        }
+      }
+      const bool need = t > 0 && Fn != Fp;
       if (__any_sync(0xFFFFFFFFu, need)) {
-        // the frame moves: O and every row sum read so far go into frame Fn;
-        // PV(t-1) must be complete (O stable, l_{t-1} readable)
-        if (t >= 1 && !wwait(&bars.pvdone[b ^ 1], ((t - 1) >> 1) & 1)) return false;
+        // the frame moves: O (PV(0..t-1), frame F_{t-1}) goes into frame Fn
+        // before PV(t); PV(t-1) must be complete (PV(t-2) is, so that
+        // barrier is at most one phase behind)
+        if (!wwait(&bars.pvdone[w ^ 1], ((t - 1) >> 1) & 1)) return false;
         tc_fence_after();
-        if (g == 0) {
-          for (; nread < t; ++nread) read_l(nread);
-          if (need) {
-            lt *= sc;
-            for (int i = 0; i < LSLOTS; ++i) sLb[i * 128 + r] *= sc;
-          }
-        }
-        uint32_t o[64];
-        tmem_ld32(lrow + TM_O + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
-        tmem_ld32(lrow + TM_O + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
-        tmem_wait_ld();
+        const float sc = need ? frame_scale(Fp, Fn) : 1.0f;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * sc);
-        tmem_st32(lrow + TM_O + 64 * g, *reinterpret_cast<const uint32_t(*)[32]>(&o[0]));
-        tmem_st32(lrow + TM_O + 64 * g + 32, *reinterpret_cast<const uint32_t(*)[32]>(&o[32]));
-      } else if (g == 0 && t >= 2 && nread <= t - 2) {
-        tc_fence_after();
-        read_l(t - 2);
-        nread = t - 1;
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t o[64];
+          tmem_ld32(lrow + TM_O + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+          tmem_ld32(lrow + TM_O + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 64; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * sc);
+          tmem_st32(lrow + TM_O + 64 * hf, *reinterpret_cast<const uint32_t(*)[32]>(&o[0]));
+          tmem_st32(lrow + TM_O + 64 * hf + 32, *reinterpret_cast<const uint32_t(*)[32]>(&o[32]));
+        }
       }
-      if (g == 0 && t >= 33 && ((t - 33) & 31) == 0) {
-        // chunk (t-33)/32 is complete (its last tile, t-2, has been read): its
-        // row sums in frame Fn for the restore issued right before PV(t)
-        flush((t - 33) >> 5, 32);
+      if (t >= 33 && ((t - 33) & 31) == 0) {
+        // (t odd: warpgroup 1) chunk (t-33)/32 is complete: l_{t-2} was read
+        // above, l_{t-3} by warpgroup 0 at tile t-1 (lslot); its row sums in
+        // frame Fn for the restore issued right before PV(t)
+        if (!wwait(&bars.lslot[q4], ((t - 33) >> 5) & 1)) return false;
+        flush((t - 33) >> 5, 32, Fn);
         fence_proxy_async_smem();
       }
-      tmem_st16(lrow + tm_p(b) + 16 * g, w);
+      tmem_st32(lrow + tm_p(w), wb);
       tmem_wait_st();  // the bytes and any O rescale are in TMEM
       tc_fence_before();
-      warp_arrive_cl(pfull_cl[b]);
-      F = Fn;
+      warp_arrive_cl(pfull_cl);
+      Fown = Fn;
       return true;
     };
 
     const bool ragged = tail < 128;
-    for (int t = 0; t < T - 1 && ok; ++t) ok = tile(t, std::false_type{});
-    if (ok) ok = ragged ? tile(T - 1, std::true_type{}) : tile(T - 1, std::false_type{});
-    // every product of the loop is complete once PV(T-1) is
+    for (int t = w; t < T - 1 && ok; t += 2) ok = tile(t, std::false_type{});
+    if (ok && ((T - 1) & 1) == w) ok = ragged ? tile(T - 1, std::true_type{}) : tile(T - 1, std::false_type{});
+    // every product of the loop is complete once PV(T-1) is. Parity waits
+    // only tell the current phase from the one before, so each warpgroup
+    // first waits for the PV of its own last tile (its barrier is then at most
+    // that phase behind); after that PV(T-2) is complete, and with it every
+    // earlier product, so PV(T-1)'s barrier cannot be two phases behind.
+    const int tlast = ((T - 1 - w) & ~1) + w;  // this warpgroup's last tile (if w < T)
+    if (ok && w < T) ok = wwait(&bars.pvdone[w], (tlast >> 1) & 1);
     if (ok) ok = wwait(&bars.pvdone[(T - 1) & 1], ((T - 1) >> 1) & 1);
-    if (ok && g == 0) {
+    if (ok && w < T) {
       tc_fence_after();
-      for (; nread < T; ++nread) read_l(nread);
+      read_l(tlast, Fown);
+    }
+    if (w == 1) {
+      sLt1[r] = lt;
+      sLt1[128 + r] = Flt;
+    }
+    if (((T - 1) & 1) == w) sF[2 * 128 + r] = Fown;  // the final frame F_{T-1}
+    softmax_bar256();
+    const float F = sF[2 * 128 + r];
+    if (ok && w == 0) {
+      // the row sum over all tiles, in the final frame
+      const float l0 = Flt == -INFINITY ? 0.0f : lt * frame_scale(Flt, F);
+      const float F1 = sLt1[128 + r];
+      const float l1 = F1 == -INFINITY ? 0.0f : sLt1[r] * frame_scale(F1, F);
+      s_lt[r] = __fadd_rn(l0, l1);
       const uint32_t epi_cl = at0(&bars.epi);
       for (int X = X0; X <= X_last && ok; ++X) {
-        flush(X, min(32, T - 32 * X));
+        flush(X, min(32, T - 32 * X), F);
         fence_proxy_async_smem();
         tc_fence_before();
         warp_arrive_cl(epi_cl);
         ok = wwait(&bars.rdone, (X - X0) & 1);  // the restore operand is read before the next flush
       }
-      s_lt[r] = lt;
     }
 
     // ---------------------------------------------------------- repair
@@ -584,6 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
     // columns of the bf16 probabilities over the V ring. Every softmax thread
     // takes the same barriers on every path.
     softmax_bar256();
+    const int g = w;  // key half of the repair scores
     const float c24f = (static_cast<float>(p.C) - F) * TWO_M24;
     uint8_t *prep = sV + g * (128 * 128);
     const uint32_t repk_cl = at0(&bars.repk), repp_cl = at0(&bars.repp);
@@ -613,17 +664,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
         s_skR[r] = i < p.R ? skh[p.rep_idx[static_cast<size_t>(bh) * p.R + i] >> 7] : 0.0f;
       }
       softmax_bar256();  // s_skR visible to both warpgroups
-      if (!ok) continue;
       const int u = T + rc, b = u & 1;
-      ok = wwait(&bars.sfull[b], (u >> 1) & 1);
-      if (!ok) continue;
-      tc_fence_after();
       uint32_t sv[64];
-      tmem_ld32(lrow + tm_s(b) + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(lrow + tm_s(b) + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      warp_arrive_cl(sfree_cl[b]);
+      bool got = false;
+      if (ok) {
+        ok = wwait(&bars.sfull[b], (u >> 1) & 1);
+        if (ok) {
+          tc_fence_after();
+          tmem_ld32(lrow + tm_s(b) + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(lrow + tm_s(b) + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_wait_ld();
+          tc_fence_before();
+          got = true;
+        }
+      }
+      // both halves of S(b) are read: warpgroup 0 releases it for both (the
+      // barrier counts one warpgroup per CTA)
+      softmax_bar256();
+      if (g == 0) warp_arrive_cl(at0(&bars.sfree[b]));
+      if (!got) continue;
       const int nval = min(128, p.R - rc * 128);
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
@@ -666,7 +725,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
   if (lead && (warp == 1 || warp == 2)) {
     // bounded: after a timeout there is nothing more to do for products that
     // never complete
-    mbar_wait_cl(&bars.drain, 0);
+    mbar_wait(&bars.drain, 0);
   }
   if (s_abort) {
     // a wait ran out: give copies still in flight a moment to land before the

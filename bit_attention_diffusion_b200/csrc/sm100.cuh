@@ -261,38 +261,14 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
-// Arrive on an mbarrier given by its shared::cluster address (own or peer CTA),
-// releasing this thread's prior writes at cluster scope.
+// Arrive on an mbarrier given by its shared::cluster address (own or peer CTA).
+// The data the pair hands over this way is either in TMEM (ordered by the
+// tcgen05 fences around the arrive and the wait) or shared memory that only
+// the tensor cores read (made visible to them by fence.proxy.async before the
+// arrive), so the default CTA-scope semantics suffice; cluster scope costs
+// a full cluster-wide fence per arrive and per wait.
 __device__ __forceinline__ void mbar_arrive_cl(uint32_t cl_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx_cl(uint32_t cl_addr, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cl_addr),
-               "r"(bytes)
-               : "memory");
-}
-// try_wait with acquire at cluster scope: for barriers that other CTAs of the
-// cluster arrive at (or whose transaction bytes another CTA's copies complete).
-__device__ __forceinline__ bool mbar_try_wait_cl(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_cl(uint64_t *bar, uint32_t parity, long long limit = VC_WAIT_LIMIT_CYCLES) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait_cl(a, parity)) return true;
-  const long long t0 = clock64();
-  uint32_t n = 0;
-  while (true) {
-    if (mbar_try_wait_cl(a, parity)) return true;
-    if ((++n & 255u) == 0u && clock64() - t0 > limit) return false;
-  }
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
 }
 // Whole-cluster barrier (every thread of both CTAs, converged warps).
 __device__ __forceinline__ void cluster_sync_all() {

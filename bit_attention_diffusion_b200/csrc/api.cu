@@ -2,7 +2,6 @@
 // validation, workspace layout, TMA tensor maps and kernel launches.
 #include <atomic>
 #include <cmath>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -168,8 +167,6 @@ vc_status check_device() {
     if (ok_cache[dev] == 1) {
       if (cudaFuncSetAttribute(k_vc_attn_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(attn_fp8_smem_bytes())) != cudaSuccess ||
-          cudaFuncSetAttribute(k_vc_attn_fwd_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(attn_fp8_pair_smem_bytes())) != cudaSuccess ||
           cudaFuncSetAttribute(k_attn_ref_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(attn_bf16_smem_bytes())) != cudaSuccess ||
           cudaFuncSetAttribute(k_kmeans_pass, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -426,16 +423,6 @@ vc_status launch_prologue_fused(const Shape &sh, const Ws &w, const uint16_t *Q,
   return VC_OK;
 }
 
-// Development switch between the two FP8 attention kernels (SM pairs by
-// default; VC_ATTN_SINGLE_SM=1 selects the one-SM kernel), read once.
-bool use_pair_kernel() {
-  static const bool pair = [] {
-    const char *e = std::getenv("VC_ATTN_SINGLE_SM");
-    return !(e && e[0] == '1');
-  }();
-  return pair;
-}
-
 float kappa_of(float softmax_scale) {
   return static_cast<float>(8.0 * 1.4426950408889634074 * static_cast<double>(softmax_scale));
 }
@@ -661,26 +648,7 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
   ap.k8 = k8;
   ap.O = static_cast<uint16_t *>(O);
   ap.status = w.at<uint32_t>(w.L.status);
-  if (use_pair_kernel()) {
-    CUtensorMap tkh, tv0, tv1, tmuh, tdth;
-    ok = map2d(&tkh, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, rows, 128, 64) &&
-         map2d(&tv0, v8t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, sh.Npad, static_cast<uint64_t>(sh.BH) * 128, 128, 72) &&
-         map2d(&tv1, v8t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, sh.Npad, static_cast<uint64_t>(sh.BH) * 128, 128, 56) &&
-         map2d(&tmuh, w.at<uint16_t>(w.L.mut2), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64,
-               static_cast<uint64_t>(sh.BH) * sh.nch32 * 128, 64, 64);
-    if (ok) {
-      if (sh.R > 0)
-        ok = map2d(&tdth, w.at<uint16_t>(w.L.deltat), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sh.Rpad,
-                   static_cast<uint64_t>(sh.BH) * 128, 64, 64);
-      else
-        tdth = tmuh;  // unused when R == 0
-    }
-    if (!ok) return VC_ERR_CUDA;
-    k_vc_attn_fwd_pair<<<dim3(2 * ((sh.Nb + 1) / 2), sh.BH), 352, attn_fp8_pair_smem_bytes(), s>>>(
-        tq, tkh, tv0, tv1, tmuh, tdth, ap);
-  } else {
-    k_vc_attn_fwd<<<dim3((sh.Nb + 1) / 2, sh.BH), 352, attn_fp8_smem_bytes(), s>>>(tq, tk, tv, tmu, tdt, ap);
-  }
+  k_vc_attn_fwd<<<dim3((sh.Nb + 1) / 2, sh.BH), 352, attn_fp8_smem_bytes(), s>>>(tq, tk, tv, tmu, tdt, ap);
   count_launch();
   prof_mark(4, s);
   if (g_prof.on) ++g_prof.calls;

@@ -22,15 +22,4 @@ __global__ void k_vc_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __g
                               const __grid_constant__ CUtensorMap tmDT, const AttnFp8Params p);
 uint32_t attn_fp8_smem_bytes();
 
-// The same forward on clusters of two CTAs (the two SMs of a pair, tcgen05
-// cta_group::2): grid 2*ceil(Nb/2) x B*H, CTA x takes query tile x. Maps: Q
-// tiles (128 x 128 bytes), K half tiles (64 rows), V channel-major half tiles
-// (72 rows for the even CTA, 56 for the odd one), block-mean half chunks and
-// repair-delta tiles (64 bf16 x 64 rows).
-__global__ void k_vc_attn_fwd_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                                   const __grid_constant__ CUtensorMap tmV0, const __grid_constant__ CUtensorMap tmV1,
-                                   const __grid_constant__ CUtensorMap tmMu, const __grid_constant__ CUtensorMap tmDT,
-                                   const AttnFp8Params p);
-uint32_t attn_fp8_pair_smem_bytes();
-
 }  // namespace vc

@@ -181,6 +181,10 @@ vc_status check_device() {
                                static_cast<int>(attn_fp4_smem_bytes(true))) != cudaSuccess ||
           cudaFuncSetAttribute(k_kmeans_pass8, cudaFuncAttributeMaxDynamicSharedMemorySize, KMEANS8_SMEM) !=
               cudaSuccess ||
+          cudaFuncSetAttribute(k_kmeans_pass8tc, cudaFuncAttributeMaxDynamicSharedMemorySize, KMEANS8TC_SMEM) !=
+              cudaSuccess ||
+          cudaFuncSetAttribute(k_kmeans_pass8tc, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
           cudaFuncSetAttribute(k_prologue_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, FUSED_SMEM) !=
               cudaSuccess) {
         ok_cache[dev] = 0;
@@ -289,8 +293,13 @@ vc_status clear_small(const Ws &w, cudaStream_t s) {
   return VC_OK;
 }
 
-void launch_cluster(const Shape &sh, const Ws &w, const uint16_t *V, int32_t *perm, float *cent, cudaStream_t s) {
+vc_status launch_cluster(const Shape &sh, const Ws &w, const uint16_t *V, int32_t *perm, float *cent,
+                         cudaStream_t s) {
   int32_t *labels = w.at<int32_t>(w.L.labels);
+  CUtensorMap tmv;
+  if (sh.k <= 8 &&
+      !map2d(&tmv, V, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, static_cast<uint64_t>(sh.BH) * sh.N, 64, TILE))
+    return VC_ERR_CUDA;
   if (!(sh.flags & VC_WARMSTART)) {  // warm start: cent already holds the previous step's centroids
     k_kmeans_init<<<sh.BH, 128, 0, s>>>(V, sh.N, sh.k, cent);
     count_launch();
@@ -299,9 +308,10 @@ void launch_cluster(const Shape &sh, const Ws &w, const uint16_t *V, int32_t *pe
   const dim3 grid(sh.km_nblk, sh.BH);
   for (int it = 0; it <= sh.iters; ++it) {
     if (sh.k <= 8)
-      k_kmeans_pass8<<<grid, 256, KMEANS8_SMEM, s>>>(V, sh.N, sh.k, sh.km_cpb, sh.km_nblk, cent, labels,
-                                          w.at<double>(w.L.km_psum), w.at<int>(w.L.km_pcnt),
-                                          w.at<unsigned>(w.L.km_counter), it < sh.iters ? 1 : 0);
+      k_kmeans_pass8tc<<<grid, 256, KMEANS8TC_SMEM, s>>>(tmv, sh.N, sh.k, sh.km_cpb, sh.km_nblk, cent, labels,
+                                                         w.at<double>(w.L.km_psum), w.at<int>(w.L.km_pcnt),
+                                                         w.at<unsigned>(w.L.km_counter), it < sh.iters ? 1 : 0,
+                                                         w.at<uint32_t>(w.L.status));
     else
       k_kmeans_pass<<<grid, 128, smem, s>>>(V, sh.N, sh.k, sh.km_cpb, sh.km_nblk, cent, labels,
                                             w.at<double>(w.L.km_psum), w.at<int>(w.L.km_pcnt),
@@ -310,6 +320,7 @@ void launch_cluster(const Shape &sh, const Ws &w, const uint16_t *V, int32_t *pe
   }
   k_perm_sort<<<sh.BH, 1024, 0, s>>>(labels, sh.N, sh.k, perm);
   count_launch();
+  return VC_OK;
 }
 
 // parts: QK_Q = the K channel means and Q (no permutation needed), QK_K = K'
@@ -480,7 +491,9 @@ vc_status vc_attn_cluster(const void *V, int B, int H, int N, int d, const vc_pa
   if ((st = check_device()) != VC_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((st = clear_small(w, s)) != VC_OK) return st;
-  launch_cluster(sh, w, static_cast<const uint16_t *>(V), perm, centroids ? centroids : w.at<float>(w.L.cent), s);
+  if ((st = launch_cluster(sh, w, static_cast<const uint16_t *>(V), perm, centroids ? centroids : w.at<float>(w.L.cent),
+                           s)) != VC_OK)
+    return st;
   return last_error();
 }
 
@@ -569,7 +582,7 @@ vc_status vc_attn_fwd(const void *Q, const void *K, const void *V, int B, int H,
     if (clusters) {
       Shape cold = sh;  // vc_attn_fwd has no centroid input: always the default start
       cold.flags &= ~VC_WARMSTART;
-      launch_cluster(cold, w, Vh, w.at<int32_t>(w.L.perm), w.at<float>(w.L.cent), s);
+      if ((st = launch_cluster(cold, w, Vh, w.at<int32_t>(w.L.perm), w.at<float>(w.L.cent), s)) != VC_OK) return st;
       pm = w.at<int32_t>(w.L.perm);
     }
     prof_mark(1, s);
@@ -834,7 +847,7 @@ extern "C" vc_status vc_attn_cluster_noalloc(const void *V, int B, int H, int N,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the completion counters must start at zero; the array keeps the previous call's contents
   if ((st = clear_small(w, s)) != VC_OK) return st;
-  launch_cluster(sh, w, static_cast<const uint16_t *>(V), perm, centroids, s);
+  if ((st = launch_cluster(sh, w, static_cast<const uint16_t *>(V), perm, centroids, s)) != VC_OK) return st;
   const cudaError_t e = cudaGetLastError();
   if (e == cudaErrorContextIsDestroyed || e == cudaErrorDeviceUninitialized || e == cudaErrorInvalidResourceHandle) {
     // the context that held the array is gone: look its address up again next time

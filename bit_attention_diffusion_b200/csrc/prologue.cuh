@@ -1,6 +1,7 @@
 // prologue.cuh - declarations of the prologue kernels (see prologue.cu).
 #pragma once
 #include <cstdint>
+#include <cuda.h>
 
 namespace vc {
 
@@ -9,6 +10,13 @@ __global__ void k_kmeans_pass(const uint16_t *V, int N, int k, int cpb, int nblk
                               double *psum, int *pcnt, unsigned *counter, int accumulate);
 __global__ void k_kmeans_pass8(const uint16_t *V, int N, int k, int cpb, int nblk, float *cent, int32_t *labels,
                                double *psum, int *pcnt, unsigned *counter, int accumulate);
+// k <= 8 with the labels decided on the tensor cores (kmeans_tc.cu); status:
+// the workspace status word (a bounded wait that runs out sets ST_TIMEOUT).
+// tmV: 2-D map over V as [B*H*N rows][128] bf16, boxes of 64 channels x 128
+// rows, 128-byte swizzle.
+__global__ void k_kmeans_pass8tc(const __grid_constant__ CUtensorMap tmV, int N, int k, int cpb, int nblk, float *cent,
+                                 int32_t *labels, double *psum, int *pcnt, unsigned *counter, int accumulate,
+                                 uint32_t *status);
 __global__ void k_perm_sort(const int32_t *labels, int N, int k, int32_t *perm);
 __global__ void k_kbar(const uint16_t *K, int N, int nchunk, int ksmooth, double *part, unsigned *counter,
                        float *kbar);
@@ -64,6 +72,7 @@ __global__ void k_prologue_fused(const FusedPrologueParams p);
 constexpr int QUANTV1_SMEM = 128 * 272;              // gathered rows
 constexpr int QUANTV2_SMEM = 128 * 272 + 128 * 144;  // rows + transposed codes
 constexpr int KMEANS8_SMEM = 2 * 128 * 272;  // double-buffered chunk rows
+constexpr int KMEANS8TC_SMEM = 2 * 128 * 256 + 4096 + 1024;  // two swizzled chunks, the centroid operand, alignment
 constexpr int FUSED_SMEM = KMEANS8_SMEM > QUANTV2_SMEM ? KMEANS8_SMEM : QUANTV2_SMEM;  // the largest phase
 constexpr int KMEANS_SMEM_FIXED = 128 * 66 * 4;  // chunk rows; + k*128*(4+8) for centroids and sums
 

@@ -179,8 +179,6 @@ vc_status check_device() {
                                static_cast<int>(attn_fp4_smem_bytes(false))) != cudaSuccess ||
           cudaFuncSetAttribute(k_vc_attn_fwd44, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(attn_fp4_smem_bytes(true))) != cudaSuccess ||
-          cudaFuncSetAttribute(k_kmeans_pass8, cudaFuncAttributeMaxDynamicSharedMemorySize, KMEANS8_SMEM) !=
-              cudaSuccess ||
           cudaFuncSetAttribute(k_kmeans_pass8tc, cudaFuncAttributeMaxDynamicSharedMemorySize, KMEANS8TC_SMEM) !=
               cudaSuccess ||
           cudaFuncSetAttribute(k_kmeans_pass8tc, cudaFuncAttributePreferredSharedMemoryCarveout,

@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(128) k_kmeans_pass(const uint16_t *__restrict_
   if (tid == 0) counter[bh] = 0u;
 }
 
-// Fast path of the Lloyd pass for k <= 8, same arithmetic per (token,
+// The Lloyd pass for k <= 8 inside the one-launch prologue (the separate
+// launch uses k_kmeans_pass8tc), same arithmetic per (token,
 // cluster) as k_kmeans_pass: d = fp32(v - c) and acc = fma(d, d, acc) in
 // channel order, two clusters per packed f32x2 instruction (each lane rounds
 // exactly like the scalar instruction). 256 threads; the block's 128-token
@@ -348,13 +349,6 @@ __device__ __forceinline__ void kmeans_pass8_body(const uint16_t *__restrict__ V
     }
   }
   if (tid == 0) counter[bh] = 0u;
-}
-__global__ void __launch_bounds__(256) k_kmeans_pass8(const uint16_t *__restrict__ V, int N, int k, int cpb,
-                                                      int nblk, float *__restrict__ cent,
-                                                      int32_t *__restrict__ labels, double *__restrict__ psum,
-                                                      int *__restrict__ pcnt, unsigned *__restrict__ counter,
-                                                      int accumulate) {
-  kmeans_pass8_body(V, N, k, cpb, nblk, cent, labels, psum, pcnt, counter, accumulate, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
 // Stable counting sort of token indices by label, one block per (b,h): a

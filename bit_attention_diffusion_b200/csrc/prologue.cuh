@@ -8,8 +8,6 @@ namespace vc {
 __global__ void k_kmeans_init(const uint16_t *V, int N, int k, float *cent);
 __global__ void k_kmeans_pass(const uint16_t *V, int N, int k, int cpb, int nblk, float *cent, int32_t *labels,
                               double *psum, int *pcnt, unsigned *counter, int accumulate);
-__global__ void k_kmeans_pass8(const uint16_t *V, int N, int k, int cpb, int nblk, float *cent, int32_t *labels,
-                               double *psum, int *pcnt, unsigned *counter, int accumulate);
 // k <= 8 with the labels decided on the tensor cores (kmeans_tc.cu); status:
 // the workspace status word (a bounded wait that runs out sets ST_TIMEOUT).
 // tmV: 2-D map over V as [B*H*N rows][128] bf16, boxes of 64 channels x 128

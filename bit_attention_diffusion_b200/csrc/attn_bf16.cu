@@ -7,8 +7,11 @@
 // fp32 in TMEM, double-buffered); online softmax in log2 units with exp2 on
 // the SFU; the running max used for P is only moved when the true max exceeds
 // it by more than 8 (a factor 256, far inside fp32 and bf16 range), which keeps
-// O rescales rare; P in bf16 to shared memory; O += P V with V consumed
-// MN-major straight from its [token][channel] layout; O = acc / l.
+// O rescales rare; P in bf16 to shared memory, two slots (tile t in slot t % 2),
+// so the softmax of tile t+1 runs while PV(t) does: a tile waits for the PV of
+// tile t-2 (its slot) and, only when it moves the max, for PV(t-1); O += P V
+// with V consumed MN-major straight from its [token][channel] layout;
+// O = acc / l.
 #include "common.cuh"
 #include "sm100.cuh"
 #include "attn_bf16.cuh"
@@ -24,14 +27,14 @@ constexpr uint32_t B_OFF_Q = 0;
 constexpr uint32_t B_OFF_K = B_OFF_Q + SZ_T16;
 constexpr uint32_t B_OFF_V = B_OFF_K + ST * SZ_T16;
 constexpr uint32_t B_OFF_P = B_OFF_V + ST * SZ_T16;
-constexpr uint32_t B_SMEM = B_OFF_P + SZ_T16 + 1024;
+constexpr uint32_t B_SMEM = B_OFF_P + 2 * SZ_T16 + 1024;
 static_assert(B_SMEM <= 232448, "shared memory budget");
 
 constexpr uint32_t IDESC_S = idesc_make(1, 1, 128, 128, false, false);  // Q K^T, both K-major
 constexpr uint32_t IDESC_O = idesc_make(1, 1, 128, 128, false, true);   // P V, V MN-major
 
 struct BarsB {
-  uint64_t q, kfull[ST], kempty[ST], vfull[ST], vempty[ST], sfull[2], pfull, pvdone, main;
+  uint64_t q, kfull[ST], kempty[ST], vfull[ST], vempty[ST], sfull[2], pfull[2], pvdone[2], main;
 };
 
 __device__ __forceinline__ uint64_t kdesc(const uint8_t *p) { return sdesc_sw128(smem_u32(p), 16, 1024); }
@@ -70,7 +73,8 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&bars.vfull[i], 1); mbar_init(&bars.vempty[i], 1);
     }
     mbar_init(&bars.sfull[0], 1); mbar_init(&bars.sfull[1], 1);
-    mbar_init(&bars.pfull, 128); mbar_init(&bars.pvdone, 1); mbar_init(&bars.main, 1);
+    mbar_init(&bars.pfull[0], 128); mbar_init(&bars.pfull[1], 128);
+    mbar_init(&bars.pvdone[0], 1); mbar_init(&bars.pvdone[1], 1); mbar_init(&bars.main, 1);
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(&s_tmem, 512);
@@ -129,18 +133,19 @@ __global__ void __launch_bounds__(192, 1)
       if (ok) ok = issue_qk(0);
       if (ok && T > 1) ok = issue_qk(1);
       for (int t = 0; t < T && ok; ++t) {
-        ok = wait(&bars.pfull, t & 1);
+        ok = wait(&bars.pfull[t & 1], (t >> 1) & 1);
         if (!ok) break;
         const int s = t % ST;
         ok = wait(&bars.vfull[s], (t / ST) & 1);
         if (!ok) break;
         tc_fence_after();
+        const uint8_t *sPt = sP + (t & 1) * SZ_T16;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_f16_ss(tmem + 256, kdesc(sP + (kk >> 2) * ATOM + 32 * (kk & 3)), mndesc(sV + s * SZ_T16 + kk * 2048),
+          mma_f16_ss(tmem + 256, kdesc(sPt + (kk >> 2) * ATOM + 32 * (kk & 3)), mndesc(sV + s * SZ_T16 + kk * 2048),
                      IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars.vempty[s]);
-        mma_commit(&bars.pvdone);
+        mma_commit(&bars.pvdone[t & 1]);
         if (t + 2 < T) ok = issue_qk(t + 2);
       }
       if (ok) mma_commit(&bars.main);
@@ -179,12 +184,19 @@ __global__ void __launch_bounds__(192, 1)
       for (int j = 0; j < 126; j += 3) mx = fmax3(mx, fmax3(s[j], s[j + 1], s[j + 2]), mx);
       mx = fmax3(mx, s[126], s[127]);
       const float mt = mx * p.scale_log2;
-      if (t > 0) {
-        ok = wwait(&bars.pvdone, (t - 1) & 1);
+      // slot t % 2 is free once PV(t-2) is complete
+      if (t >= 2) {
+        ok = wwait(&bars.pvdone[b], ((t >> 1) - 1) & 1);
         if (!ok) break;
-        tc_fence_after();
+      }
+      if (t > 0) {
         const bool need = mt > m_use + 8.0f;
         if (__any_sync(0xFFFFFFFFu, need)) {
+          // O must hold PV(0..t-1) before it is rescaled (PV(t-2) is complete,
+          // so this barrier is at most one phase behind)
+          ok = wwait(&bars.pvdone[b ^ 1], ((t - 1) >> 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
           const float sc = need ? ex2(m_use - mt) : 1.0f;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -202,6 +214,7 @@ __global__ void __launch_bounds__(192, 1)
       } else {
         m_use = mt;
       }
+      uint8_t *sPt = sP + b * SZ_T16;
 #pragma unroll
       for (int ch = 0; ch < 16; ++ch) {
         uint32_t w[4];
@@ -214,11 +227,11 @@ __global__ void __launch_bounds__(192, 1)
           const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
           w[e] = *reinterpret_cast<const uint32_t *>(&pb);
         }
-        *reinterpret_cast<uint4 *>(sP + (ch >> 3) * ATOM + sw128_off(r, ch & 7)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4 *>(sPt + (ch >> 3) * ATOM + sw128_off(r, ch & 7)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars.pfull);
+      mbar_arrive(&bars.pfull[b]);
     }
     if (ok) ok = wwait(&bars.main, 0);
     if (ok) {

@@ -295,8 +295,16 @@ vc_status vc_attn_fwd_host(const void *hQ, const void *hK, const void *hV, int B
 
 /*
  * In-library comparator: exact-softmax attention in BF16 on the tcgen05
- * tensor cores (bf16 operands, fp32 accumulation, fp32 exp2 softmax).
- * softmax_scale 0 => 1/sqrt(d). O bf16 [B,H,N,d].
+ * tensor cores (bf16 operands, fp32 accumulation, fp32 exp2 softmax). The
+ * pages measure VC-Attention against a BF16 FlashAttention-class kernel
+ * ([IP73] intro: 1.46-1.59x over BF16 FlashAttention-4 on datacenter
+ * Blackwell and Hopper; [VCA] "Benchmarks"); this is the library's own BF16
+ * attention on the same tiling, for the same comparison on one GPU.
+ *   Q, K, V  bf16 [B,H,N,d] in (d = 128), device pointers, 16-byte aligned
+ *   O        bf16 [B,H,N,d] out, rows in query order
+ *   softmax_scale 0 => 1/sqrt(d)
+ * No workspace: a bounded device wait that runs out shows only as a wrong
+ * result. Errors as vc_attn_fwd's argument and device checks.
  */
 vc_status vc_attn_fwd_ref_bf16(const void *Q, const void *K, const void *V, int B, int H, int N, int d,
                                float softmax_scale, void *O, void *stream);

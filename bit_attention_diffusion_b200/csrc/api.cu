@@ -29,7 +29,9 @@ Shape make_shape(int B, int H, int N, const vc_params &p, int R) {
   s.R = R;
   s.Rpad = R > 0 ? ((R + 127) / 128) * 128 : 0;
   s.nch32 = (s.Nb + CHUNK32 - 1) / CHUNK32;
-  const int target = std::max(1, (3 * 148) / s.BH);  // k-means blocks per (b,h): three resident per SM
+  // k-means blocks per (b,h): two resident per SM for the k <= 8 pass (512
+  // threads, a three-chunk ring), three for the generic pass
+  const int target = std::max(1, ((p.k <= 8 ? 2 : 3) * 148) / s.BH);
   s.km_cpb = std::max(1, (s.Nb + target - 1) / target);
   s.km_nblk = (s.Nb + s.km_cpb - 1) / s.km_cpb;
   s.kb_nchunk = std::max(1, std::min(s.Nb, (4 * 148 + s.BH - 1) / s.BH));
@@ -306,7 +308,7 @@ vc_status launch_cluster(const Shape &sh, const Ws &w, const uint16_t *V, int32_
   const dim3 grid(sh.km_nblk, sh.BH);
   for (int it = 0; it <= sh.iters; ++it) {
     if (sh.k <= 8)
-      k_kmeans_pass8tc<<<grid, 256, KMEANS8TC_SMEM, s>>>(tmv, sh.N, sh.k, sh.km_cpb, sh.km_nblk, cent, labels,
+      k_kmeans_pass8tc<<<grid, KM_THREADS, KMEANS8TC_SMEM, s>>>(tmv, sh.N, sh.k, sh.km_cpb, sh.km_nblk, cent, labels,
                                                          w.at<double>(w.L.km_psum), w.at<int>(w.L.km_pcnt),
                                                          w.at<unsigned>(w.L.km_counter), it < sh.iters ? 1 : 0,
                                                          w.at<uint32_t>(w.L.status));

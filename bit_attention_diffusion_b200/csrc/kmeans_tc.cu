@@ -18,19 +18,28 @@
 // remainder, the fp32 combination) below 4.3e-5 (|v|^2 + |c_j|^2). When every
 // other cluster's estimate exceeds the smallest one, e_b, by more than
 // E_b + E_j, cluster b is the label (strictly smaller d~ than every other
-// cluster, so no tie arises); otherwise the token goes on a list whose pinned
-// chains (all clusters) the block's warps then run, one token per warp at a
-// time. Labels are therefore exactly k_kmeans_pass's.
+// cluster, so no tie arises); otherwise the pinned chains of all clusters
+// decide. Labels are therefore exactly k_kmeans_pass's.
 //
-// Per block: `cpb` consecutive 128-token chunks of one (b,h), double-buffered
-// in shared memory by TMA in the K-major 128-byte-swizzled layout the MMA
-// reads (two 64-channel atoms per chunk). The product of chunk i+1 goes to the
-// tensor cores, into the second of two 16-column accumulators, while chunk i
-// is labelled: all 256 threads compute the tokens' |v|^2, then warps 0-3 take
-// one token each (TMEM lane = token). In an update pass warp j then adds, in
-// fp64, the channels of the chunk's tokens labelled j (lane l: channels 4l ..
-// 4l+3; exact, so the order is free), and the last block of a (b,h) adds the
-// blocks' partial sums in block order into the new centroids.
+// A block takes `cpb` consecutive 128-token chunks of one (b,h) and runs them
+// through a ring of KS shared-memory stages, one warp role per step, each
+// step handing the stage to the next through an mbarrier:
+//   warp 0      TMA: the chunk, K-major with the 128-byte swizzle the MMA
+//               reads (two 64-channel atoms), once the stage is empty;
+//   warp 1      the product of the chunk with the centroid operand into the
+//               stage's 16 TMEM columns, once the labels of the stage's
+//               previous chunk have been read out of them;
+//   warps 4-7   one token per thread (TMEM lane = token): |v|^2, the
+//               estimates, the label or a place on the fallback list;
+//   warps 2-3   the fallback list: the pinned chains, eight lanes per token
+//               (lane j of the group is cluster j), four tokens per warp;
+//   warps 8-15  update passes: warp j lists the chunk's tokens labelled j
+//               and adds them, in fp64, four rows per step (lane l: channels
+//               4l .. 4l+3), then frees the stage.
+// No step waits for the whole block: a slow step (many fallback tokens, a
+// large cluster) holds its stage, and the others go on until the ring is
+// full. The last block of a (b,h) adds the blocks' partial sums in block order
+// into the new centroids.
 #include "common.cuh"
 #include "prologue.cuh"
 #include "sm100.cuh"
@@ -40,6 +49,7 @@ namespace vc {
 namespace {
 
 constexpr int KT_CHUNK_BYTES = TILE * D * 2;                     // 32 KB: two 16 KB atoms
+constexpr int KS = KMEANS8TC_STAGES;                             // ring stages
 constexpr uint32_t KT_IDESC = idesc_make(1, 1, 128, 16, false, false);  // bf16 x bf16 -> f32, N = 16
 
 __device__ __forceinline__ uint32_t kt_off(int row, int ch16) {  // 16-byte chunk ch16 (0..15) of a token row
@@ -63,24 +73,46 @@ __device__ __forceinline__ void kt_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
+// Shared-memory loads at a 32-bit shared address. Volatile, so they stay
+// after the barrier wait that precedes them; without a memory clobber, so the
+// compiler may issue several before using the first.
+__device__ __forceinline__ uint2 lds64_nc(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(256, 3) k_kmeans_pass8tc(const __grid_constant__ CUtensorMap tmV, int N, int k,
-                                                           int cpb, int nblk, float *__restrict__ cent,
-                                                        int32_t *__restrict__ labels, double *__restrict__ psum,
-                                                        int *__restrict__ pcnt, unsigned *__restrict__ counter,
-                                                        int accumulate, uint32_t *__restrict__ status) {
+struct BarsKm {
+  uint64_t full[KS], mma[KS], lab[KS], fbd[KS], empty[KS];
+};
+
+__global__ void __launch_bounds__(KM_THREADS, 2) k_kmeans_pass8tc(const __grid_constant__ CUtensorMap tmV, int N,
+                                                                  int k, int cpb, int nblk, float *__restrict__ cent,
+                                                                  int32_t *__restrict__ labels,
+                                                                  double *__restrict__ psum, int *__restrict__ pcnt,
+                                                                  unsigned *__restrict__ counter, int accumulate,
+                                                                  uint32_t *__restrict__ status) {
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
-  uint8_t *dsm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sB = dsm + 2 * KT_CHUNK_BYTES;        // B operand: rows 0-7 hi(c_j), 8-15 lo(c_j); two 2 KB atoms
+  uint8_t *dsm = smem_align1024(dsm_raw);
+  uint8_t *sB = dsm + KS * KT_CHUNK_BYTES;       // B operand: rows 0-7 hi(c_j), 8-15 lo(c_j); two 2 KB atoms
+  __shared__ BarsKm bars;
   __shared__ float scc[8];                       // |c_j|^2
-  __shared__ float svv[2][TILE];                 // |v|^2 over channels 0-63 / 64-127
-  __shared__ int slab[TILE];
-  __shared__ int sfb[TILE];                      // tokens the estimate cannot decide
-  __shared__ int s_nfb;
+  __shared__ __align__(16) float scent[8][D + 4];  // fp32 centroids (rows padded: the 8 lanes of a chain group hit 8 banks)
+  __shared__ int8_t slab[KS][TILE];              // label of each token of the stage's chunk (-1: not yet)
+  __shared__ uint8_t sfb[KS][4][32];             // fallback tokens, per label warp
+  __shared__ int snfb[KS][4];
+  __shared__ __align__(16) uint8_t sidx[8][TILE];  // sum warp j: its cluster's tokens of the current chunk
+  __shared__ int s_fail;
   __shared__ int s_last;
   __shared__ uint32_t s_tmem;
-  __shared__ uint64_t mbar[2], full[2];
+  __shared__ int s_tma_issued, s_tma_seen, s_mma_issued, s_mma_seen;
   const int bh = blockIdx.y, blk = blockIdx.x, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   float *cent_h = cent + static_cast<size_t>(bh) * k * D;
@@ -90,19 +122,28 @@ __global__ void __launch_bounds__(256, 3) k_kmeans_pass8tc(const __grid_constant
   const int nchunk = (n_end - n_begin + TILE - 1) / TILE;
   const int row_base = bh * N + n_begin;  // map row of the block's first token
   if (tid == 0) {
-    mbar_init(&mbar[0], 1);
-    mbar_init(&mbar[1], 1);
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.mma[s], 1);
+      mbar_init(&bars.lab[s], 128);
+      mbar_init(&bars.fbd[s], 64);
+      mbar_init(&bars.empty[s], 256);
+    }
     fence_mbar_init();
     prefetch_tmap(&tmV);
-    for (int i = 0; i < 2 && i < nchunk; ++i) kt_load_chunk(dsm + i * KT_CHUNK_BYTES, &tmV, &full[i], row_base + i * TILE);
+    s_fail = 0;
+    s_tma_issued = min(KS, nchunk);
+    s_tma_seen = 0;
+    s_mma_issued = 0;
+    s_mma_seen = 0;
+    for (int i = 0; i < KS && i < nchunk; ++i)
+      kt_load_chunk(dsm + i * KT_CHUNK_BYTES, &tmV, &bars.full[i], row_base + i * TILE);
   }
 
   // centroids: the bf16 hi/lo operand and |c_j|^2 (the pinned chains read
   // the fp32 centroids from global memory, through L1)
-  for (int i = tid; i < 16 * 16; i += 256) {  // 16 rows x 16 chunks of 8 channels
-    const int row = i >> 4, ch16 = i & 15, j = row & 7;
+  if (tid < 16 * 16) {  // 16 rows x 16 chunks of 8 channels
+    const int row = tid >> 4, ch16 = tid & 15, j = row & 7;
     uint32_t w[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -118,10 +159,9 @@ __global__ void __launch_bounds__(256, 3) k_kmeans_pass8tc(const __grid_constant
       w[e] = static_cast<uint32_t>(h2[0]) | (static_cast<uint32_t>(h2[1]) << 16);
     }
     *reinterpret_cast<uint4 *>(sB + (ch16 >> 3) * 2048 + sw128_off(row, ch16 & 7)) = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-  {
-    // |c_j|^2 in fp64, warp j (8 warps)
-    const int j = warp;
+  } else if (warp < 16) {
+    // |c_j|^2 in fp64, warp 8 + j
+    const int j = warp - 8;
     double s2 = 0.0;
     if (j < k)
       for (int c = lane; c < D; c += 32) {
@@ -132,152 +172,113 @@ __global__ void __launch_bounds__(256, 3) k_kmeans_pass8tc(const __grid_constant
     for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, o);
     if (lane == 0) scc[j] = j < k ? static_cast<float>(s2) : 0.0f;
   }
-  if (warp == 0) tmem_alloc(&s_tmem, 32);
-  if (tid == 0) s_nfb = 0;
+  for (int i = tid; i < 8 * D; i += KM_THREADS) scent[i / D][i % D] = (i / D) < k ? cent_h[i] : 0.0f;
+  if (warp == 1) tmem_alloc(&s_tmem, 64);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  const uint64_t dB = sdesc_sw128(smem_u32(sB), 16, 1024);
-  // v . hi(c_j), v . lo(c_j) of chunk `ci` (landed) into D(ci % 2): columns 16 (ci % 2) ..
-  auto issue_mma = [&](int ci) {
-    const uint64_t dA = sdesc_sw128(smem_u32(dsm + (ci & 1) * KT_CHUNK_BYTES), 16, 1024);
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      mma_f16_ss(tmem + 16u * (ci & 1), dA + (kk >> 2) * ((TILE * 128) >> 4) + 2 * (kk & 3),
-                 dB + (kk >> 2) * (2048 >> 4) + 2 * (kk & 3), KT_IDESC, kk > 0);
-    mma_commit(&mbar[ci & 1]);
-  };
-  bool ok = true;
-  if (tid == 0 && nchunk > 0) {
-    ok = mbar_wait(&full[0], 0);
-    if (ok) {
-      tc_fence_after();
-      issue_mma(0);
-    } else {
-      atomicOr(status, ST_TIMEOUT);
-    }
-  }
 
-  // sums: warp j < k owns cluster j, lane l channels 4l .. 4l+3
   double acc4[4] = {0.0, 0.0, 0.0, 0.0};
-  int cnt_own = 0;  // tokens of cluster `warp` (lane 0)
-  for (int i = 0; i < nchunk; ++i) {
-    const int n0 = n_begin + i * TILE, cnt = min(TILE, n_end - n0);
-    uint8_t *buf = dsm + (i & 1) * KT_CHUNK_BYTES;
-    // the chunk has landed (its product was issued when it did)
-    const bool landed = ok && mbar_wait(&full[i & 1], (i >> 1) & 1);
-    if (!__syncthreads_and(landed)) {
-      if (tid == 0) atomicOr(status, ST_TIMEOUT);
-      ok = false;
-    }
-    {
-      // |v|^2 of token tid % 128 over channels [64 h, 64 h + 64), h = tid / 128
-      const int t = tid & 127, h = tid >> 7;
-      float a = 0.0f;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint4 w = *reinterpret_cast<const uint4 *>(buf + kt_off(t, 8 * h + q));
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x0 = __uint_as_float(ws[e] << 16), x1 = __uint_as_float(ws[e] & 0xFFFF0000u);
-          a = fmaf(x0, x0, a);
-          a = fmaf(x1, x1, a);
+  int cnt_own = 0;  // tokens of cluster warp - 8 (sum warps)
+  if (warp == 0) {
+    // ---- TMA producer: chunk i into stage i % KS once chunk i - KS has left it
+    if (lane == 0)
+      for (int i = KS; i < nchunk; ++i) {
+        const int s = i % KS;
+        if (!mbar_wait(&bars.empty[s], ((i / KS) - 1) & 1)) {
+          atomicOr(status, ST_TIMEOUT);
+          s_fail = 1;
+          break;
         }
+        kt_load_chunk(dsm + s * KT_CHUNK_BYTES, &tmV, &bars.full[s], row_base + i * TILE);
+        s_tma_issued = i + 1;
       }
-      svv[h][t] = a;
+  } else if (warp == 1) {
+    // ---- MMA issuer: v . hi(c_j), v . lo(c_j) of chunk i into TMEM columns 16 s
+    if (lane == 0) {
+      const uint64_t dB = sdesc_sw128(smem_u32(sB), 16, 1024);
+      for (int i = 0; i < nchunk; ++i) {
+        const int s = i % KS;
+        if (!mbar_wait(&bars.full[s], (i / KS) & 1)) {
+          atomicOr(status, ST_TIMEOUT);
+          s_fail = 1;
+          break;
+        }
+        s_tma_seen = i + 1;
+        if (i >= KS && !mbar_wait(&bars.lab[s], ((i / KS) - 1) & 1)) {  // the stage's columns were read
+          atomicOr(status, ST_TIMEOUT);
+          s_fail = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t dA = sdesc_sw128(smem_u32(dsm + s * KT_CHUNK_BYTES), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_f16_ss(tmem + 16u * s, dA + (kk >> 2) * ((TILE * 128) >> 4) + 2 * (kk & 3),
+                     dB + (kk >> 2) * (2048 >> 4) + 2 * (kk & 3), KT_IDESC, kk > 0);
+        mma_commit(&bars.mma[s]);
+        s_mma_issued = i + 1;
+      }
     }
-    __syncthreads();
-    if (warp < 4) {
-      const int tok = tid;  // TMEM lane tid
-      const bool w_ok = ok && mbar_wait(&mbar[i & 1], (i >> 1) & 1);
-      if (!__all_sync(0xFFFFFFFFu, w_ok)) {
+  } else if (warp < 4) {
+    // ---- fallback warps: the pinned chains of the undecided tokens, four
+    // tokens per warp at a time (lane group g = lane / 8, cluster j = lane % 8)
+    const int fw = warp - 2, g = lane >> 3, j = lane & 7;
+    for (int i = 0; i < nchunk; ++i) {
+      const int s = i % KS;
+      const int n0 = n_begin + i * TILE;
+      if (!mbar_wait(&bars.lab[s], (i / KS) & 1)) {
         if (lane == 0) atomicOr(status, ST_TIMEOUT);
-        ok = false;
+        s_fail = 1;
+        break;
       }
-      tc_fence_after();
-      uint32_t dr[16];
-      kt_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + 16u * (i & 1), dr);
-      tmem_wait_ld();
-      tc_fence_before();
-      int lab = 0;
-      bool fallback = false;
-      if (tok < cnt && k > 1) {
-        const float vv = __fadd_rn(svv[0][tok], svv[1][tok]);
-        float e[8], bnd[8];
-        float best = INFINITY;
-        int jb = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float dot = __fadd_rn(__uint_as_float(dr[j]), __uint_as_float(dr[8 + j]));
-          e[j] = __fsub_rn(__fadd_rn(vv, scc[j]), 2.0f * dot);
-          bnd[j] = 1.220703125e-4f * __fadd_rn(vv, scc[j]);  // E_j = 2^-13 (|v|^2 + |c_j|^2)
-          if (j < k && e[j] < best) {
-            best = e[j];
-            jb = j;
-          }
+      const int c0 = snfb[s][0], c1 = snfb[s][1], c2 = snfb[s][2], c3 = snfb[s][3];
+      const int nfb = c0 + c1 + c2 + c3;
+      const uint32_t sbuf = smem_u32(dsm) + s * KT_CHUNK_BYTES;
+      for (int f0 = 0; f0 < nfb; f0 += 8) {
+        const int f = f0 + 2 * g + fw;
+        int t2 = -1;
+        if (f < nfb) {
+          const int w = f < c0 ? 0 : f < c0 + c1 ? 1 : f < c0 + c1 + c2 ? 2 : 3;
+          const int base = w == 0 ? 0 : w == 1 ? c0 : w == 2 ? c0 + c1 : c0 + c1 + c2;
+          t2 = sfb[s][w][f - base];
         }
-        lab = jb;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (j < k && j != jb && !(__fsub_rn(e[j], best) > __fadd_rn(bnd[jb], bnd[j]))) fallback = true;
-      }
-      if (tok < cnt && !fallback) {
-        slab[tok] = lab;
-        labels[static_cast<size_t>(bh) * N + n0 + tok] = lab;
-      }
-      const unsigned fbm = __ballot_sync(0xFFFFFFFFu, fallback);
-      int at = 0;
-      if (lane == 0 && fbm) at = atomicAdd(&s_nfb, __popc(fbm));
-      at = __shfl_sync(0xFFFFFFFFu, at, 0);
-      if (fallback) sfb[at + __popc(fbm & ((1u << lane) - 1u))] = tok;
-      if (warp == 0 && i + 1 < nchunk) {
-        // the next chunk's product, into the other accumulator
-        bool nxt = true;
-        if (lane == 0) {
-          nxt = ok && mbar_wait(&full[(i + 1) & 1], ((i + 1) >> 1) & 1);
-          if (nxt) {
-            tc_fence_after();
-            issue_mma(i + 1);
-          } else {
-            atomicOr(status, ST_TIMEOUT);
-          }
-        }
-        if (!__shfl_sync(0xFFFFFFFFu, nxt, 0)) ok = false;
-      }
-    }
-    __syncthreads();
-    {
-      // ---- the pinned distances for the undecided tokens, one token per warp
-      // at a time: lane j < k runs cluster j's chain over the channels in
-      // order, then the warp takes the smallest (ties to the lowest cluster)
-      const int nfb = s_nfb;
-      for (int f = warp; f < nfb; f += 8) {
-        const int t2 = sfb[f];
         float d = INFINITY;
-        if (lane < k) {
-          const float4 *cj = reinterpret_cast<const float4 *>(cent_h + lane * D);
+        if (t2 >= 0 && j < k) {
+          const float4 *cj = reinterpret_cast<const float4 *>(&scent[j][0]);
           float a = 0.0f;
+          // channel order (the pinned chain); the next 8 channels' operands
+          // are loaded while the current ones are accumulated
+          uint4 w = lds128(sbuf + kt_off(t2, 0));
+          float4 cA = cj[0], cB = cj[1];
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(buf + kt_off(t2, q));
-            const float4 c0 = cj[2 * q], c1 = cj[2 * q + 1];
+            uint4 wn = w;
+            float4 cAn = cA, cBn = cB;
+            if (q < 15) {
+              wn = lds128(sbuf + kt_off(t2, q + 1));
+              cAn = cj[2 * q + 2];
+              cBn = cj[2 * q + 3];
+            }
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-            const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            const float cc[8] = {cA.x, cA.y, cA.z, cA.w, cB.x, cB.y, cB.z, cB.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const float v = (e & 1) ? __uint_as_float(ws[e >> 1] & 0xFFFF0000u) : __uint_as_float(ws[e >> 1] << 16);
               const float x = __fsub_rn(v, cc[e]);
               a = fmaf(x, x, a);
             }
+            w = wn;
+            cA = cAn;
+            cB = cBn;
           }
           d = a;
         }
-        int jmin = lane < k ? lane : 8;
+        int jmin = j < k ? j : 8;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
+        for (int o = 4; o > 0; o >>= 1) {  // within the lane group
           const float d2 = __shfl_xor_sync(0xFFFFFFFFu, d, o);
           const int j2 = __shfl_xor_sync(0xFFFFFFFFu, jmin, o);
           if (d2 < d || (d2 == d && j2 < jmin)) {
@@ -285,52 +286,153 @@ __global__ void __launch_bounds__(256, 3) k_kmeans_pass8tc(const __grid_constant
             jmin = j2;
           }
         }
-        if (lane == 0) {
-          slab[t2] = jmin;
+        if (j == 0 && t2 >= 0) {
+          slab[s][t2] = static_cast<int8_t>(jmin);
           labels[static_cast<size_t>(bh) * N + n0 + t2] = jmin;
         }
       }
+      __syncwarp();
+      mbar_arrive(&bars.fbd[s]);
     }
-    if (accumulate) {
-      __syncthreads();  // every label of the chunk is in slab
-      // ---- fp64 sums: warp j adds the tokens labelled j, lane l its channels
-      // 4l .. 4l+3 (exact, so the order is free)
-      const int j = warp;
-      if (j < k) {
-        unsigned m[4];
+  } else if (warp < 8) {
+    // ---- label warps: one token per thread, TMEM lane = token
+    const int tok = tid - 128, lw = warp - 4;
+    for (int i = 0; i < nchunk; ++i) {
+      const int s = i % KS;
+      const int n0 = n_begin + i * TILE, cnt = min(TILE, n_end - n0);
+      const uint32_t sbuf = smem_u32(dsm) + s * KT_CHUNK_BYTES;
+      const bool w_ok = mbar_wait(&bars.mma[s], (i / KS) & 1);
+      if (!__all_sync(0xFFFFFFFFu, w_ok)) {
+        if (lane == 0) atomicOr(status, ST_TIMEOUT);
+        s_fail = 1;
+        break;
+      }
+      tc_fence_after();
+      uint32_t dr[16];
+      kt_ld16(tmem + (static_cast<uint32_t>(lw * 32) << 16) + 16u * s, dr);
+      tmem_wait_ld();
+      tc_fence_before();
+      if (tid == 128) s_mma_seen = i + 1;
+      int lab = 0;
+      bool fallback = false;
+      if (tok < cnt && k > 1) {
+        // |v|^2: eight partial sums (16-byte chunk q into sum q % 8), then
+        // added pairwise (any order keeps its rounding inside the bound)
+        float vh[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) m[q] = __ballot_sync(0xFFFFFFFFu, 32 * q + lane < cnt && slab[32 * q + lane] == j);
-        cnt_own += __popc(m[0]) + __popc(m[1]) + __popc(m[2]) + __popc(m[3]);
+        for (int q = 0; q < 8; ++q) vh[q] = 0.0f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          unsigned mm = m[q];
-          while (mm) {
-            const int t = 32 * q + __ffs(mm) - 1;
-            mm &= mm - 1;
-            const uint2 w = *reinterpret_cast<const uint2 *>(buf + kt_off(t, lane >> 1) + 8 * (lane & 1));
-            acc4[0] += static_cast<double>(__uint_as_float(w.x << 16));
-            acc4[1] += static_cast<double>(__uint_as_float(w.x & 0xFFFF0000u));
-            acc4[2] += static_cast<double>(__uint_as_float(w.y << 16));
-            acc4[3] += static_cast<double>(__uint_as_float(w.y & 0xFFFF0000u));
+        for (int q = 0; q < 16; ++q) {
+          const uint4 w = lds128(sbuf + kt_off(tok, q));
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = __uint_as_float(ws[e] << 16), x1 = __uint_as_float(ws[e] & 0xFFFF0000u);
+            vh[q & 7] = fmaf(x0, x0, vh[q & 7]);
+            vh[q & 7] = fmaf(x1, x1, vh[q & 7]);
           }
         }
+        const float vv = __fadd_rn(__fadd_rn(__fadd_rn(vh[0], vh[1]), __fadd_rn(vh[2], vh[3])),
+                                   __fadd_rn(__fadd_rn(vh[4], vh[5]), __fadd_rn(vh[6], vh[7])));
+        float e[8];
+        float best = INFINITY;
+        int jb = 0;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const float dot = __fadd_rn(__uint_as_float(dr[jj]), __uint_as_float(dr[8 + jj]));
+          e[jj] = __fsub_rn(__fadd_rn(vv, scc[jj]), 2.0f * dot);
+          if (jj < k && e[jj] < best) {
+            best = e[jj];
+            jb = jj;
+          }
+        }
+        lab = jb;
+        const float bnd_b = 1.220703125e-4f * __fadd_rn(vv, scc[jb]);  // E_j = 2^-13 (|v|^2 + |c_j|^2)
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+          if (jj < k && jj != jb &&
+              !(__fsub_rn(e[jj], best) > __fadd_rn(bnd_b, 1.220703125e-4f * __fadd_rn(vv, scc[jj]))))
+            fallback = true;
       }
+      slab[s][tok] = (tok < cnt && !fallback) ? static_cast<int8_t>(lab) : static_cast<int8_t>(-1);
+      if (tok < cnt && !fallback) labels[static_cast<size_t>(bh) * N + n0 + tok] = lab;
+      const unsigned fbm = __ballot_sync(0xFFFFFFFFu, fallback);
+      if (fallback) sfb[s][lw][__popc(fbm & ((1u << lane) - 1u))] = static_cast<uint8_t>(tok);
+      if (lane == 0) snfb[s][lw] = __popc(fbm);
+      mbar_arrive(&bars.lab[s]);
     }
-    tc_fence_before();
-    __syncthreads();  // every read of this buffer and of D is done
-    tc_fence_after();
-    if (tid == 0) {
-      s_nfb = 0;
-      if (ok && i + 2 < nchunk) kt_load_chunk(buf, &tmV, &full[i & 1], row_base + (i + 2) * TILE);
+  } else {
+    // ---- sum warps: warp 8 + j adds the chunk's tokens labelled j
+    const int j = warp - 8;
+    for (int i = 0; i < nchunk; ++i) {
+      const int s = i % KS;
+      const int n0 = n_begin + i * TILE, cnt = min(TILE, n_end - n0);
+      const uint32_t sbuf = smem_u32(dsm) + s * KT_CHUNK_BYTES;
+      if (!mbar_wait(&bars.fbd[s], (i / KS) & 1)) {
+        if (lane == 0) atomicOr(status, ST_TIMEOUT);
+        s_fail = 1;
+        break;
+      }
+      if (accumulate && j < k) {
+        // the chunk's tokens of cluster j, listed in token order
+        int cj = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const bool mine = 32 * q + lane < cnt && slab[s][32 * q + lane] == j;
+          const unsigned b = __ballot_sync(0xFFFFFFFFu, mine);
+          if (mine) sidx[j][cj + __popc(b & ((1u << lane) - 1u))] = static_cast<uint8_t>(32 * q + lane);
+          cj += __popc(b);
+        }
+        __syncwarp();
+        cnt_own += cj;
+        // fp64 sums of the listed tokens, four tokens per step (their rows
+        // loaded together), two accumulator sets (even and odd list
+        // positions) added at the end: exact, so the order does not change
+        // the sums
+        double B[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int n = 0; n < cj; n += 4) {
+          const uint32_t t4 = *reinterpret_cast<const uint32_t *>(&sidx[j][n]);  // four listed tokens
+          uint2 w4[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)  // (entries past the list are stale: masked to a row of the chunk, read, dropped)
+            w4[u] = lds64_nc(sbuf + kt_off((t4 >> (8 * u)) & 0x7Fu, lane >> 1) + 8 * (lane & 1));
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (n + u >= cj) break;
+            double *acc = (u & 1) ? B : acc4;
+            acc[0] += static_cast<double>(__uint_as_float(w4[u].x << 16));
+            acc[1] += static_cast<double>(__uint_as_float(w4[u].x & 0xFFFF0000u));
+            acc[2] += static_cast<double>(__uint_as_float(w4[u].y << 16));
+            acc[3] += static_cast<double>(__uint_as_float(w4[u].y & 0xFFFF0000u));
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc4[c] += B[c];
+        __syncwarp();  // the list is rewritten for the next chunk
+      }
+      __syncwarp();
+      mbar_arrive(&bars.empty[s]);
     }
   }
-  if (warp == 0) tmem_dealloc(tmem, 32);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (s_fail && tid == 0) {
+    // a wait ran out: let the copies and products still in flight land before
+    // the block leaves (bounded waits, again)
+    for (int i = s_tma_seen; i < s_tma_issued; ++i)
+      if (!mbar_wait(&bars.full[i % KS], (i / KS) & 1)) break;
+    for (int i = s_mma_seen; i < s_mma_issued; ++i)
+      if (!mbar_wait(&bars.mma[i % KS], (i / KS) & 1)) break;
+  }
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 64);
   if (!accumulate) return;
   double *ps = psum + (static_cast<size_t>(bh) * nblk + blk) * k * D;
   int *pc = pcnt + (static_cast<size_t>(bh) * nblk + blk) * k;
-  if (warp < k) {
-    *reinterpret_cast<double4 *>(ps + warp * D + 4 * lane) = make_double4(acc4[0], acc4[1], acc4[2], acc4[3]);
-    if (lane == 0) pc[warp] = cnt_own;
+  if (warp >= 8 && warp - 8 < k) {
+    *reinterpret_cast<double4 *>(ps + (warp - 8) * D + 4 * lane) = make_double4(acc4[0], acc4[1], acc4[2], acc4[3]);
+    if (lane == 0) pc[warp - 8] = cnt_own;
   }
   __threadfence();
   __syncthreads();
@@ -341,7 +443,7 @@ __global__ void __launch_bounds__(256, 3) k_kmeans_pass8tc(const __grid_constant
   // every (cluster, channel) of the head: partial sums added in block order
   {
     const int c = tid & 127;
-    for (int j = tid >> 7; j < k; j += 2) {
+    for (int j = tid >> 7; j < k; j += KM_THREADS / 128) {
       double sum = 0.0;
       long long n = 0;
 #pragma unroll 16

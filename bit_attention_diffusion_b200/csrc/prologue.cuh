@@ -70,7 +70,9 @@ __global__ void k_prologue_fused(const FusedPrologueParams p);
 constexpr int QUANTV1_SMEM = 128 * 272;              // gathered rows
 constexpr int QUANTV2_SMEM = 128 * 272 + 128 * 144;  // rows + transposed codes
 constexpr int KMEANS8_SMEM = 2 * 128 * 272;  // double-buffered chunk rows
-constexpr int KMEANS8TC_SMEM = 2 * 128 * 256 + 4096 + 1024;  // two swizzled chunks, the centroid operand, alignment
+constexpr int KMEANS8TC_STAGES = 3;   // chunk ring of k_kmeans_pass8tc
+constexpr int KM_THREADS = 512;       // k_kmeans_pass8tc: 16 warps, two blocks per SM
+constexpr int KMEANS8TC_SMEM = KMEANS8TC_STAGES * 128 * 256 + 4096 + 1024;  // swizzled chunks, centroid operand, alignment
 constexpr int FUSED_SMEM = KMEANS8_SMEM > QUANTV2_SMEM ? KMEANS8_SMEM : QUANTV2_SMEM;  // the largest phase
 constexpr int KMEANS_SMEM_FIXED = 128 * 66 * 4;  // chunk rows; + k*128*(4+8) for centroids and sums
 

@@ -48,6 +48,14 @@ namespace vc {
 
 namespace {
 
+// The dynamic shared-memory base rounded up to a multiple of 1024 bytes by
+// pointer arithmetic on the array itself, so that the compiler still knows the
+// result points into shared memory and accesses through it compile to
+// shared-memory instructions (an integer round trip would make them generic).
+__device__ __forceinline__ uint8_t *smem_align1024(uint8_t *raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 constexpr int KT_CHUNK_BYTES = TILE * D * 2;                     // 32 KB: two 16 KB atoms
 constexpr int KS = KMEANS8TC_STAGES;                             // ring stages
 constexpr uint32_t KT_IDESC = idesc_make(1, 1, 128, 16, false, false);  // bf16 x bf16 -> f32, N = 16

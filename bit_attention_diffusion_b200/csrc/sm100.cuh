@@ -20,14 +20,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// The dynamic shared-memory base rounded up to a multiple of 1024 bytes by
-// pointer arithmetic on the array itself, so that the compiler still knows the
-// result points into shared memory and accesses through it compile to
-// shared-memory instructions (an integer round trip would make them generic).
-__device__ __forceinline__ uint8_t *smem_align1024(uint8_t *raw) {
-  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
-}
-
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

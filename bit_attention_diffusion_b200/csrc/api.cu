@@ -173,7 +173,7 @@ vc_status check_device() {
                                static_cast<int>(attn_bf16_smem_bytes())) != cudaSuccess ||
           cudaFuncSetAttribute(k_kmeans_pass, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                KMEANS_SMEM_FIXED + 64 * D * 12) != cudaSuccess ||
-          cudaFuncSetAttribute(k_quantv_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, QUANTV2_SMEM) !=
+          cudaFuncSetAttribute(k_quantv_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, QUANTV2E_SMEM) !=
               cudaSuccess ||
           cudaFuncSetAttribute(k_quantv4_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, QUANTV2_SMEM) !=
               cudaSuccess ||
@@ -362,7 +362,7 @@ void launch_quant_v(const Shape &sh, const Ws &w, const uint16_t *V, const int32
                                                                   vexpo, v8t, w.at<float>(w.L.err),
                                                                   w.at<uint16_t>(w.L.mut2));
   else
-    k_quantv_pass2<<<dim3(sh.Nb, sh.BH), 256, QUANTV2_SMEM, s>>>(V, perm, sh.N, sh.Nb, sh.Npad, sh.nch32, vmean,
+    k_quantv_pass2<<<dim3(sh.Nb, sh.BH), 256, QUANTV2E_SMEM, s>>>(V, perm, sh.N, sh.Nb, sh.Npad, sh.nch32, vmean,
                                                                  vscale, vexpo, v8t, w.at<float>(w.L.err),
                                                                  w.at<uint16_t>(w.L.mut2));
   count_launch();

@@ -747,7 +747,11 @@ __global__ void __launch_bounds__(256) k_quantv_pass1(const uint16_t *__restrict
 // owns token r: its error is fmaf-accumulated in channel order; the residual,
 // scaling and dequantization of a channel pair are packed f32x2 operations
 // (each lane rounds as the scalar one; differences are sums with negated
-// operands, exactly the same values).
+// operands, exactly the same values). The codes of channels c0..c0+7 go over
+// bytes c0..c0+7 of the token's own row, whose values there (channels below
+// c0/2 + 4) have been read already; then every thread transposes 16 rows x 4
+// channels in registers and writes four 16-byte pieces of channel rows. The
+// tile therefore needs only its row buffer (six blocks per SM).
 __device__ __forceinline__ void quantv_pass2_body(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,
                                                       int N, int Nb, int Npad, int nch32,
                                                       const uint16_t *__restrict__ vmean,
@@ -755,8 +759,7 @@ __device__ __forceinline__ void quantv_pass2_body(const uint16_t *__restrict__ V
                                                       uint8_t *__restrict__ v8t, float *__restrict__ err,
                                                       uint16_t *__restrict__ mut2, int bx, int by, int bz) {
   extern __shared__ __align__(16) uint8_t dsm[];
-  uint8_t *sv = dsm;                            // 128 rows x 272 bytes
-  uint8_t *codeT = dsm + TILE * VQ_ROW_BYTES;   // 128 channels x 144 bytes
+  uint8_t *sv = dsm;                            // 128 rows x 272 bytes; then the codes, row-major
   __shared__ __align__(16) float snmu[D], smult[D], snscale[D];  // -mean, 2^-e, -scale
   const int t = bx, bh = by, tid = threadIdx.x;
   const int p0 = t * TILE, cnt = min(TILE, N - p0);
@@ -784,11 +787,12 @@ __device__ __forceinline__ void quantv_pass2_body(const uint16_t *__restrict__ V
   if (tid < 128) {
     const int r = tid;
     float acc = 0.0f;
-    const uint8_t *row = sv + r * VQ_ROW_BYTES;
+    uint8_t *row = sv + r * VQ_ROW_BYTES;
 #pragma unroll 2
     for (int c0 = 0; c0 < D; c0 += 8) {
       float x[8];
       bf16x8(*reinterpret_cast<const uint4 *>(row + 2 * c0), x);
+      uint32_t cw[2] = {0u, 0u};  // the codes of channels c0 .. c0+7
 #pragma unroll
       for (int j = 0; j < 8; j += 2) {
         const int c = c0 + j;
@@ -802,20 +806,35 @@ __device__ __forceinline__ void quantv_pass2_body(const uint16_t *__restrict__ V
           acc = __fmaf_rn(ee.x, ee.x, acc);
           acc = __fmaf_rn(ee.y, ee.y, acc);
         }
-        codeT[c * 144 + r] = static_cast<uint8_t>(codes & 0xFF);
-        codeT[(c + 1) * 144 + r] = static_cast<uint8_t>(codes >> 8);
+        cw[j >> 2] |= static_cast<uint32_t>(codes) << (8 * (j & 3));
       }
+      *reinterpret_cast<uint2 *>(row + c0) = make_uint2(cw[0], cw[1]);  // over values already read
     }
     if (r < cnt) err[static_cast<size_t>(bh) * N + p0 + r] = acc;
   }
   __syncthreads();
   {
-    const int c = tid >> 1, half = tid & 1;
-    uint8_t *dst = v8t + (static_cast<size_t>(bh) * D + c) * Npad + p0 + 64 * half;
-    const uint8_t *srcT = codeT + c * 144 + 64 * half;
+    // thread (rg, cg): rows 16 rg .. 16 rg + 15, channels 4 cg .. 4 cg + 3
+    const int cg = tid & 31, rg = tid >> 5;
+    uint32_t wv[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) wv[q] = *reinterpret_cast<const uint32_t *>(sv + (16 * rg + q) * VQ_ROW_BYTES + 4 * cg);
+    uint32_t ch[4][4];  // [channel][4-row group]: the channel's bytes of those rows
+#pragma unroll
+    for (int g4 = 0; g4 < 4; ++g4) {
+      const uint32_t t0 = __byte_perm(wv[4 * g4], wv[4 * g4 + 1], 0x5140);
+      const uint32_t t1 = __byte_perm(wv[4 * g4], wv[4 * g4 + 1], 0x7362);
+      const uint32_t t2 = __byte_perm(wv[4 * g4 + 2], wv[4 * g4 + 3], 0x5140);
+      const uint32_t t3 = __byte_perm(wv[4 * g4 + 2], wv[4 * g4 + 3], 0x7362);
+      ch[0][g4] = __byte_perm(t0, t2, 0x5410);
+      ch[1][g4] = __byte_perm(t0, t2, 0x7632);
+      ch[2][g4] = __byte_perm(t1, t3, 0x5410);
+      ch[3][g4] = __byte_perm(t1, t3, 0x7632);
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      *reinterpret_cast<uint4 *>(dst + 16 * i) = *reinterpret_cast<const uint4 *>(srcT + 16 * i);
+      *reinterpret_cast<uint4 *>(v8t + (static_cast<size_t>(bh) * D + 4 * cg + i) * Npad + p0 + 16 * rg) =
+          make_uint4(ch[i][0], ch[i][1], ch[i][2], ch[i][3]);
   }
 }
 __global__ void __launch_bounds__(256) k_quantv_pass2(const uint16_t *__restrict__ V, const int32_t *__restrict__ perm,

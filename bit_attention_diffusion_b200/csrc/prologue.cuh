@@ -68,7 +68,8 @@ struct FusedPrologueParams {
 __global__ void k_prologue_fused(const FusedPrologueParams p);
 
 constexpr int QUANTV1_SMEM = 128 * 272;              // gathered rows
-constexpr int QUANTV2_SMEM = 128 * 272 + 128 * 144;  // rows + transposed codes
+constexpr int QUANTV2_SMEM = 128 * 272 + 128 * 144;  // NVFP4 pass 2: rows + transposed codes
+constexpr int QUANTV2E_SMEM = 128 * 272;            // E4M3 pass 2: rows, then the codes in place
 constexpr int KMEANS8_SMEM = 2 * 128 * 272;  // double-buffered chunk rows
 constexpr int KMEANS8TC_STAGES = 3;   // chunk ring of k_kmeans_pass8tc
 constexpr int KM_THREADS = 512;       // k_kmeans_pass8tc: 16 warps, two blocks per SM

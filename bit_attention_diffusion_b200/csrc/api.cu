@@ -318,7 +318,10 @@ vc_status launch_cluster(const Shape &sh, const Ws &w, const uint16_t *V, int32_
                                             w.at<unsigned>(w.L.km_counter), it < sh.iters ? 1 : 0);
     count_launch();
   }
-  k_perm_sort<<<sh.BH, 1024, 0, s>>>(labels, sh.N, sh.k, perm);
+  if (sh.k <= 8 && sh.km_nblk <= PERM_SCATTER_MAX_BLOCKS)
+    k_perm_scatter<<<grid, 256, 0, s>>>(labels, w.at<int>(w.L.km_pcnt), sh.N, sh.k, sh.km_cpb, sh.km_nblk, perm);
+  else
+    k_perm_sort<<<sh.BH, 1024, 0, s>>>(labels, sh.N, sh.k, perm);
   count_launch();
   return VC_OK;
 }

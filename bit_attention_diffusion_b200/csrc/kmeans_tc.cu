@@ -35,7 +35,9 @@
 //               (lane j of the group is cluster j), four tokens per warp;
 //   warps 8-15  update passes: warp j lists the chunk's tokens labelled j
 //               and adds them, in fp64, four rows per step (lane l: channels
-//               4l .. 4l+3), then frees the stage.
+//               4l .. 4l+3), then frees the stage; in the label pass warp j
+//               counts them (the block's counts go to pcnt for the
+//               permutation's scatter).
 // No step waits for the whole block: a slow step (many fallback tokens, a
 // large cluster) holds its stage, and the others go on until the ring is
 // full. The last block of a (b,h) adds the blocks' partial sums in block order
@@ -417,6 +419,12 @@ __global__ void __launch_bounds__(KM_THREADS, 2) k_kmeans_pass8tc(const __grid_c
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc4[c] += B[c];
         __syncwarp();  // the list is rewritten for the next chunk
+      } else if (!accumulate && j < k) {
+        // the label pass: count the chunk's tokens of cluster j (the
+        // permutation's scatter places each block's tokens from these counts)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          cnt_own += __popc(__ballot_sync(0xFFFFFFFFu, 32 * q + lane < cnt && slab[s][32 * q + lane] == j));
       }
       __syncwarp();
       mbar_arrive(&bars.empty[s]);
@@ -435,7 +443,10 @@ __global__ void __launch_bounds__(KM_THREADS, 2) k_kmeans_pass8tc(const __grid_c
   }
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, 64);
-  if (!accumulate) return;
+  if (!accumulate) {
+    if (warp >= 8 && warp - 8 < k && lane == 0) pcnt[(static_cast<size_t>(bh) * nblk + blk) * k + warp - 8] = cnt_own;
+    return;
+  }
   double *ps = psum + (static_cast<size_t>(bh) * nblk + blk) * k * D;
   int *pc = pcnt + (static_cast<size_t>(bh) * nblk + blk) * k;
   if (warp >= 8 && warp - 8 < k) {

@@ -404,6 +404,75 @@ __global__ void __launch_bounds__(1024) k_perm_sort(const int32_t *__restrict__ 
   perm_sort_body<1024>(labels, N, k, perm, blockIdx.x, blockIdx.y, blockIdx.z);
 }
 
+// The same stable sort, spread over the k-means blocks of each (b,h) (k <= 8):
+// block b of the Lloyd pass counted its tokens per label (pcnt[bh][b][j], the
+// final label pass); label j's tokens of block b start at the tokens of the
+// labels below j plus label j's tokens in the blocks before b, and the block
+// scatters its own range [b cpb 128, (b+1) cpb 128) in rounds of 256 tokens.
+__global__ void __launch_bounds__(256) k_perm_scatter(const int32_t *__restrict__ labels,
+                                                      const int *__restrict__ pcnt, int N, int k, int cpb, int nblk,
+                                                      int32_t *__restrict__ perm) {
+  __shared__ int base[8], tot[8];
+  __shared__ int wcnt[8][8];
+  __shared__ int spc[PERM_SCATTER_MAX_BLOCKS * 8];  // the head's counts [block][label]
+  const int blk = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_begin = blk * cpb * TILE, n_end = min(N, n_begin + cpb * TILE);
+  const int32_t *lab = labels + static_cast<size_t>(bh) * N;
+  int32_t *out = perm + static_cast<size_t>(bh) * N;
+  const int *pc = pcnt + static_cast<size_t>(bh) * nblk * k;
+  for (int i = tid; i < nblk * k; i += 256) spc[i] = pc[i];
+  __syncthreads();
+  if (warp < k) {
+    // warp j: label j's tokens in all blocks (tot) and in the blocks before this one
+    int all = 0, before = 0;
+    for (int b = lane; b < nblk; b += 32) {
+      const int c = spc[b * k + warp];
+      all += c;
+      if (b < blk) before += c;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      all += __shfl_xor_sync(0xFFFFFFFFu, all, o);
+      before += __shfl_xor_sync(0xFFFFFFFFu, before, o);
+    }
+    if (lane == 0) {
+      tot[warp] = all;
+      base[warp] = before;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;  // tokens of the labels below j, all blocks
+    for (int j = 0; j < k; ++j) {
+      base[j] += run;
+      run += tot[j];
+    }
+  }
+  for (int n0 = n_begin; n0 < n_end; n0 += 256) {
+    if (tid < 64) (&wcnt[0][0])[tid] = 0;
+    __syncthreads();
+    const int n = n0 + tid;
+    const int L = n < n_end ? lab[n] : -1;
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, L);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (L >= 0 && rank == 0) wcnt[warp][L] = __popc(peers);
+    __syncthreads();
+    if (tid < k) {
+      int run = 0;
+      for (int w = 0; w < 8; ++w) {
+        const int c = wcnt[w][tid];
+        wcnt[w][tid] = run;
+        run += c;
+      }
+      tot[tid] = run;
+    }
+    __syncthreads();
+    if (L >= 0) out[base[L] + wcnt[warp][L] + rank] = n;
+    __syncthreads();
+    if (tid < k) base[tid] += tot[tid];
+  }
+}
+
 // ============================================================== streaming helpers
 // The HBM-bound kernels below move a 128-row tile with 256 threads: thread
 // (g, c) = (tid / 16, tid % 16) owns the 16-byte chunk c (channels 8c..8c+7)

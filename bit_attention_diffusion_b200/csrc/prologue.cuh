@@ -16,6 +16,12 @@ __global__ void k_kmeans_pass8tc(const __grid_constant__ CUtensorMap tmV, int N,
                                  int32_t *labels, double *psum, int *pcnt, unsigned *counter, int accumulate,
                                  uint32_t *status);
 __global__ void k_perm_sort(const int32_t *labels, int N, int k, int32_t *perm);
+// k <= 8: the stable sort spread over the k-means blocks, from the label
+// pass's per-block counts pcnt[bh][block][label].
+// At most PERM_SCATTER_MAX_BLOCKS k-means blocks per (b,h) (two per SM).
+constexpr int PERM_SCATTER_MAX_BLOCKS = 2 * 148;
+__global__ void k_perm_scatter(const int32_t *labels, const int *pcnt, int N, int k, int cpb, int nblk,
+                               int32_t *perm);
 __global__ void k_kbar(const uint16_t *K, int N, int nchunk, int ksmooth, double *part, unsigned *counter,
                        float *kbar);
 __global__ void k_qk_quant(const uint16_t *Q, const uint16_t *K, const int32_t *perm, const float *kbar, int N,

@@ -146,8 +146,9 @@ vc_status vc_attn_cluster(const void *V, int B, int H, int N, int d, const vc_pa
  *   blocks in all: 3.6 MB at k = 8 for up to 444 heads) and 256-byte-aligned
  *   counters. Shapes
  *   whose scratch exceeds 32 MiB (vc_attn_cluster_noalloc_max_bytes) return
- *   VC_ERR_WORKSPACE before any launch: about B*H*N <= 7.4 M tokens at k = 8
- *   (the 720p video workload, 3.0 M tokens, fits).
+ *   VC_ERR_WORKSPACE before any launch: about B*H*N <= 7.7 M tokens at k = 8
+ *   while B*H <= 296 (each head past that adds 8 KB of partial sums); the
+ *   720p video workload, 3.0 M tokens, fits.
  *   Set-up: the first call on each device looks up the array's device
  *   address (cudaGetSymbolAddress) with that device current; make that first
  *   call before any stream capture. cudaDeviceReset() ends the context that

@@ -34,10 +34,11 @@
 //   warps 2-3   the fallback list: the pinned chains, eight lanes per token
 //               (lane j of the group is cluster j), four tokens per warp;
 //   warps 8-15  update passes: warp j lists the chunk's tokens labelled j
-//               and adds them, in fp64, four rows per step (lane l: channels
-//               4l .. 4l+3), then frees the stage; in the label pass warp j
-//               counts them (the block's counts go to pcnt for the
-//               permutation's scatter).
+//               and j ^ 4 and adds, in fp64, the first half of the first
+//               list and the second half of the second, four rows per step
+//               (lane l: channels 4l .. 4l+3), then frees the stage; in the
+//               label pass warp j counts cluster j's tokens (the block's
+//               counts go to pcnt for the permutation's scatter).
 // No step waits for the whole block: a slow step (many fallback tokens, a
 // large cluster) holds its stage, and the others go on until the ring is
 // full. The last block of a (b,h) adds the blocks' partial sums in block order
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(KM_THREADS, 2) k_kmeans_pass8tc(const __grid_c
   __shared__ int8_t slab[KS][TILE];              // label of each token of the stage's chunk (-1: not yet)
   __shared__ uint8_t sfb[KS][4][32];             // fallback tokens, per label warp
   __shared__ int snfb[KS][4];
-  __shared__ __align__(16) uint8_t sidx[8][TILE];  // sum warp j: its cluster's tokens of the current chunk
+  __shared__ __align__(16) uint8_t sidx[8][2][TILE];  // sum warp j: the chunk's tokens of clusters j, j^4
   __shared__ int s_fail;
   __shared__ int s_last;
   __shared__ uint32_t s_tmem;
@@ -190,7 +191,8 @@ __global__ void __launch_bounds__(KM_THREADS, 2) k_kmeans_pass8tc(const __grid_c
   tc_fence_after();
   const uint32_t tmem = s_tmem;
 
-  double acc4[4] = {0.0, 0.0, 0.0, 0.0};
+  double acc4[4] = {0.0, 0.0, 0.0, 0.0};  // sum warps: cluster warp - 8 (its first halves)
+  double accB[4] = {0.0, 0.0, 0.0, 0.0};  // sum warps: cluster (warp - 8) ^ 4 (its second halves)
   int cnt_own = 0;  // tokens of cluster warp - 8 (sum warps)
   if (warp == 0) {
     // ---- TMA producer: chunk i into stage i % KS once chunk i - KS has left it
@@ -372,8 +374,35 @@ __global__ void __launch_bounds__(KM_THREADS, 2) k_kmeans_pass8tc(const __grid_c
       mbar_arrive(&bars.lab[s]);
     }
   } else {
-    // ---- sum warps: warp 8 + j adds the chunk's tokens labelled j
-    const int j = warp - 8;
+    // ---- sum warps: warp 8 + j adds the first half of the chunk's tokens
+    // labelled j and the second half of those labelled j ^ 4 (the halves split
+    // at a multiple of four), so a large cluster is shared by two warps
+    const int j = warp - 8, jb = j ^ 4;
+    // fp64 sums of list positions [from, to) (from a multiple of 4), four rows
+    // per step loaded together; the sums are exact, so the order does not
+    // change them
+    auto add_list = [&](const uint8_t *list, int from, int to, uint32_t sbuf, double (&acc)[4]) {
+      double o[4] = {0.0, 0.0, 0.0, 0.0};
+      for (int n = from; n < to; n += 4) {
+        const uint32_t t4 = *reinterpret_cast<const uint32_t *>(list + n);  // four listed tokens
+        uint2 w4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)  // (entries past the range are read, masked to a row of the chunk, dropped)
+          w4[u] = lds64_nc(sbuf + kt_off((t4 >> (8 * u)) & 0x7Fu, lane >> 1) + 8 * (lane & 1));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (n + u >= to) break;
+          double *a = (u & 1) ? o : acc;
+          a[0] += static_cast<double>(__uint_as_float(w4[u].x << 16));
+          a[1] += static_cast<double>(__uint_as_float(w4[u].x & 0xFFFF0000u));
+          a[2] += static_cast<double>(__uint_as_float(w4[u].y << 16));
+          a[3] += static_cast<double>(__uint_as_float(w4[u].y & 0xFFFF0000u));
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[c] += o[c];
+    };
+    auto split = [](int c) { return min(c, (((c + 1) >> 1) + 3) & ~3); };  // first-half length
     for (int i = 0; i < nchunk; ++i) {
       const int s = i % KS;
       const int n0 = n_begin + i * TILE, cnt = min(TILE, n_end - n0);
@@ -383,43 +412,27 @@ __global__ void __launch_bounds__(KM_THREADS, 2) k_kmeans_pass8tc(const __grid_c
         s_fail = 1;
         break;
       }
-      if (accumulate && j < k) {
-        // the chunk's tokens of cluster j, listed in token order
-        int cj = 0;
+      if (accumulate) {
+        // the chunk's tokens of clusters j and jb, each listed in token order
+        int ca = 0, cb = 0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const bool mine = 32 * q + lane < cnt && slab[s][32 * q + lane] == j;
-          const unsigned b = __ballot_sync(0xFFFFFFFFu, mine);
-          if (mine) sidx[j][cj + __popc(b & ((1u << lane) - 1u))] = static_cast<uint8_t>(32 * q + lane);
-          cj += __popc(b);
+          const int l = 32 * q + lane < cnt ? slab[s][32 * q + lane] : -1;
+          const unsigned ba = __ballot_sync(0xFFFFFFFFu, l == j), bb = __ballot_sync(0xFFFFFFFFu, l == jb);
+          const unsigned below = (1u << lane) - 1u;
+          if (l == j) sidx[j][0][ca + __popc(ba & below)] = static_cast<uint8_t>(32 * q + lane);
+          if (l == jb) sidx[j][1][cb + __popc(bb & below)] = static_cast<uint8_t>(32 * q + lane);
+          ca += __popc(ba);
+          cb += __popc(bb);
         }
         __syncwarp();
-        cnt_own += cj;
-        // fp64 sums of the listed tokens, four tokens per step (their rows
-        // loaded together), two accumulator sets (even and odd list
-        // positions) added at the end: exact, so the order does not change
-        // the sums
-        double B[4] = {0.0, 0.0, 0.0, 0.0};
-        for (int n = 0; n < cj; n += 4) {
-          const uint32_t t4 = *reinterpret_cast<const uint32_t *>(&sidx[j][n]);  // four listed tokens
-          uint2 w4[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u)  // (entries past the list are stale: masked to a row of the chunk, read, dropped)
-            w4[u] = lds64_nc(sbuf + kt_off((t4 >> (8 * u)) & 0x7Fu, lane >> 1) + 8 * (lane & 1));
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if (n + u >= cj) break;
-            double *acc = (u & 1) ? B : acc4;
-            acc[0] += static_cast<double>(__uint_as_float(w4[u].x << 16));
-            acc[1] += static_cast<double>(__uint_as_float(w4[u].x & 0xFFFF0000u));
-            acc[2] += static_cast<double>(__uint_as_float(w4[u].y << 16));
-            acc[3] += static_cast<double>(__uint_as_float(w4[u].y & 0xFFFF0000u));
-          }
+        if (j < k) {
+          cnt_own += ca;
+          add_list(sidx[j][0], 0, split(ca), sbuf, acc4);
         }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc4[c] += B[c];
-        __syncwarp();  // the list is rewritten for the next chunk
-      } else if (!accumulate && j < k) {
+        if (jb < k) add_list(sidx[j][1], split(cb), cb, sbuf, accB);
+        __syncwarp();  // the lists are rewritten for the next chunk
+      } else if (j < k) {
         // the label pass: count the chunk's tokens of cluster j (the
         // permutation's scatter places each block's tokens from these counts)
 #pragma unroll
@@ -447,10 +460,18 @@ __global__ void __launch_bounds__(KM_THREADS, 2) k_kmeans_pass8tc(const __grid_c
     if (warp >= 8 && warp - 8 < k && lane == 0) pcnt[(static_cast<size_t>(bh) * nblk + blk) * k + warp - 8] = cnt_own;
     return;
   }
+  // each cluster's second halves go to its own sum warp over the chunk ring,
+  // free now (every copy has landed and every read is done: barriers above)
+  double *hand = reinterpret_cast<double *>(dsm);  // [cluster][channel]
+  if (warp >= 8 && ((warp - 8) ^ 4) < k)
+    *reinterpret_cast<double4 *>(hand + ((warp - 8) ^ 4) * D + 4 * lane) = make_double4(accB[0], accB[1], accB[2], accB[3]);
+  __syncthreads();
   double *ps = psum + (static_cast<size_t>(bh) * nblk + blk) * k * D;
   int *pc = pcnt + (static_cast<size_t>(bh) * nblk + blk) * k;
   if (warp >= 8 && warp - 8 < k) {
-    *reinterpret_cast<double4 *>(ps + (warp - 8) * D + 4 * lane) = make_double4(acc4[0], acc4[1], acc4[2], acc4[3]);
+    const double4 h = *reinterpret_cast<const double4 *>(hand + (warp - 8) * D + 4 * lane);
+    *reinterpret_cast<double4 *>(ps + (warp - 8) * D + 4 * lane) =
+        make_double4(acc4[0] + h.x, acc4[1] + h.y, acc4[2] + h.z, acc4[3] + h.w);
     if (lane == 0) pc[warp - 8] = cnt_own;
   }
   __threadfence();

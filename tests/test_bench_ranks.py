@@ -46,3 +46,29 @@ def test_two_gloo_ranks_take_the_slowest_time_and_count_both_replicas():
 def test_single_rank_is_the_identity():
     assert bench.max_over_ranks(1.5, 1) == 1.5
     assert bench.job_tflops(1, 4.0e12, 2.0) == pytest.approx(2000.0)
+
+
+def test_reference_arm_prints_the_contract_line_with_the_gpu_arms_config():
+    """The reference arm (the oracle on the host cores) on a small workload:
+    one JSON line with impl=reference, the same config dict the GPU arm
+    prints, the cpu_baseline description of this run and an e2e entry with no
+    host-device traffic."""
+    import json
+    import subprocess
+    import sys
+
+    from bit_attention_diffusion_b200 import synth
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3", "--workload", "tiny_b1h2n1024"],
+                       capture_output=True, text=True, timeout=300, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    wl, _ = synth.make_by_name("tiny_b1h2n1024")
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.bench_config(wl, "e4m3", 1)
+    assert line["unit"] == "TFLOPS" and line["higher_is_better"] is True and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["cores"] >= 1 and "head" in line["cpu_baseline"]["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert line["steps"] == 1 and line["warmup"] == 3 and line["n_gpus"] == 1

@@ -140,3 +140,21 @@ def test_vsmooth_schedule_clusters_in_the_first_quarter(L):
     assert sched.last_cluster_step == 4
     sched._perm = object()   # as after a first clustering
     assert [sched.clusters_at(s) for s in range(7)] == [True] * 5 + [False] * 2
+
+
+def test_noalloc_cluster_rejects_bad_arguments_on_host(L):
+    """The allocation-free clustering entry point checks its arguments, and
+    that the clustering scratch fits its fixed array, before touching a
+    device."""
+    p = vcattn.params()
+    ok = (FAKE, 1, 2, 1024, 128, p, FAKE, FAKE, None)
+    assert vcattn.vc_attn_cluster_noalloc_max_bytes() == 32 << 20
+    for i, bad in ((0, None), (6, None), (7, None), (0, FAKE + 8), (6, FAKE + 4)):
+        args = list(ok)
+        args[i] = bad
+        assert vcattn.vc_attn_cluster_noalloc(*args) == vcattn.VC_ERR_INVALID_ARG, (i, bad)
+    assert vcattn.vc_attn_cluster_noalloc(FAKE, 1, 2, 1024, 64, p, FAKE, FAKE, None) == vcattn.VC_ERR_UNSUPPORTED
+    assert vcattn.vc_attn_cluster_noalloc(FAKE, 1, 2, 1024, 128, vcattn.params(k=0), FAKE, FAKE, None) == \
+        vcattn.VC_ERR_INVALID_ARG
+    # about 7.8 M tokens fit at k = 8; 8.4 M do not
+    assert vcattn.vc_attn_cluster_noalloc(FAKE, 4, 64, 32768, 128, p, FAKE, FAKE, None) == vcattn.VC_ERR_WORKSPACE
